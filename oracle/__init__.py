@@ -1,0 +1,234 @@
+"""CPU oracle for the MixLLM mixed-precision quantized linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product path (the C-ABI library and its Python binding) never
+imports, links or runs it, and the two share no code.
+
+The arithmetic lives in ``mx_oracle.c`` (plain C, single thread, exact int64 and
+fp64 after the fp32 quantization decisions).  This module only compiles it with
+gcc and marshals numpy arrays through ctypes.  Every function cites the passage
+of the MixLLM paper digest it follows (see the C file for the full list).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mx_oracle.c")
+_LIB = os.path.join(_HERE, "libmx_oracle.so")
+_CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE fp32/fp64, no contraction); return the .so path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *_CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    lib.mxo_fp16_round.argtypes = [ctypes.c_double]
+    lib.mxo_fp16_round.restype = ctypes.c_double
+    lib.mxo_fp16_bits_of.argtypes = [ctypes.c_double]
+    lib.mxo_fp16_bits_of.restype = ctypes.c_uint16
+    lib.mxo_fp16_value.argtypes = [ctypes.c_uint16]
+    lib.mxo_fp16_value.restype = ctypes.c_double
+    lib.mxo_quant_sym8.argtypes = [P, I, P, P]
+    lib.mxo_quant_sym8.restype = None
+    lib.mxo_quant_asym4.argtypes = [P, I, P, P, P]
+    lib.mxo_quant_asym4.restype = None
+    lib.mxo_quant_act.argtypes = [P, I, I, I, I, P, P]
+    lib.mxo_quant_act.restype = I
+    lib.mxo_pack.argtypes = [P, I, I, I, I, P, P, P, P, P, P, P]
+    lib.mxo_pack.restype = I
+    lib.mxo_partials.argtypes = [P, I, I, I, I, P, I, P, P, P, P]
+    lib.mxo_partials.restype = ctypes.c_int64
+    lib.mxo_gemm.argtypes = [P, P, I, I, I, I, I, P, I, P, P, P, P, P, P, P, ctypes.c_long, P, P]
+    lib.mxo_gemm.restype = I
+    _lib = lib
+    return lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+# ----------------------------------------------------------------- fp16 helpers
+def fp16_round(v: float) -> float:
+    """Nearest IEEE binary16 value (ties to even), overflow to inf."""
+    return _load().mxo_fp16_round(float(v))
+
+
+def fp16_bits(v: float) -> int:
+    """Bit pattern of an exactly representable binary16 value."""
+    return int(_load().mxo_fp16_bits_of(float(v)))
+
+
+def fp16_value(bits: int) -> float:
+    return _load().mxo_fp16_value(int(bits) & 0xFFFF)
+
+
+def fp16_values(bits: np.ndarray) -> np.ndarray:
+    """Vector form of fp16_value (loop over the C routine; for small arrays)."""
+    lib = _load()
+    flat = np.asarray(bits, dtype=np.uint16).ravel()
+    out = np.array([lib.mxo_fp16_value(int(b)) for b in flat], dtype=np.float64)
+    return out.reshape(np.shape(bits))
+
+
+# ----------------------------------------------------------------- quantizers
+def quant_sym8(x) -> tuple[np.ndarray, int]:
+    """Symmetric 8-bit quantizer of one group (MixLLM section 2.1; range +-127)."""
+    x = _f32(x).ravel()
+    q = np.zeros(x.size, np.int8)
+    s = np.zeros(1, np.uint16)
+    _load().mxo_quant_sym8(_p(x), x.size, _p(q), _p(s))
+    return q, int(s[0])
+
+
+def quant_asym4(x) -> tuple[np.ndarray, int, int]:
+    """Asymmetric 4-bit quantizer of one group (MixLLM section 2.1 affine form)."""
+    x = _f32(x).ravel()
+    q = np.zeros(x.size, np.uint8)
+    z = np.zeros(1, np.uint8)
+    s = np.zeros(1, np.uint16)
+    _load().mxo_quant_asym4(_p(x), x.size, _p(q), _p(z), _p(s))
+    return q, int(z[0]), int(s[0])
+
+
+def quant_act(X, act_group: int = 0) -> tuple[np.ndarray, np.ndarray]:
+    """8-bit symmetric activation quantization (MixLLM section 3.1.2).
+
+    act_group == 0: one fp16 scale per token, s_a shape [M].
+    act_group == g: one scale per (token, group of g columns), shape [M, K/g].
+    Returns (Aq int8 [M, K], s_a fp16 bits uint16).
+    """
+    X = _f32(X)
+    M, K = X.shape
+    na = 1 if act_group == 0 else K // act_group
+    Aq = np.zeros((M, K), np.int8)
+    sa = np.zeros((M, na), np.uint16)
+    rc = _load().mxo_quant_act(_p(X), M, K, K, act_group, _p(Aq), _p(sa))
+    if rc != 0:
+        raise ValueError("mxo_quant_act: bad arguments")
+    return Aq, (sa[:, 0].copy() if act_group == 0 else sa)
+
+
+@dataclass
+class Canonical:
+    """Canonical packed form: the compare target for the GPU blob."""
+    N: int
+    K: int
+    group: int
+    n8: int
+    perm: np.ndarray      # int32 [N]: packed row -> original row
+    codes8: np.ndarray    # int8  [n8, K]
+    scales8: np.ndarray   # uint16 fp16 bits [n8, G]
+    codes4: np.ndarray    # uint8 [N-n8, K], one code per byte
+    zeros4: np.ndarray    # uint8 [N-n8, G]
+    scales4: np.ndarray   # uint16 fp16 bits [N-n8, G]
+
+    @property
+    def G(self) -> int:
+        return self.K // self.group
+
+
+def pack(W, is8, group: int) -> Canonical:
+    """Row split + permutation + per-group quantization (MixLLM sections 3.1.1, 2.1)."""
+    W = _f32(W)
+    N, K = W.shape
+    is8 = np.ascontiguousarray(is8, dtype=np.uint8)
+    assert is8.shape == (N,)
+    G = K // group
+    n8 = int((is8 != 0).sum())
+    perm = np.zeros(N, np.int32)
+    c8 = np.zeros((n8, K), np.int8)
+    s8 = np.zeros((n8, G), np.uint16)
+    c4 = np.zeros((N - n8, K), np.uint8)
+    z4 = np.zeros((N - n8, G), np.uint8)
+    s4 = np.zeros((N - n8, G), np.uint16)
+    rc = _load().mxo_pack(_p(W), N, K, K, group, _p(is8), _p(perm), _p(c8), _p(s8),
+                          _p(c4), _p(z4), _p(s4))
+    if rc != n8:
+        raise ValueError("mxo_pack: bad arguments")
+    return Canonical(N, K, group, n8, perm, c8, s8, c4, z4, s4)
+
+
+def partials(Aq: np.ndarray, c: Canonical) -> tuple[np.ndarray, int]:
+    """int64 P[m, n, g] in original row order (MixLLM section 3.3 step one)."""
+    Aq = np.ascontiguousarray(Aq, dtype=np.int8)
+    M = Aq.shape[0]
+    P = np.zeros((M, c.N, c.G), np.int64)
+    pmax = _load().mxo_partials(_p(Aq), M, c.K, c.group, c.N, _p(c.perm), c.n8,
+                                _p(c.codes8), _p(c.codes4), _p(c.zeros4), _p(P))
+    if pmax < 0:
+        raise ValueError("mxo_partials: bad arguments")
+    return P, int(pmax)
+
+
+def gemm(Aq: np.ndarray, s_a: np.ndarray, c: Canonical, act_group: int = 0,
+         pairs: tuple[np.ndarray, np.ndarray] | None = None) -> tuple[np.ndarray, np.ndarray]:
+    """fp64 Y two ways (plain definition, two-step form of MixLLM section 3.3).
+
+    pairs=None: all outputs, shape [M, N].  pairs=(m_idx, n_idx): those entries only
+    (n in original row order), shape [len(m_idx)].
+    """
+    Aq = np.ascontiguousarray(Aq, dtype=np.int8)
+    s_a = np.ascontiguousarray(s_a, dtype=np.uint16)
+    M = Aq.shape[0]
+    if pairs is None:
+        pm = pn = None
+        cnt = M * c.N
+        shape = (M, c.N)
+    else:
+        pm = np.ascontiguousarray(pairs[0], dtype=np.int32)
+        pn = np.ascontiguousarray(pairs[1], dtype=np.int32)
+        cnt = pm.size
+        shape = (cnt,)
+    yd = np.zeros(cnt, np.float64)
+    yt = np.zeros(cnt, np.float64)
+    rc = _load().mxo_gemm(_p(Aq), _p(s_a), act_group, M, c.K, c.group, c.N, _p(c.perm), c.n8,
+                          _p(c.codes8), _p(c.scales8), _p(c.codes4), _p(c.zeros4), _p(c.scales4),
+                          None if pm is None else _p(pm), None if pn is None else _p(pn),
+                          cnt, _p(yd), _p(yt))
+    if rc != 0:
+        raise ValueError("mxo_gemm: bad arguments")
+    return yd.reshape(shape), yt.reshape(shape)
+
+
+def dequant_weights(c: Canonical) -> np.ndarray:
+    """Dequantized W' [N, K] (fp64, original row order): (W_q - z) s_w (section 2.1)."""
+    G, g = c.G, c.group
+    W = np.zeros((c.N, c.K), np.float64)
+    s8 = fp16_values(c.scales8) if c.n8 else np.zeros((0, G))
+    s4 = fp16_values(c.scales4) if c.N - c.n8 else np.zeros((0, G))
+    for j in range(c.N):
+        n = int(c.perm[j])
+        if j < c.n8:
+            w = c.codes8[j].astype(np.float64)
+            W[n] = w * np.repeat(s8[j], g)
+        else:
+            r = j - c.n8
+            w = c.codes4[r].astype(np.float64) - np.repeat(c.zeros4[r].astype(np.float64), g)
+            W[n] = w * np.repeat(s4[r], g)
+    return W

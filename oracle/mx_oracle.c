@@ -1,0 +1,325 @@
+/*
+ * mx_oracle.c -- plain, slow, single-threaded CPU oracle for the MixLLM
+ * mixed-precision quantized linear layer (W4.4A8).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark use it.  It shares no code, header, table or helper with the
+ * CUDA library; both sides are written independently from the method's text.
+ *
+ * Sources (MixLLM: "LLM Quantization with Global Mixed-precision between
+ * Output-features and Highly-efficient System Design", paper digest page):
+ *   - affine quantizer  X_q = clamp(round(X/s) + z, range), X' = (X_q - z) s
+ *       (section 2.1, "quantization principle")
+ *   - symmetric quantizer X_q = clamp(round(W/s), range), X' = X_q s
+ *       (section 2.1, "quantization scheme")
+ *   - 8-bit symmetric activations, 8-bit symmetric / 4-bit asymmetric
+ *     group-wise weights, group 128 (section 3.1.2; section 4 setup)
+ *   - output-feature mixed precision: every output row is an independent
+ *     sub-problem, results gathered into one Y (section 3.1.1, Figure 1)
+ *   - two-step dequantization: (W_q - z) times A_q on integers per group,
+ *     then both scales per group (section 3.3); W_q, z are uint4, s_w, s_a
+ *     are float16 (section 3.3)
+ *   - restricted symmetric range +-(2^(b-1) - 1) (SBVR page, section 2.1)
+ *
+ * Readings where the text is silent (each one is listed in the design notes):
+ *   R1 symmetric range [-127, 127], s = absmax / 127
+ *   R3 the 4-bit range [lo, hi] always contains 0, so z fits uint4
+ *   R4 round() is round-half-to-even
+ *   R5 scales are computed in fp32, rounded to fp16 (nearest-even) and the
+ *      ROUNDED fp16 value is the one used to quantize
+ *   R7 a zero (or fp16-underflowed) scale becomes 1.0; an fp16 overflow
+ *      saturates to 65504
+ *   R10 fp32 quantization decisions: amax/127, (hi-lo)/15, x/s, -lo/s are
+ *      each one IEEE fp32 operation; everything after the integer codes is
+ *      exact integer (int64) or fp64 arithmetic here
+ *
+ * Parity of every function below is pinned by CPU tests against closed
+ * forms, brute force, textbook special cases and library conversions.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC
+ * (x86-64 evaluates float in SSE single precision, FLT_EVAL_METHOD == 0).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#if defined(__FLT_EVAL_METHOD__) && __FLT_EVAL_METHOD__ != 0
+#error "the oracle needs IEEE single-precision evaluation of float expressions"
+#endif
+
+/* ------------------------------------------------------------------------ */
+/* IEEE-754 binary16 rounding, written from the format's definition:        */
+/* 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits; normal numbers  */
+/* have exponents -14..15, subnormals a fixed quantum of 2^-24; the largest */
+/* finite value is 65504; round-to-nearest, ties-to-even.                   */
+/* ------------------------------------------------------------------------ */
+
+/* nearest binary16 value of v, as a double (exact); overflow gives +-inf */
+double mxo_fp16_round(double v)
+{
+    if (v != v) return v;
+    double a = fabs(v);
+    if (a == 0.0) return v;
+    int e;
+    frexp(a, &e);                 /* a in [2^(e-1), 2^e) */
+    int E = e - 1;                /* unbiased exponent of a */
+    if (E < -14) E = -14;         /* subnormal binade: quantum stays 2^-24 */
+    double quantum = ldexp(1.0, E - 10);
+    double r = rint(a / quantum) * quantum;   /* a/quantum is exact */
+    if (r >= 65536.0) r = INFINITY;           /* beyond 65504 + half ulp */
+    return copysign(r, v);
+}
+
+/* bit pattern of a value that is already exactly representable in binary16 */
+uint16_t mxo_fp16_bits_of(double r)
+{
+    uint16_t sign = signbit(r) ? 0x8000u : 0u;
+    double a = fabs(r);
+    if (a != a) return 0x7E00u;
+    if (isinf(a)) return (uint16_t)(sign | 0x7C00u);
+    if (a == 0.0) return sign;
+    if (a < ldexp(1.0, -14)) {                       /* subnormal */
+        return (uint16_t)(sign | (uint16_t)(a / ldexp(1.0, -24)));
+    }
+    int e;
+    double f = frexp(a, &e);                         /* a = f 2^e, f in [0.5,1) */
+    int E = e - 1;
+    uint16_t frac = (uint16_t)((f * 2.0 - 1.0) * 1024.0);
+    return (uint16_t)(sign | (uint16_t)((E + 15) << 10) | frac);
+}
+
+/* value of a binary16 bit pattern */
+double mxo_fp16_value(uint16_t h)
+{
+    int s = (h >> 15) & 1, E = (h >> 10) & 31, f = h & 1023;
+    double v;
+    if (E == 31) v = f ? NAN : INFINITY;
+    else if (E == 0) v = ldexp((double)f, -24);
+    else v = ldexp(1024.0 + f, E - 25);
+    return s ? -v : v;
+}
+
+/* R5/R7: the fp16 scale actually used by the quantizers */
+static float scale_to_fp16(float s32, uint16_t *bits)
+{
+    double s16 = mxo_fp16_round((double)s32);
+    if (s16 > 65504.0) s16 = 65504.0;          /* R7 saturation */
+    if (s16 == 0.0) s16 = 1.0;                 /* R7 degenerate group */
+    *bits = mxo_fp16_bits_of(s16);
+    return (float)s16;                         /* exact */
+}
+
+static float clampf_(float v, float lo, float hi)
+{
+    return v < lo ? lo : (v > hi ? hi : v);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Symmetric 8-bit quantizer (section 2.1 "quantization scheme", range      */
+/* +-127 by R1): s = fp16(absmax/127), q = clamp(round(x/s), -127, 127).    */
+/* ------------------------------------------------------------------------ */
+void mxo_quant_sym8(const float *x, int n, int8_t *q, uint16_t *s_bits)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    float s = scale_to_fp16(amax / 127.0f, s_bits);
+    for (int i = 0; i < n; ++i) {
+        float r = rintf(x[i] / s);
+        q[i] = (int8_t)clampf_(r, -127.0f, 127.0f);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Asymmetric 4-bit quantizer (section 2.1 affine form; z is uint4 per      */
+/* section 3.3, so the range includes 0 by R3):                              */
+/*   lo = min(0, min x), hi = max(0, max x), s = fp16((hi - lo)/15),         */
+/*   z = clamp(round(-lo/s), 0, 15), q = clamp(round(x/s) + z, 0, 15).       */
+/* ------------------------------------------------------------------------ */
+void mxo_quant_asym4(const float *x, int n, uint8_t *q, uint8_t *z, uint16_t *s_bits)
+{
+    float lo = 0.0f, hi = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        if (x[i] < lo) lo = x[i];
+        if (x[i] > hi) hi = x[i];
+    }
+    float range = hi - lo;
+    float s = scale_to_fp16(range / 15.0f, s_bits);
+    float zf = clampf_(rintf(-lo / s), 0.0f, 15.0f);
+    *z = (uint8_t)zf;
+    for (int i = 0; i < n; ++i) {
+        float r = rintf(x[i] / s) + zf;
+        q[i] = (uint8_t)clampf_(r, 0.0f, 15.0f);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Activation quantization: 8-bit symmetric per token (act_group == 0) or   */
+/* per group of act_group columns (section 3.1.2 reading, see R2).          */
+/* X: [M][ldx] fp32.  Aq: [M][K] int8.  s_a: [M] (per token) or [M][K/ag].  */
+/* Returns 0, or -1 on bad arguments.                                       */
+/* ------------------------------------------------------------------------ */
+int mxo_quant_act(const float *X, int M, int K, int ldx, int act_group,
+                  int8_t *Aq, uint16_t *s_a)
+{
+    if (M < 0 || K <= 0 || ldx < K) return -1;
+    int ag = act_group == 0 ? K : act_group;
+    if (ag <= 0 || K % ag) return -1;
+    int na = K / ag;
+    for (int m = 0; m < M; ++m)
+        for (int j = 0; j < na; ++j)
+            mxo_quant_sym8(X + (size_t)m * ldx + (size_t)j * ag, ag,
+                           Aq + (size_t)m * K + (size_t)j * ag, s_a + (size_t)m * na + j);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Packing into the CANONICAL form (the compare target of the GPU blob):    */
+/*   perm[N]           packed row j -> original row; the 8-bit rows first   */
+/*                     in ascending original index, then the 4-bit rows in  */
+/*                     ascending original index (section 3.1.1, Figure 1:   */
+/*                     independent sub-problems, gathered afterwards)       */
+/*   codes8[N8][K]     int8, scales8[N8][G] fp16 bits                        */
+/*   codes4[N4][K]     uint8 (one code per byte), zeros4[N4][G] uint8,      */
+/*                     scales4[N4][G] fp16 bits                              */
+/* W: [N][ldw] fp32; is8[N]: nonzero = salient row kept at 8 bits.          */
+/* Returns N8 (>= 0), or -1 on bad arguments.                               */
+/* ------------------------------------------------------------------------ */
+int mxo_pack(const float *W, int N, int K, int ldw, int group, const uint8_t *is8,
+             int32_t *perm, int8_t *codes8, uint16_t *scales8,
+             uint8_t *codes4, uint8_t *zeros4, uint16_t *scales4)
+{
+    if (N < 0 || K <= 0 || ldw < K || group <= 0 || K % group) return -1;
+    int G = K / group;
+    int n8 = 0;
+    for (int n = 0; n < N; ++n) if (is8[n]) perm[n8++] = n;
+    int j = n8;
+    for (int n = 0; n < N; ++n) if (!is8[n]) perm[j++] = n;
+    for (int r = 0; r < n8; ++r) {
+        const float *w = W + (size_t)perm[r] * ldw;
+        for (int g = 0; g < G; ++g)
+            mxo_quant_sym8(w + (size_t)g * group, group,
+                           codes8 + (size_t)r * K + (size_t)g * group,
+                           scales8 + (size_t)r * G + g);
+    }
+    for (int r = 0; r < N - n8; ++r) {
+        const float *w = W + (size_t)perm[n8 + r] * ldw;
+        for (int g = 0; g < G; ++g)
+            mxo_quant_asym4(w + (size_t)g * group, group,
+                            codes4 + (size_t)r * K + (size_t)g * group,
+                            zeros4 + (size_t)r * G + g,
+                            scales4 + (size_t)r * G + g);
+    }
+    return n8;
+}
+
+/* packed index of every original row (inverse of perm) */
+static int32_t *invert_perm(const int32_t *perm, int N)
+{
+    int32_t *inv = (int32_t *)malloc(sizeof(int32_t) * (size_t)(N > 0 ? N : 1));
+    if (!inv) return NULL;
+    for (int j = 0; j < N; ++j) inv[perm[j]] = j;
+    return inv;
+}
+
+/* integer weight (W_q - z) of packed row j at column k: the first step of  */
+/* the two-step dequantization (section 3.3); z = 0 for the 8-bit rows       */
+static int wint(int j, int k, int K, int group, int n8, const int8_t *codes8,
+                const uint8_t *codes4, const uint8_t *zeros4)
+{
+    if (j < n8) return (int)codes8[(size_t)j * K + k];
+    int r = j - n8, G = K / group;
+    return (int)codes4[(size_t)r * K + k] - (int)zeros4[(size_t)r * G + k / group];
+}
+
+static double wscale(int j, int g, int G, int n8, const uint16_t *scales8,
+                     const uint16_t *scales4)
+{
+    if (j < n8) return mxo_fp16_value(scales8[(size_t)j * G + g]);
+    return mxo_fp16_value(scales4[(size_t)(j - n8) * G + g]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Per-group integer partials (section 3.3 step one):                        */
+/*   P[m][n][g] = sum_{k in group g} Aq[m][k] * (W_q[n][k] - z[n][g])        */
+/* in int64, n in ORIGINAL row order.  Returns the largest |P| seen, or -1.  */
+/* ------------------------------------------------------------------------ */
+int64_t mxo_partials(const int8_t *Aq, int M, int K, int group, int N,
+                     const int32_t *perm, int n8,
+                     const int8_t *codes8, const uint8_t *codes4, const uint8_t *zeros4,
+                     int64_t *P)
+{
+    if (M < 0 || K <= 0 || group <= 0 || K % group || N < 0) return -1;
+    int G = K / group;
+    int32_t *inv = invert_perm(perm, N);
+    if (!inv) return -1;
+    int64_t pmax = 0;
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) {
+            int j = inv[n];
+            for (int g = 0; g < G; ++g) {
+                int64_t acc = 0;
+                for (int k = g * group; k < (g + 1) * group; ++k)
+                    acc += (int64_t)Aq[(size_t)m * K + k] *
+                           (int64_t)wint(j, k, K, group, n8, codes8, codes4, zeros4);
+                P[((size_t)m * N + n) * G + g] = acc;
+                if (llabs(acc) > pmax) pmax = llabs(acc);
+            }
+        }
+    free(inv);
+    return pmax;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Y = dequant(Xq) . dequant(Wq)^T, fp64, at the listed (m, n) pairs        */
+/* (n in original row order), two ways that must agree:                     */
+/*  Y_def: the plain definition, sum_k (Aq s_a)[m][k] * ((W_q - z) s_w)[n][k]*/
+/*         (section 2.1 dequantization applied to both operands)            */
+/*  Y_two: the two-step form of section 3.3,                                */
+/*         sum_g s_a[m][g] s_w[n][g] P[m][n][g]  (s_a per token when        */
+/*         act_group == 0)                                                  */
+/* pairs == NULL means every (m, n), written row-major [M][N].              */
+/* Returns 0, or -1 on bad arguments.                                       */
+/* ------------------------------------------------------------------------ */
+int mxo_gemm(const int8_t *Aq, const uint16_t *s_a, int act_group, int M, int K,
+             int group, int N, const int32_t *perm, int n8,
+             const int8_t *codes8, const uint16_t *scales8,
+             const uint8_t *codes4, const uint8_t *zeros4, const uint16_t *scales4,
+             const int32_t *pair_m, const int32_t *pair_n, long n_pairs,
+             double *Y_def, double *Y_two)
+{
+    if (M < 0 || K <= 0 || group <= 0 || K % group || N < 0) return -1;
+    if (act_group != 0 && act_group != group) return -1;
+    int G = K / group;
+    int na = act_group == 0 ? 1 : G;
+    int32_t *inv = invert_perm(perm, N);
+    if (!inv) return -1;
+    long total = pair_m ? n_pairs : (long)M * N;
+    for (long t = 0; t < total; ++t) {
+        int m = pair_m ? pair_m[t] : (int)(t / (N > 0 ? N : 1));
+        int n = pair_m ? pair_n[t] : (int)(t % (N > 0 ? N : 1));
+        if (m < 0 || m >= M || n < 0 || n >= N) { free(inv); return -1; }
+        int j = inv[n];
+        double ydef = 0.0, ytwo = 0.0;
+        for (int g = 0; g < G; ++g) {
+            double sa = mxo_fp16_value(s_a[(size_t)m * na + (na == 1 ? 0 : g)]);
+            double sw = wscale(j, g, G, n8, scales8, scales4);
+            int64_t p = 0;
+            for (int k = g * group; k < (g + 1) * group; ++k) {
+                int a = Aq[(size_t)m * K + k];
+                int w = wint(j, k, K, group, n8, codes8, codes4, zeros4);
+                ydef += ((double)a * sa) * ((double)w * sw);
+                p += (int64_t)a * (int64_t)w;
+            }
+            ytwo += sa * sw * (double)p;
+        }
+        Y_def[t] = ydef;
+        Y_two[t] = ytwo;
+    }
+    free(inv);
+    return 0;
+}
