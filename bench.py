@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Benchmark of the MixLLM mixed-precision quantized linear layer on B200.
+
+One step = the run-time hot path over one batch of synthetic tokens:
+quantize the activations (per-token 8-bit symmetric) and run the mixed W8/W4
+GEMM with two-step dequantization and scatter into Y.  Weight packing is the
+method's offline step (weights are pre-packed once, MixLLM section 3.3) and is
+done before timing; its own throughput is reported under "pack".
+
+Timing: inputs live in HBM before the timed region; each step uses the next of R
+rotated copies of the packed weights, activations and outputs, with R chosen so
+that the bytes touched between two uses of one copy exceed 4x the L2 size.  The
+K timed steps are replayed from CUDA graphs, bracketed by a barrier and device
+synchronisation, timed with CUDA events and max-reduced over ranks.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+       python bench.py --impl reference ...   (the CPU oracle on the same workload)
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mixed W4.4A8 GEMM TOPS and GB/s, % of INT8 TC peak / HBM roofline"
+
+WORKLOADS = {
+    # name: (M, K, N) -- Llama 3 layer shapes, 10% 8-bit rows, group 128
+    "llama3-8b-qo-m1": (1, 4096, 4096),
+    "llama3-8b-qo-m16": (16, 4096, 4096),
+    "llama3-8b-up-m256": (256, 4096, 14336),
+    "llama3-8b-up-m2048": (2048, 4096, 14336),
+    "llama3-8b-down-m2048": (2048, 14336, 4096),
+    "llama3-70b-up-m1": (1, 8192, 28672),
+    "llama3-70b-down-m1": (1, 28672, 8192),
+    "llama3-70b-up-m4096": (4096, 8192, 28672),
+    "llama3-70b-down-m4096": (4096, 28672, 8192),
+}
+DEFAULT_WORKLOAD = "llama3-8b-qo-m1"
+HBM_BOUND_MAX_M = 128        # below the ~150-token ridge the step is bound by HBM
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=0, help="timed steps (0: about one second of work)")
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    p.add_argument("--frac8", type=float, default=0.10)
+    p.add_argument("--group", type=int, default=128)
+    p.add_argument("--path", type=int, default=0, help="0 auto, 1 split-K CUDA cores, 2 tensor cores")
+    p.add_argument("--impl", default="mx", choices=["mx", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--seed", type=int, default=0)
+    a = p.parse_args()
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    return a
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def src_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mixed_precision_quantized_mx_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------------ clocks (NVML)
+class ClockSampler:
+    """Samples SM clock and clock-event reasons of one GPU every few ms."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = str(e)
+        self.samples = []
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def start(self):
+        if self.ok:
+            self._stop.clear()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self, t0=None, t1=None):
+        if not self.ok:
+            return {"error": self.err}
+        s = [x for x in self.samples if (t0 is None or x[0] >= t0) and (t1 is None or x[0] <= t1)]
+        if not s:
+            return None
+        mhz = [x[1] for x in s]
+        bits = 0
+        for x in s:
+            bits |= x[2]
+        reasons = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": reasons, "samples": len(s)}
+
+
+# ------------------------------------------------------------------ reference arm
+def oracle_step_sample(lay, budget_s: float = 0.5):
+    """A bounded sample of one step for the CPU oracle: which (m, n) outputs to compute."""
+    M, N, K = lay.M, lay.N, lay.K
+    per_pair = K * 12e-9                     # ~12 ns per MAC pair on one core (both forms)
+    budget = max(64, int(budget_s / per_pair))
+    if M * N <= budget:
+        m = np.repeat(np.arange(M, dtype=np.int32), N)
+        n = np.tile(np.arange(N, dtype=np.int32), M)
+        return m, n, f"all {M}x{N} outputs"
+    rng = np.random.default_rng(1)
+    m = rng.integers(0, M, budget).astype(np.int32)
+    n = rng.integers(0, N, budget).astype(np.int32)
+    return m, n, f"{budget} random (token, row) outputs of {M}x{N}"
+
+
+def time_oracle(lay, canonical, steps: int, min_seconds: float = 0.0):
+    """Run the oracle's quantize + sampled GEMM; return (seconds per step, sample, fraction)."""
+    import oracle
+    m, n, desc = oracle_step_sample(lay)
+    frac = len(m) / (lay.M * lay.N)
+    X = lay.X.astype(np.float32)
+    done, t0 = 0, time.perf_counter()
+    while done < steps or time.perf_counter() - t0 < min_seconds:
+        Aq, sa = oracle.quant_act(X)
+        oracle.gemm(Aq, sa, canonical, pairs=(m, n))
+        done += 1
+    return (time.perf_counter() - t0) / done, desc, frac, done
+
+
+def step_units(M, K, N, g, n8, unit):
+    from mixed_precision_quantized_mx_b200 import model
+    if unit == "GB/s":
+        return model.step_bytes(M, N, K, g, n8, 2) / 1e9
+    return model.gemm_ops(M, N, K) / 1e12
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from mixed_precision_quantized_mx_b200 import inputs
+    import oracle
+    M, K, N = WORKLOADS[a.workload]
+    lay = inputs.llama_layer(M, K, N, a.frac8, a.group, seed=a.seed)
+    can = oracle.pack(lay.W, lay.is8, lay.group)
+    unit = "GB/s" if M <= HBM_BOUND_MAX_M else "TOPS"
+    time_oracle(lay, can, a.warmup)
+    sec, desc, frac, done = time_oracle(lay, can, a.steps or 5)
+    value = step_units(M, K, N, a.group, lay.n8, unit) * frac / sec
+    sample = f"each step: quantize {M}x{K} activations + {desc} (fraction {frac:.3g} of the step)"
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "impl": "reference",
+        "n_gpus": a.gpus, "steps": done, "warmup": a.warmup, "ms_per_step": sec * 1e3 / frac,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": a.workload, "M": M, "K": K, "N": N, "group": a.group,
+                   "frac8": a.frac8, "n8": lay.n8},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main arm
+def main():
+    a = parse()
+    if a.impl == "reference":
+        return run_reference(a)
+
+    import torch
+    import torch.distributed as dist
+    from mixed_precision_quantized_mx_b200 import binding as mx
+    from mixed_precision_quantized_mx_b200 import build as mxbuild
+    from mixed_precision_quantized_mx_b200 import inputs, model
+    from mixed_precision_quantized_mx_b200.layer import MixedPrecisionLinear
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    mxbuild.build()
+    mx.lib()
+
+    M, K, N = WORKLOADS[a.workload]
+    g = a.group
+    lay = inputs.llama_layer(M, K, N, a.frac8, g, seed=a.seed + rank)   # each rank its own batch
+    n8 = lay.n8
+    L = mx.mx_layout_init(N, K, g, n8)
+    unit = "GB/s" if M <= HBM_BOUND_MAX_M else "TOPS"
+    bound = "hbm" if unit == "GB/s" else "tensor"
+
+    # ---- pack once (offline step), timed on its own
+    Wd = torch.from_numpy(lay.W).to(dev)
+    is8d = torch.from_numpy(lay.is8).to(dev)
+    blob0 = torch.empty(L.total_bytes, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    mx.mx_pack_weights(L, Wd, is8d, blob0, status=status)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise SystemExit("packer reported an error")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        mx.mx_pack_weights(L, Wd, is8d, blob0)
+    e1.record()
+    torch.cuda.synchronize()
+    pack_ms = e0.elapsed_time(e1) / 3
+    del Wd
+
+    # ---- rotated copies beyond L2
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per_step = model.step_bytes(M, N, K, g, n8, 2)
+    R = int(min(64, max(2, math.ceil(4 * l2 / per_step))))
+    R = max(2, min(R, int(20e9 // max(per_step, 1))))
+    Xh = torch.from_numpy(lay.X)
+    Xs = [Xh.to(dev) for _ in range(R)]
+    blobs = [blob0] + [blob0.clone() for _ in range(R - 1)]
+    Aqs = [torch.empty((M, K), dtype=torch.int8, device=dev) for _ in range(R)]
+    sas = [torch.empty((M,), dtype=torch.float16, device=dev) for _ in range(R)]
+    Ys = [torch.empty((M, N), dtype=torch.float16, device=dev) for _ in range(R)]
+    ws_bytes = mx.mx_gemm_workspace_size(L, M, path=a.path)
+    ws = torch.empty(max(16, ws_bytes), dtype=torch.uint8, device=dev)
+    path_used = mx.mx_gemm_select_path(L, M, path=a.path)
+
+    def step(i):
+        mx.mx_quant_act(Xs[i], Aqs[i], sas[i])
+        mx.mx_gemm(L, blobs[i], Aqs[i], sas[i], Ys[i], workspace=ws, path=a.path)
+
+    def gemm_only(i):
+        mx.mx_gemm(L, blobs[i], Aqs[i], sas[i], Ys[i], workspace=ws, path=a.path)
+
+    s = torch.cuda.Stream(dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        for i in range(R):          # eager pass: configures kernels before capture
+            step(i)
+    torch.cuda.synchronize()
+
+    def capture(fn, count, start=0):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=s):
+            for j in range(count):
+                fn((start + j) % R)
+        return gr
+
+    g_full = capture(step, R)
+    # estimate step time to size the default K (about one second of timed work)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(3):
+        g_full.replay()
+    torch.cuda.synchronize()
+    est = (time.perf_counter() - t0) / (3 * R)
+    K_steps = a.steps or int(min(200000, max(50, 1.0 / max(est, 1e-7))))
+    q, rem = divmod(K_steps, R)
+    g_rem = capture(step, rem) if rem else None
+    qw, rw = divmod(a.warmup, R)
+    g_wrem = capture(step, rw) if rw else None
+
+    def replay_steps(nfull, grem):
+        for _ in range(nfull):
+            g_full.replay()
+        if grem is not None:
+            grem.replay()
+
+    sampler = ClockSampler(local)
+    # sustained run of the same step graph (clock reference even for short timed regions)
+    sampler.start()
+    t_load0 = time.perf_counter()
+    while time.perf_counter() - t_load0 < 0.6:
+        g_full.replay()
+    torch.cuda.synchronize()
+    t_load1 = time.perf_counter()
+
+    replay_steps(qw, g_wrem)                       # W warm-up steps
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_time0 = time.perf_counter()
+    ev0.record(s)
+    with torch.cuda.stream(s):
+        replay_steps(q, g_rem)
+    ev1.record(s)
+    torch.cuda.synchronize()
+    t_time1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    units_per_step = step_units(M, K, N, g, n8, unit)
+    value = units_per_step * K_steps * world / (ms / 1e3)
+
+    # ---- dominant kernel: the GEMM call alone, timed live on its stream
+    nd = max(R, min(4 * R, 400))
+    g_gemm = capture(gemm_only, nd)
+    g_gemm.replay()
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(s)
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            g_gemm.replay()
+    d1.record(s)
+    torch.cuda.synchronize()
+    gemm_ms = d0.elapsed_time(d1) / (3 * nd)
+    peaks = load_peaks()
+    if bound == "hbm":
+        algo = model.gemm_bytes(M, N, K, g, n8)
+        achieved = algo / (gemm_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        r_unit = "GB/s"
+    else:
+        algo = model.gemm_ops(M, N, K)
+        achieved = algo / (gemm_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"] * 2.0    # dense int8 = 2x dense bf16 (nominal 4.5 / 2.25 PF)
+        r_unit = "TOPS"
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if os.path.exists(tfile):
+        rec = json.load(open(tfile)).get(a.workload)
+        if rec and rec.get("src_digest") == src_digest() and rec.get("path") == path_used:
+            traffic = rec["dram_bytes_per_launch"]
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "mx_gemm (split-K + reduce)" if path_used == 1 else "mx_gemm (tcgen05)",
+                "algorithmic_per_launch": algo, "launch_ms": gemm_ms,
+                "peak_source": (f"{peaks['source']} HBM copy" if bound == "hbm" else
+                                f"{peaks['source']} bf16 cuBLAS burst x 2 (nominal int8/bf16 ratio)")}
+
+    # ---- end to end through the public API: pinned host X in, host Y out
+    layer = MixedPrecisionLinear.from_blob(blob0)
+    Xpin = Xh.pin_memory()
+    Ypin = torch.empty((M, N), dtype=torch.float16).pin_memory()
+    Xdev = torch.empty_like(Xs[0])
+    Ke = max(20, min(K_steps, 2000))
+    for _ in range(3):
+        Xdev.copy_(Xpin, non_blocking=True)
+        Ypin.copy_(layer(Xdev, path=a.path), non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(Ke):
+        Xdev.copy_(Xpin, non_blocking=True)
+        Ypin.copy_(layer(Xdev, path=a.path), non_blocking=True)
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / Ke
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": units_per_step * world / (e2e_ms / 1e3), "unit": unit,
+           "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+           "ms_per_step": e2e_ms, "api": "MixedPrecisionLinear.forward (eager, per-call launches)"}
+
+    clocks = sampler.summary(t_time0, t_time1) or sampler.summary(t_load0, t_load1)
+    if clocks is not None and "error" not in clocks:
+        clocks["window"] = ("timed region" if sampler.summary(t_time0, t_time1)
+                            else "sustained replay of the same step graph just before the timed region")
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        import oracle
+        can = oracle.pack(lay.W, lay.is8, g)
+        sec, desc, frac, done = time_oracle(lay, can, 1, min_seconds=10.0)
+        cpu = {"value": units_per_step * frac / sec, "unit": unit, "cores": 1, "kind": "oracle",
+               "sample": f"{done} steps, each: quantize {M}x{K} activations + {desc}"}
+
+    kernels_per_step = 1 + (2 if path_used == 1 else 1)
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K_steps,
+        "warmup": a.warmup, "ms_per_step": ms / K_steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": a.workload, "M": M, "K": K, "N": N, "group": g, "frac8": a.frac8,
+                   "n8": n8, "path": path_used,
+                   "l2": f"inputs rotate over {R} copies ({R * per_step / 1e6:.0f} MB >= 4x the "
+                         f"{l2 / 1e6:.0f} MB L2); no flush",
+                   "graphs": "timed steps replayed from CUDA graphs"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": kernels_per_step * K_steps, "clocks": clocks,
+        "tops": model.gemm_ops(M, N, K) * K_steps * world / (ms / 1e3) / 1e12,
+        "gbs": model.step_bytes(M, N, K, g, n8, 2) * K_steps * world / (ms / 1e3) / 1e9,
+        "pack": {"ms": pack_ms, "weights_gb_per_s": (N * K * 4) / (pack_ms / 1e3) / 1e9},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g_full, g_rem, g_wrem, g_gemm
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

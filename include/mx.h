@@ -1,0 +1,200 @@
+/*
+ * mx.h -- C ABI of the B200 (sm_100a) MixLLM mixed-precision quantized linear layer.
+ *
+ * The method (MixLLM: "LLM Quantization with Global Mixed-precision between
+ * Output-features and Highly-efficient System Design"):
+ *   - output features (rows of W [N, K]) are split by saliency into 8-bit
+ *     symmetric rows and 4-bit asymmetric rows, each quantized group-wise along
+ *     K (group 64 or 128) with fp16 scales (section 3.1.1, Figure 1;
+ *     section 3.1.2; section 2.1 for the two quantizer formulas);
+ *   - activations X [M, K] are quantized to 8-bit symmetric codes, one fp16
+ *     scale per token (section 3.1.2);
+ *   - Y = dequant(Xq) dequant(Wq)^T is computed by two-step dequantization:
+ *     int8 products of A_q and (W_q - z) summed per group into int32, then
+ *     both scales applied per group in fp32 (section 3.3); the two row sets
+ *     are independent sub-problems whose outputs are scattered back into one
+ *     Y by the epilogue (section 3.3, "parallel execution of sub-problems").
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer named "device" is caller-owned device memory (for example
+ *     a torch tensor).  The library never allocates device memory and keeps no
+ *     device state between calls.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All device work is enqueued asynchronously on it.
+ *   - Argument errors are detected on the host BEFORE anything is enqueued and
+ *     returned as an mx_status; mx_last_error() then holds a one-line message
+ *     for the calling thread.  Errors found by a kernel while it runs are
+ *     written to the optional device `status` word (0 = ok) and never trap.
+ *   - fp16 values cross the boundary as uint16_t bit patterns (IEEE binary16).
+ *   - Device pointers must be 16-byte aligned; leading dimensions are in
+ *     elements and must keep every row 16-byte aligned.
+ */
+#ifndef MX_H
+#define MX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MX_ABI_VERSION 1
+
+typedef enum mx_status {
+    MX_OK = 0,
+    MX_ERR_INVALID_ARG = 1,   /* null/negative/inconsistent argument */
+    MX_ERR_UNSUPPORTED = 2,   /* valid for the method, not supported by this build */
+    MX_ERR_ALIGNMENT = 3,     /* pointer or leading dimension not 16-byte aligned */
+    MX_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (message says which) */
+    MX_ERR_TIMEOUT = 5,       /* device status only: a bounded wait gave up */
+    MX_ERR_BAD_BLOB = 6,      /* packed-weight header does not match the layout */
+    MX_ERR_WORKSPACE = 7      /* workspace missing or smaller than required */
+} mx_status;
+
+typedef enum mx_dtype { MX_F32 = 0, MX_F16 = 1 } mx_dtype;
+
+/* Rows per packed row tile and K columns per packed k-block. */
+#define MX_TILE_ROWS 128
+#define MX_KBLOCK 128
+#define MX_HEADER_BYTES 256
+#define MX_BLOB_MAGIC 0x4B50584Du /* "MXPK" */
+
+/*
+ * Geometry of one packed layer.  Filled by mx_layout_init (or read back from a
+ * blob header by mx_layout_from_header); treated as read-only afterwards.
+ *
+ * Packed blob (one device buffer, `total_bytes` long, every section 256-byte
+ * aligned, offsets from the blob start):
+ *   header   [256 B]   magic, version, N, K, group, n8 (see mx_layout_from_header)
+ *   rowmap   int32 [(t8 + t4) * 128]   packed slot -> original row of W, -1 for
+ *                      padding.  Slots 0 .. 128*t8-1 hold the 8-bit rows in
+ *                      ascending original index; slots from 128*t8 on hold the
+ *                      4-bit rows in ascending original index.
+ *   scales8  fp16  [t8][G][128]        scale of (row tile, group, row in tile)
+ *   codes8   int8  [t8][K/128][128 x 128 B]  one 16 KB block per (tile, k-block):
+ *                      row r's 128 codes occupy bytes r*128 .. r*128+127, and
+ *                      the 16-byte chunk holding k = 16c .. 16c+15 sits at chunk
+ *                      position (c XOR (r mod 8)) -- the 128-byte swizzle that
+ *                      the tensor-core shared-memory operand layout expects.
+ *   scales4  fp16  [t4][G][128]
+ *   zeros4   uint8 [t4][G][128]        zero point z in 0..15 (one byte each)
+ *   codes4   uint8 [t4][K/128][128 x 64 B]   one 8 KB block per (tile, k-block):
+ *                      row r's 64 bytes at r*64; the 32-bit word w (0..15) of a
+ *                      row holds k = 8w .. 8w+7: byte b has k = 8w+b in its low
+ *                      nibble and k = 8w+4+b in its high nibble.
+ * Padding rows have zero codes, zero scales and zero zero-points.
+ */
+typedef struct mx_layout {
+    int32_t N, K, group, n8;   /* problem: W is [N, K]; n8 rows at 8 bits */
+    int32_t n4, G;             /* N - n8, K / group */
+    int32_t t8, t4;            /* row tiles of 128 in each part (ceil) */
+    int32_t kblocks;           /* K / 128 */
+    int32_t reserved0;
+    uint64_t off_rowmap, off_scales8, off_codes8, off_scales4, off_zeros4, off_codes4;
+    uint64_t total_bytes;
+} mx_layout;
+
+/* Options of mx_gemm; pass NULL for the defaults (all fields zero). */
+typedef struct mx_gemm_opts {
+    int32_t path;              /* 0 auto; 1 split-K CUDA-core path; 2 tensor-core path */
+    int32_t split;             /* split-K factor for 4-bit tiles (0 = auto); path 1 */
+    int32_t* debug_partials;   /* device int32 [M][N][G] or NULL: every per-group
+                                  int32 partial P[m][n][g] (original row order) */
+    int32_t* status;           /* device int32 or NULL: kernel-side error code */
+} mx_gemm_opts;
+
+/* ABI version of the loaded library (MX_ABI_VERSION). */
+int mx_version(void);
+
+/* One-line description of the calling thread's last error ("" if none). */
+const char* mx_last_error(void);
+
+/*
+ * mx_layout_init -- host only, no device work.  Computes the packed geometry
+ * and the blob size of a layer with W [N, K], group size `group` and `n8`
+ * 8-bit rows (the rest 4-bit).
+ * Constraints: N >= 1, 0 <= n8 <= N, group in {64, 128}, K a positive multiple
+ * of 128 (the k-block of the packed layout).  Groups of 64/128 columns follow
+ * the MixLLM experimental setting (group 128) and keep every group's int8 dot
+ * product inside the fast int-to-float window (section 3.3).
+ * Returns MX_ERR_INVALID_ARG / MX_ERR_UNSUPPORTED otherwise.
+ */
+mx_status mx_layout_init(int N, int K, int group, int n8, mx_layout* out);
+
+/*
+ * mx_layout_from_header -- host only.  Validates a copy of a blob's first
+ * MX_HEADER_BYTES bytes (copied to host memory by the caller) and rebuilds its
+ * layout.  Returns MX_ERR_BAD_BLOB if the magic, version or geometry is wrong.
+ */
+mx_status mx_layout_from_header(const void* host_header, size_t bytes, mx_layout* out);
+
+/*
+ * mx_pack_weights -- offline weight packing (MixLLM section 3.3: the weight
+ * layout is pre-packed so that no permutation happens at run time; section
+ * 3.1.1: the 8-bit and 4-bit rows form separate sub-problems).
+ *   W       device [N][ldw] fp32 or fp16 (wdtype), row-major, ldw >= K
+ *   is8     device uint8 [N], nonzero = the row is salient and stays 8-bit;
+ *           exactly L->n8 entries must be nonzero
+ *   blob    device, L->total_bytes bytes, written completely
+ *   status  device int32 or NULL; set to MX_ERR_INVALID_ARG if the mask does
+ *           not hold exactly n8 ones (the blob is then unusable)
+ * 8-bit rows: s = fp16(absmax/127) (zero scale -> 1, fp16 overflow saturates),
+ *   q = clamp(round_half_even(w / s), -127, 127)        (section 2.1, symmetric)
+ * 4-bit rows: lo = min(0, min w), hi = max(0, max w), s = fp16((hi - lo)/15),
+ *   z = clamp(round(-lo / s), 0, 15), q = clamp(round(w / s) + z, 0, 15)
+ *                                                       (section 2.1, affine)
+ * Every fp32 step is one IEEE operation (no contraction, true division).
+ */
+mx_status mx_pack_weights(const mx_layout* L, const void* W, mx_dtype wdtype, int64_t ldw,
+                          const uint8_t* is8, void* blob, int32_t* status, void* stream);
+
+/*
+ * mx_quant_act -- per-token 8-bit symmetric activation quantization
+ * (MixLLM section 3.1.2; quantizer of section 2.1, range +-127).
+ *   X    device [M][ldx] fp32 or fp16 (xdtype), ldx >= K
+ *   Aq   device int8 [M][K] (dense, row stride K)
+ *   s_a  device fp16 bits [M]: s_a = fp16(max_k |X[m,k]| / 127), 0 -> 1
+ *   Aq[m,k] = clamp(round_half_even(X[m,k] / s_a[m]), -127, 127)
+ * M = 0 is a no-op.  K must be a positive multiple of 8.
+ */
+mx_status mx_quant_act(const void* X, mx_dtype xdtype, int M, int K, int64_t ldx,
+                       int8_t* Aq, uint16_t* s_a, void* stream);
+
+/*
+ * mx_gemm_workspace_size -- host only.  Bytes of device workspace mx_gemm
+ * needs for this layer at M tokens with these options (0 if none).
+ */
+mx_status mx_gemm_workspace_size(const mx_layout* L, int M, const mx_gemm_opts* opts,
+                                 size_t* bytes);
+
+/*
+ * mx_gemm_select_path -- host only.  The GEMM path mx_gemm will take for this
+ * layer at M tokens with these options: 1 = split-K CUDA-core path (decode-sized
+ * M, HBM-bound), 2 = tensor-core path.  Negative mx_status on bad arguments.
+ */
+int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts);
+
+/*
+ * mx_gemm -- Y = dequant(Aq, s_a) . dequant(W_packed)^T  (MixLLM section 3.3).
+ *   L       host layout of the blob (mx_layout_init / mx_layout_from_header)
+ *   blob    device, produced by mx_pack_weights for the same layout
+ *   Aq      device int8 [M][K] row-major (dense); s_a device fp16 bits [M]
+ *   Y       device fp16 [M][ldy], ldy >= N; column n is original row n of W
+ *   workspace / ws_bytes: device scratch of at least
+ *           mx_gemm_workspace_size(L, M, opts) bytes (may be NULL if 0)
+ * Per group g: P = sum_{k in g} Aq[m,k] (W_q[n,k] - z[n,g]) exactly in int32
+ * (|P| <= 127*127*128 < 2^22), acc[m,n] = sum_g float(P) * s_w[n,g] in fp32,
+ * then Y[m,n] = fp16_rn(acc * s_a[m]).  The fp32 summation order depends on the
+ * path and split but is fixed for a given configuration (deterministic).
+ * M = 0 is a no-op; M <= 65535.
+ */
+mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const uint16_t* s_a,
+                  int M, uint16_t* Y, int64_t ldy, void* workspace, size_t ws_bytes,
+                  const mx_gemm_opts* opts, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MX_H */

@@ -1,0 +1,173 @@
+"""Thin ctypes binding of the C ABI in include/mx.h.
+
+Argument marshalling only: every function forwards torch tensors' device
+pointers, sizes and the current CUDA stream to the function of the same name in
+libmx.so.  There is no host-side computation and no fallback: if the library is
+missing, or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmx.so")
+
+MX_OK = 0
+STATUS_NAMES = {
+    0: "MX_OK", 1: "MX_ERR_INVALID_ARG", 2: "MX_ERR_UNSUPPORTED", 3: "MX_ERR_ALIGNMENT",
+    4: "MX_ERR_CUDA", 5: "MX_ERR_TIMEOUT", 6: "MX_ERR_BAD_BLOB", 7: "MX_ERR_WORKSPACE",
+}
+MX_F32, MX_F16 = 0, 1
+TILE_ROWS, KBLOCK, HEADER_BYTES = 128, 128, 256
+PATH_AUTO, PATH_SPLITK, PATH_TENSOR = 0, 1, 2
+
+EXPORTED = ("mx_version", "mx_last_error", "mx_layout_init", "mx_layout_from_header",
+            "mx_pack_weights", "mx_quant_act", "mx_gemm_workspace_size", "mx_gemm_select_path",
+            "mx_gemm")
+
+
+class MXError(RuntimeError):
+    def __init__(self, status: int, fn: str, msg: str):
+        super().__init__(f"{fn}: {STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Layout(ctypes.Structure):
+    """mirror of mx_layout"""
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("N", "K", "group", "n8", "n4", "G", "t8", "t4", "kblocks", "reserved0")] + \
+               [(n, ctypes.c_uint64) for n in
+                ("off_rowmap", "off_scales8", "off_codes8", "off_scales4", "off_zeros4",
+                 "off_codes4", "total_bytes")]
+
+
+class GemmOpts(ctypes.Structure):
+    """mirror of mx_gemm_opts"""
+    _fields_ = [("path", ctypes.c_int32), ("split", ctypes.c_int32),
+                ("debug_partials", ctypes.c_void_p), ("status", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmx.so (built in-tree); raise if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m mixed_precision_quantized_mx_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, I64, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    L.mx_version.restype = I
+    L.mx_last_error.restype = ctypes.c_char_p
+    L.mx_layout_init.argtypes = [I, I, I, I, ctypes.POINTER(Layout)]
+    L.mx_layout_from_header.argtypes = [P, Z, ctypes.POINTER(Layout)]
+    L.mx_pack_weights.argtypes = [ctypes.POINTER(Layout), P, I, I64, P, P, P, P]
+    L.mx_quant_act.argtypes = [P, I, I, I, I64, P, P, P]
+    L.mx_gemm_workspace_size.argtypes = [ctypes.POINTER(Layout), I, ctypes.POINTER(GemmOpts),
+                                         ctypes.POINTER(Z)]
+    L.mx_gemm_select_path.argtypes = [ctypes.POINTER(Layout), I, ctypes.POINTER(GemmOpts)]
+    L.mx_gemm_select_path.restype = I
+    L.mx_gemm.argtypes = [ctypes.POINTER(Layout), P, P, P, I, P, I64, P, Z,
+                          ctypes.POINTER(GemmOpts), P]
+    for n in ("mx_layout_init", "mx_layout_from_header", "mx_pack_weights", "mx_quant_act",
+              "mx_gemm_workspace_size", "mx_gemm"):
+        getattr(L, n).restype = I
+    _lib = L
+    return L
+
+
+def _check(st: int, fn: str):
+    if st != MX_OK:
+        raise MXError(st, fn, lib().mx_last_error().decode())
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return MX_F16
+    if t.dtype == torch.float32:
+        return MX_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _opts(path=0, split=0, debug_partials=None, status=None) -> GemmOpts:
+    return GemmOpts(path, split, _ptr(debug_partials), _ptr(status))
+
+
+# ------------------------------------------------------------------ entry points
+def mx_version() -> int:
+    return lib().mx_version()
+
+
+def mx_layout_init(N: int, K: int, group: int, n8: int) -> Layout:
+    L = Layout()
+    _check(lib().mx_layout_init(N, K, group, n8, ctypes.byref(L)), "mx_layout_init")
+    return L
+
+
+def mx_layout_from_header(header) -> Layout:
+    """header: bytes, or a host uint8 tensor holding the blob's first 256 bytes."""
+    if isinstance(header, torch.Tensor):
+        header = bytes(header[:HEADER_BYTES].cpu().numpy().tobytes())
+    buf = ctypes.create_string_buffer(bytes(header), len(header))
+    L = Layout()
+    _check(lib().mx_layout_from_header(buf, len(header), ctypes.byref(L)), "mx_layout_from_header")
+    return L
+
+
+def mx_pack_weights(L: Layout, W: torch.Tensor, is8: torch.Tensor, blob: torch.Tensor,
+                    status: torch.Tensor | None = None, stream=None) -> None:
+    assert W.dim() == 2 and W.stride(1) == 1
+    _check(lib().mx_pack_weights(ctypes.byref(L), _ptr(W), _dtype_code(W), W.stride(0), _ptr(is8),
+                                 _ptr(blob), _ptr(status), _stream(stream)), "mx_pack_weights")
+
+
+def mx_quant_act(X: torch.Tensor, Aq: torch.Tensor, s_a: torch.Tensor, stream=None) -> None:
+    assert X.dim() == 2 and X.stride(1) == 1
+    M, K = X.shape
+    _check(lib().mx_quant_act(_ptr(X), _dtype_code(X), M, K, X.stride(0), _ptr(Aq), _ptr(s_a),
+                              _stream(stream)), "mx_quant_act")
+
+
+def mx_gemm_workspace_size(L: Layout, M: int, path: int = 0, split: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    o = _opts(path, split)
+    _check(lib().mx_gemm_workspace_size(ctypes.byref(L), M, ctypes.byref(o), ctypes.byref(n)),
+           "mx_gemm_workspace_size")
+    return n.value
+
+
+def mx_gemm_select_path(L: Layout, M: int, path: int = 0, split: int = 0) -> int:
+    o = _opts(path, split)
+    r = lib().mx_gemm_select_path(ctypes.byref(L), M, ctypes.byref(o))
+    if r < 0:
+        _check(-r, "mx_gemm_select_path")
+    return r
+
+
+def mx_gemm(L: Layout, blob: torch.Tensor, Aq: torch.Tensor, s_a: torch.Tensor, Y: torch.Tensor,
+            workspace: torch.Tensor | None = None, path: int = 0, split: int = 0,
+            debug_partials: torch.Tensor | None = None, status: torch.Tensor | None = None,
+            stream=None) -> None:
+    M = Aq.shape[0]
+    o = _opts(path, split, debug_partials, status)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().mx_gemm(ctypes.byref(L), _ptr(blob), _ptr(Aq), _ptr(s_a), M, _ptr(Y), Y.stride(0),
+                         _ptr(workspace), ws_bytes, ctypes.byref(o), _stream(stream)), "mx_gemm")

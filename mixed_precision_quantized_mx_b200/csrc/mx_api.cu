@@ -1,0 +1,222 @@
+// mx_api.cu -- the extern "C" boundary: argument validation, packed-layout
+// geometry, workspace sizing and dispatch between the two GEMM paths.
+// Nothing here computes on the host beyond sizes; every step of the method
+// runs in the kernels of the other translation units.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "mx_internal.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+mx_status fail(mx_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+mx_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(MX_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+uint64_t align256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Device (or managed) memory that kernels may dereference; host pointers are
+// rejected so that nothing ever runs through a host-side data path.
+mx_status check_device_ptr(const void* p, const char* name) {
+    if (p == nullptr) return fail(MX_ERR_INVALID_ARG, "%s is NULL", name);
+    cudaPointerAttributes at;
+    cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MX_ERR_INVALID_ARG, "%s: not a CUDA pointer (%s)", name, cudaGetErrorString(e));
+    }
+    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
+        return fail(MX_ERR_INVALID_ARG, "%s is not device memory", name);
+    return MX_OK;
+}
+
+mx_status check_layout(const mx_layout* L) {
+    if (L == nullptr) return fail(MX_ERR_INVALID_ARG, "layout is NULL");
+    mx_layout ref;
+    mx_status st = mx_layout_init(L->N, L->K, L->group, L->n8, &ref);
+    if (st != MX_OK) return st;
+    if (memcmp(&ref, L, sizeof ref) != 0)
+        return fail(MX_ERR_INVALID_ARG, "layout was modified after mx_layout_init");
+    return MX_OK;
+}
+
+}  // namespace
+
+namespace mx {
+
+Geom make_geom(const mx_layout& L, const void* blob) {
+    const uint8_t* b = static_cast<const uint8_t*>(blob);
+    Geom g;
+    g.blob = b;
+    g.rowmap = reinterpret_cast<const int32_t*>(b + L.off_rowmap);
+    g.scales8 = reinterpret_cast<const __half*>(b + L.off_scales8);
+    g.codes8 = reinterpret_cast<const int8_t*>(b + L.off_codes8);
+    g.scales4 = reinterpret_cast<const __half*>(b + L.off_scales4);
+    g.zeros4 = b + L.off_zeros4;
+    g.codes4 = b + L.off_codes4;
+    g.N = L.N; g.K = L.K; g.group = L.group; g.G = L.G; g.n8 = L.n8;
+    g.t8 = L.t8; g.t4 = L.t4; g.kblocks = L.kblocks;
+    return g;
+}
+
+}  // namespace mx
+
+extern "C" {
+
+int mx_version(void) { return MX_ABI_VERSION; }
+
+const char* mx_last_error(void) { return g_err.c_str(); }
+
+mx_status mx_layout_init(int N, int K, int group, int n8, mx_layout* out) {
+    if (out == nullptr) return fail(MX_ERR_INVALID_ARG, "out is NULL");
+    if (N < 1 || K < 1) return fail(MX_ERR_INVALID_ARG, "N=%d K=%d must be positive", N, K);
+    if (n8 < 0 || n8 > N) return fail(MX_ERR_INVALID_ARG, "n8=%d outside [0, N=%d]", n8, N);
+    if (group != 64 && group != 128)
+        return fail(MX_ERR_UNSUPPORTED, "group=%d: supported group sizes are 64 and 128", group);
+    if (K % MX_KBLOCK != 0)
+        return fail(MX_ERR_UNSUPPORTED, "K=%d must be a multiple of %d", K, MX_KBLOCK);
+    mx_layout L;
+    memset(&L, 0, sizeof L);
+    L.N = N; L.K = K; L.group = group; L.n8 = n8;
+    L.n4 = N - n8;
+    L.G = K / group;
+    L.t8 = (n8 + MX_TILE_ROWS - 1) / MX_TILE_ROWS;
+    L.t4 = (L.n4 + MX_TILE_ROWS - 1) / MX_TILE_ROWS;
+    L.kblocks = K / MX_KBLOCK;
+    const uint64_t rows8 = uint64_t(L.t8) * MX_TILE_ROWS, rows4 = uint64_t(L.t4) * MX_TILE_ROWS;
+    uint64_t off = MX_HEADER_BYTES;
+    L.off_rowmap = off;  off = align256(off + (rows8 + rows4) * 4);
+    L.off_scales8 = off; off = align256(off + rows8 * L.G * 2);
+    L.off_codes8 = off;  off = align256(off + rows8 * K);
+    L.off_scales4 = off; off = align256(off + rows4 * L.G * 2);
+    L.off_zeros4 = off;  off = align256(off + rows4 * L.G);
+    L.off_codes4 = off;  off = align256(off + rows4 * K / 2);
+    L.total_bytes = off;
+    *out = L;
+    return MX_OK;
+}
+
+mx_status mx_layout_from_header(const void* host_header, size_t bytes, mx_layout* out) {
+    if (host_header == nullptr || out == nullptr)
+        return fail(MX_ERR_INVALID_ARG, "header or out is NULL");
+    if (bytes < MX_HEADER_BYTES) return fail(MX_ERR_BAD_BLOB, "header shorter than %d bytes", MX_HEADER_BYTES);
+    uint32_t h[6];
+    memcpy(h, host_header, sizeof h);
+    if (h[0] != MX_BLOB_MAGIC) return fail(MX_ERR_BAD_BLOB, "bad magic 0x%08x", h[0]);
+    if (h[1] != MX_ABI_VERSION) return fail(MX_ERR_BAD_BLOB, "blob version %u != %d", h[1], MX_ABI_VERSION);
+    mx_status st = mx_layout_init(int(h[2]), int(h[3]), int(h[4]), int(h[5]), out);
+    if (st != MX_OK) return fail(MX_ERR_BAD_BLOB, "header geometry invalid: %s", g_err.c_str());
+    return MX_OK;
+}
+
+mx_status mx_pack_weights(const mx_layout* L, const void* W, mx_dtype wdtype, int64_t ldw,
+                          const uint8_t* is8, void* blob, int32_t* status, void* stream) {
+    mx_status st = check_layout(L);
+    if (st != MX_OK) return st;
+    if (wdtype != MX_F32 && wdtype != MX_F16) return fail(MX_ERR_INVALID_ARG, "bad wdtype %d", int(wdtype));
+    if (ldw < L->K) return fail(MX_ERR_INVALID_ARG, "ldw=%lld < K=%d", (long long)ldw, L->K);
+    if ((st = check_device_ptr(W, "W")) != MX_OK) return st;
+    if ((st = check_device_ptr(is8, "is8")) != MX_OK) return st;
+    if ((st = check_device_ptr(blob, "blob")) != MX_OK) return st;
+    if (status && (st = check_device_ptr(status, "status")) != MX_OK) return st;
+    if (!aligned16(blob)) return fail(MX_ERR_ALIGNMENT, "blob must be 16-byte aligned");
+    cudaError_t e = mx::launch_pack(*L, W, wdtype, ldw, is8, blob, status,
+                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+    return MX_OK;
+}
+
+mx_status mx_quant_act(const void* X, mx_dtype xdtype, int M, int K, int64_t ldx,
+                       int8_t* Aq, uint16_t* s_a, void* stream) {
+    if (xdtype != MX_F32 && xdtype != MX_F16) return fail(MX_ERR_INVALID_ARG, "bad xdtype %d", int(xdtype));
+    if (M < 0 || K < 1) return fail(MX_ERR_INVALID_ARG, "M=%d K=%d", M, K);
+    if (K % 8 != 0) return fail(MX_ERR_UNSUPPORTED, "K=%d must be a multiple of 8", K);
+    if (ldx < K) return fail(MX_ERR_INVALID_ARG, "ldx=%lld < K=%d", (long long)ldx, K);
+    if (M == 0) return MX_OK;
+    mx_status st;
+    if ((st = check_device_ptr(X, "X")) != MX_OK) return st;
+    if ((st = check_device_ptr(Aq, "Aq")) != MX_OK) return st;
+    if ((st = check_device_ptr(s_a, "s_a")) != MX_OK) return st;
+    const int esz = xdtype == MX_F16 ? 2 : 4;
+    if (!aligned16(X) || (ldx * esz) % 16 != 0 || !aligned16(Aq))
+        return fail(MX_ERR_ALIGNMENT, "X, Aq and every X row must be 16-byte aligned");
+    cudaError_t e = mx::launch_quant_act(X, xdtype, M, K, ldx, Aq, s_a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "quant_act launch");
+    return MX_OK;
+}
+
+static int choose_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
+    (void)L;
+    if (opts && opts->path) return opts->path;
+    (void)M;
+    return 1;   // the tensor-core path is selected here once it is built
+}
+
+int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
+    mx_status st = check_layout(L);
+    if (st != MX_OK) return -int(st);
+    if (M < 0) return -int(fail(MX_ERR_INVALID_ARG, "M=%d", M));
+    return choose_path(L, M, opts);
+}
+
+mx_status mx_gemm_workspace_size(const mx_layout* L, int M, const mx_gemm_opts* opts, size_t* bytes) {
+    mx_status st = check_layout(L);
+    if (st != MX_OK) return st;
+    if (bytes == nullptr) return fail(MX_ERR_INVALID_ARG, "bytes is NULL");
+    if (M < 0) return fail(MX_ERR_INVALID_ARG, "M=%d", M);
+    *bytes = 0;
+    if (M == 0) return MX_OK;
+    if (choose_path(L, M, opts) == 1) *bytes = mx::plan_splitk(*L, M, opts ? opts->split : 0).ws_bytes;
+    return MX_OK;
+}
+
+mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const uint16_t* s_a,
+                  int M, uint16_t* Y, int64_t ldy, void* workspace, size_t ws_bytes,
+                  const mx_gemm_opts* opts, void* stream) {
+    mx_status st = check_layout(L);
+    if (st != MX_OK) return st;
+    if (M < 0) return fail(MX_ERR_INVALID_ARG, "M=%d", M);
+    if (ldy < L->N) return fail(MX_ERR_INVALID_ARG, "ldy=%lld < N=%d", (long long)ldy, L->N);
+    if (M == 0) return MX_OK;
+    if (M > 65535) return fail(MX_ERR_UNSUPPORTED, "M=%d above 65535", M);
+    if ((st = check_device_ptr(blob, "blob")) != MX_OK) return st;
+    if ((st = check_device_ptr(Aq, "Aq")) != MX_OK) return st;
+    if ((st = check_device_ptr(s_a, "s_a")) != MX_OK) return st;
+    if ((st = check_device_ptr(Y, "Y")) != MX_OK) return st;
+    if (!aligned16(blob) || !aligned16(Aq)) return fail(MX_ERR_ALIGNMENT, "blob and Aq must be 16-byte aligned");
+    if (opts && opts->debug_partials && (st = check_device_ptr(opts->debug_partials, "debug_partials")) != MX_OK)
+        return st;
+    if (opts && opts->status && (st = check_device_ptr(opts->status, "status")) != MX_OK) return st;
+    const int path = choose_path(L, M, opts);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (path == 1) {
+        mx::SplitPlan plan = mx::plan_splitk(*L, M, opts ? opts->split : 0);
+        if (ws_bytes < plan.ws_bytes || (plan.ws_bytes && workspace == nullptr))
+            return fail(MX_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.ws_bytes, ws_bytes);
+        if ((st = check_device_ptr(workspace, "workspace")) != MX_OK) return st;
+        if (!aligned16(workspace)) return fail(MX_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+        cudaError_t e = mx::launch_gemm_splitk(*L, blob, Aq, s_a, M, Y, ldy, static_cast<float*>(workspace),
+                                               plan, opts ? opts->debug_partials : nullptr, s);
+        if (e != cudaSuccess) return cuda_fail(e, "split-K GEMM launch");
+        return MX_OK;
+    }
+    return fail(MX_ERR_UNSUPPORTED, "GEMM path %d is not available", path);
+}
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+// quant_act.cu -- per-token 8-bit symmetric activation quantization.
+//
+// MixLLM section 3.1.2 keeps activations at 8 bits, symmetric; the quantizer is
+// the symmetric form of section 2.1 with the restricted range +-127:
+//   s_a[m] = fp16(max_k |X[m,k]| / 127)   (0 -> 1, fp16 overflow saturates)
+//   Aq[m,k] = clamp(round_half_even(X[m,k] / s_a[m]), -127, 127)
+// Every fp32 step is a single IEEE operation (__fdiv_rn, no contraction) so the
+// integer codes are decided exactly as the definition states.
+//
+// One CTA per token row.  Pass 1 reads the row with 16-byte vector loads and
+// reduces |x| with warp shuffles and one shared-memory step; pass 2 re-reads
+// the row (an L2 hit: the row was just streamed) and writes 8 codes per store.
+// HBM traffic is the algorithmic 2 MK (fp16 in) + MK + 2M bytes.
+#include "mx_internal.cuh"
+
+namespace mx {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename T> struct Vec;
+template <> struct Vec<__half> {
+    static constexpr int kElems = 8;   // 16 bytes
+    __device__ static void load(const __half* p, float (&v)[8]) {
+        uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
+        const __half2* h = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 f = __half22float2(h[i]);
+            v[2 * i] = f.x;
+            v[2 * i + 1] = f.y;
+        }
+    }
+};
+template <> struct Vec<float> {
+    static constexpr int kElems = 8;   // two 16-byte loads
+    __device__ static void load(const float* p, float (&v)[8]) {
+        float4 a = __ldg(reinterpret_cast<const float4*>(p));
+        float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+};
+
+__device__ __forceinline__ uint32_t quant4(const float* v, float s) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float q = rintf(__fdiv_rn(v[i], s));
+        q = fminf(fmaxf(q, -127.0f), 127.0f);
+        w |= (uint32_t(int32_t(q)) & 0xFFu) << (8 * i);
+    }
+    return w;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+quant_act_kernel(const T* __restrict__ X, int K, int64_t ldx, int8_t* __restrict__ Aq,
+                 __half* __restrict__ s_a) {
+    const int m = blockIdx.x;
+    const T* x = X + int64_t(m) * ldx;
+    const int nvec = K / Vec<T>::kElems;
+
+    float amax = 0.0f;
+    for (int i = threadIdx.x; i < nvec; i += kThreads) {
+        float v[8];
+        Vec<T>::load(x + i * 8, v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    __shared__ float red[kThreads / 32];
+    __shared__ float s_shared;
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float a = red[0];
+#pragma unroll
+        for (int w = 1; w < kThreads / 32; ++w) a = fmaxf(a, red[w]);
+        // fp16 scale; values above the largest finite fp16 saturate to 65504
+        __half h = __float2half_rn(fminf(__fdiv_rn(a, 127.0f), 65504.0f));
+        float s = __half2float(h);
+        if (s == 0.0f) {
+            s = 1.0f;
+            h = __float2half_rn(1.0f);
+        }
+        s_a[m] = h;
+        s_shared = s;
+    }
+    __syncthreads();
+    const float s = s_shared;
+
+    int8_t* q = Aq + int64_t(m) * K;
+    for (int i = threadIdx.x; i < nvec; i += kThreads) {
+        float v[8];
+        Vec<T>::load(x + i * 8, v);
+        uint2 out;
+        out.x = quant4(v, s);
+        out.y = quant4(v + 4, s);
+        *reinterpret_cast<uint2*>(q + i * 8) = out;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_quant_act(const void* X, mx_dtype xdt, int M, int K, int64_t ldx,
+                             int8_t* Aq, uint16_t* s_a, cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    dim3 grid(M), block(kThreads);
+    if (xdt == MX_F16)
+        quant_act_kernel<__half><<<grid, block, 0, s>>>(static_cast<const __half*>(X), K, ldx,
+                                                        Aq, reinterpret_cast<__half*>(s_a));
+    else
+        quant_act_kernel<float><<<grid, block, 0, s>>>(static_cast<const float*>(X), K, ldx,
+                                                       Aq, reinterpret_cast<__half*>(s_a));
+    return cudaGetLastError();
+}
+
+}  // namespace mx

@@ -1,0 +1,74 @@
+"""MixedPrecisionLinear: the user-facing object around the C ABI.
+
+It owns the packed weight blob (torch device memory), sizes the workspace, and
+runs one forward pass as quantize-activations -> mixed-precision GEMM on the
+current CUDA stream.  All arithmetic happens in libmx.so's kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as mx
+
+
+class MixedPrecisionLinear:
+    """Y = X W^T with W split into 8-bit symmetric / 4-bit asymmetric rows (MixLLM)."""
+
+    def __init__(self, W: torch.Tensor, is8: torch.Tensor, group: int = 128, n8: int | None = None):
+        if not W.is_cuda:
+            raise ValueError("W must be a CUDA tensor")
+        N, K = W.shape
+        if n8 is None:
+            n8 = int(is8.count_nonzero().item())
+        self.layout = mx.mx_layout_init(N, K, group, n8)
+        self.blob = torch.empty(self.layout.total_bytes, dtype=torch.uint8, device=W.device)
+        self._status = torch.zeros(1, dtype=torch.int32, device=W.device)
+        mx.mx_pack_weights(self.layout, W, is8.to(W.device, torch.uint8), self.blob, status=self._status)
+        self._ws = {}
+
+    @classmethod
+    def from_blob(cls, blob: torch.Tensor) -> "MixedPrecisionLinear":
+        """Re-open a packed blob (for example one saved with torch.save)."""
+        self = cls.__new__(cls)
+        self.layout = mx.mx_layout_from_header(blob[:mx.HEADER_BYTES].cpu())
+        if blob.numel() < self.layout.total_bytes:
+            raise ValueError("blob shorter than its header says")
+        self.blob = blob
+        self._status = torch.zeros(1, dtype=torch.int32, device=blob.device)
+        self._ws = {}
+        return self
+
+    @property
+    def N(self) -> int:
+        return self.layout.N
+
+    @property
+    def K(self) -> int:
+        return self.layout.K
+
+    def check_pack_status(self) -> None:
+        """Raise if the packer reported an error (mask count mismatch)."""
+        st = int(self._status.item())
+        if st != 0:
+            raise mx.MXError(st, "mx_pack_weights", "device-side error while packing")
+
+    def workspace(self, M: int, path: int = 0) -> torch.Tensor | None:
+        key = (M, path)
+        if key not in self._ws:
+            n = mx.mx_gemm_workspace_size(self.layout, M, path=path)
+            self._ws[key] = torch.empty(max(n, 16), dtype=torch.uint8, device=self.blob.device) if n else None
+        return self._ws[key]
+
+    def forward(self, X: torch.Tensor, out: torch.Tensor | None = None, path: int = 0) -> torch.Tensor:
+        M, K = X.shape
+        if K != self.K:
+            raise ValueError(f"X has K={K}, layer expects {self.K}")
+        dev = self.blob.device
+        Aq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sa = torch.empty((M,), dtype=torch.float16, device=dev)
+        Y = out if out is not None else torch.empty((M, self.N), dtype=torch.float16, device=dev)
+        mx.mx_quant_act(X, Aq, sa)
+        mx.mx_gemm(self.layout, self.blob, Aq, sa, Y, workspace=self.workspace(M, path), path=path)
+        return Y
+
+    __call__ = forward

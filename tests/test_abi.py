@@ -1,0 +1,126 @@
+"""The C-ABI library loads and exports every declared entry point; host-only logic.
+
+None of these tests launches a kernel or needs a GPU: they exercise the packed
+layout geometry, header validation and the argument checks that fail before any
+CUDA call is made.
+"""
+import ctypes
+import os
+import re
+import struct
+
+import pytest
+
+from mixed_precision_quantized_mx_b200 import binding as mx
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "mx.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:mx_status|int|const char\*)\s+(mx_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mixed_precision_quantized_mx_b200 import build
+    build.build()
+    return mx.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    syms = declared_symbols()
+    assert len(syms) >= 8
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert sorted(mx.EXPORTED) == syms          # the binding mirrors the header names
+
+
+def test_version(lib):
+    assert mx.mx_version() == 1
+
+
+def _expected_total(N, K, g, n8):
+    a = lambda v: (v + 255) // 256 * 256
+    t8, t4 = -(-n8 // 128), -(-(N - n8) // 128)
+    G = K // g
+    off = 256
+    off = a(off + (t8 + t4) * 128 * 4)
+    off = a(off + t8 * 128 * G * 2)
+    off = a(off + t8 * 128 * K)
+    off = a(off + t4 * 128 * G * 2)
+    off = a(off + t4 * 128 * G)
+    off = a(off + t4 * 128 * K // 2)
+    return off
+
+
+@pytest.mark.parametrize("N,K,g,n8", [(512, 512, 128, 51), (4096, 4096, 128, 410),
+                                      (300, 256, 64, 37), (128, 128, 128, 0), (128, 128, 128, 128),
+                                      (28672, 8192, 128, 2867)])
+def test_layout_geometry(lib, N, K, g, n8):
+    L = mx.mx_layout_init(N, K, g, n8)
+    assert (L.N, L.K, L.group, L.n8, L.n4, L.G) == (N, K, g, n8, N - n8, K // g)
+    assert (L.t8, L.t4, L.kblocks) == (-(-n8 // 128), -(-(N - n8) // 128), K // 128)
+    assert L.total_bytes == _expected_total(N, K, g, n8)
+    offs = [L.off_rowmap, L.off_scales8, L.off_codes8, L.off_scales4, L.off_zeros4, L.off_codes4]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert L.off_codes4 + L.t4 * 128 * K // 2 <= L.total_bytes
+
+
+@pytest.mark.parametrize("args,status", [
+    ((0, 128, 128, 0), 1), ((16, 128, 128, 17), 1), ((16, 128, 128, -1), 1),
+    ((16, 128, 32, 0), 2), ((16, 192, 64, 0), 2), ((16, 100, 128, 0), 2)])
+def test_layout_rejects(lib, args, status):
+    with pytest.raises(mx.MXError) as e:
+        mx.mx_layout_init(*args)
+    assert e.value.status == status
+    assert mx.lib().mx_last_error().decode()
+
+
+def test_header_round_trip_and_corruption(lib):
+    hdr = struct.pack("<6I", 0x4B50584D, 1, 4096, 4096, 128, 410) + bytes(256 - 24)
+    L = mx.mx_layout_from_header(hdr)
+    ref = mx.mx_layout_init(4096, 4096, 128, 410)
+    assert bytes(L) == bytes(ref)
+    bad = [struct.pack("<6I", 0x12345678, 1, 4096, 4096, 128, 410),
+           struct.pack("<6I", 0x4B50584D, 9, 4096, 4096, 128, 410),
+           struct.pack("<6I", 0x4B50584D, 1, 4096, 4096, 96, 410),
+           struct.pack("<6I", 0x4B50584D, 1, 4096, 4096, 128, 5000)]
+    for h in bad:
+        with pytest.raises(mx.MXError) as e:
+            mx.mx_layout_from_header(h + bytes(256 - 24))
+        assert e.value.status == 6
+    with pytest.raises(mx.MXError) as e:
+        mx.mx_layout_from_header(hdr[:100])
+    assert e.value.status == 6
+
+
+def test_host_argument_checks_before_any_launch(lib):
+    P = ctypes.c_void_p
+    # quant_act: K not a multiple of 8 / bad dtype / negative M
+    assert lib.mx_quant_act(None, 1, 4, 12, 12, None, None, None) == 2
+    assert lib.mx_quant_act(None, 7, 4, 16, 16, None, None, None) == 1
+    assert lib.mx_quant_act(None, 1, -1, 16, 16, None, None, None) == 1
+    assert lib.mx_quant_act(None, 1, 0, 16, 16, None, None, None) == 0      # M = 0: no-op
+    L = mx.mx_layout_init(256, 256, 128, 10)
+    # a layout edited after init is refused
+    L2 = mx.mx_layout_init(256, 256, 128, 10)
+    L2.t8 = 7
+    o = mx.GemmOpts(0, 0, None, None)
+    assert lib.mx_gemm(ctypes.byref(L2), None, None, None, 1, None, 256, None, 0, ctypes.byref(o), None) == 1
+    # ldy < N, NULL layout
+    assert lib.mx_gemm(ctypes.byref(L), None, None, None, 1, None, 100, None, 0, ctypes.byref(o), None) == 1
+    assert lib.mx_gemm(None, None, None, None, 1, None, 256, None, 0, ctypes.byref(o), None) == 1
+    # M = 0 is a no-op that touches nothing
+    assert lib.mx_gemm(ctypes.byref(L), None, None, None, 0, None, 256, None, 0, ctypes.byref(o), None) == 0
+    n = ctypes.c_size_t(123)
+    assert lib.mx_gemm_workspace_size(ctypes.byref(L), 0, ctypes.byref(o), ctypes.byref(n)) == 0
+    assert n.value == 0
+
+
+def test_split_workspace_is_sized_on_host(lib):
+    L = mx.mx_layout_init(4096, 4096, 128, 410)
+    w1 = mx.mx_gemm_workspace_size(L, 1, path=mx.PATH_SPLITK)
+    w16 = mx.mx_gemm_workspace_size(L, 16, path=mx.PATH_SPLITK)
+    assert w1 > 0 and w16 == 16 * w1 and w1 % (128 * 4) == 0
