@@ -102,6 +102,12 @@ typedef struct mx_gemm_opts {
     int32_t* debug_partials;   /* device int32 [M][N][G] or NULL: every per-group
                                   int32 partial P[m][n][g] (original row order) */
     int32_t* status;           /* device int32 or NULL: kernel-side error code */
+    int32_t wait_timeout_us;   /* bound on every in-kernel wait of the tensor-core
+                                  path (0 = 2 s); on expiry the kernel writes
+                                  MX_ERR_TIMEOUT to *status, frees what it holds
+                                  and returns */
+    int32_t test_stall;        /* testing only: the tensor-core loader issues no
+                                  copies, so the waits run out (needs status) */
 } mx_gemm_opts;
 
 /* ABI version of the loaded library (MX_ABI_VERSION). */

@@ -47,7 +47,8 @@ class Layout(ctypes.Structure):
 class GemmOpts(ctypes.Structure):
     """mirror of mx_gemm_opts"""
     _fields_ = [("path", ctypes.c_int32), ("split", ctypes.c_int32),
-                ("debug_partials", ctypes.c_void_p), ("status", ctypes.c_void_p)]
+                ("debug_partials", ctypes.c_void_p), ("status", ctypes.c_void_p),
+                ("wait_timeout_us", ctypes.c_int32), ("test_stall", ctypes.c_int32)]
 
 
 _lib = None
@@ -107,8 +108,9 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def _opts(path=0, split=0, debug_partials=None, status=None) -> GemmOpts:
-    return GemmOpts(path, split, _ptr(debug_partials), _ptr(status))
+def _opts(path=0, split=0, debug_partials=None, status=None, wait_timeout_us=0,
+          test_stall=0) -> GemmOpts:
+    return GemmOpts(path, split, _ptr(debug_partials), _ptr(status), wait_timeout_us, test_stall)
 
 
 # ------------------------------------------------------------------ entry points
@@ -165,9 +167,9 @@ def mx_gemm_select_path(L: Layout, M: int, path: int = 0, split: int = 0) -> int
 def mx_gemm(L: Layout, blob: torch.Tensor, Aq: torch.Tensor, s_a: torch.Tensor, Y: torch.Tensor,
             workspace: torch.Tensor | None = None, path: int = 0, split: int = 0,
             debug_partials: torch.Tensor | None = None, status: torch.Tensor | None = None,
-            stream=None) -> None:
+            wait_timeout_us: int = 0, test_stall: int = 0, stream=None) -> None:
     M = Aq.shape[0]
-    o = _opts(path, split, debug_partials, status)
+    o = _opts(path, split, debug_partials, status, wait_timeout_us, test_stall)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().mx_gemm(ctypes.byref(L), _ptr(blob), _ptr(Aq), _ptr(s_a), M, _ptr(Y), Y.stride(0),
                          _ptr(workspace), ws_bytes, ctypes.byref(o), _stream(stream)), "mx_gemm")

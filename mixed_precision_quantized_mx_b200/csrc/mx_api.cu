@@ -161,11 +161,14 @@ mx_status mx_quant_act(const void* X, mx_dtype xdtype, int M, int K, int64_t ldx
     return MX_OK;
 }
 
+// Decode-sized M is bound by HBM: the split-K CUDA-core path streams the
+// weights with enough CTAs; from 17 tokens on, the tensor-core path.
+constexpr int kDecodeMaxM = 16;
+
 static int choose_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
     (void)L;
     if (opts && opts->path) return opts->path;
-    (void)M;
-    return 1;   // the tensor-core path is selected here once it is built
+    return M <= kDecodeMaxM ? 1 : 2;
 }
 
 int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
@@ -216,7 +219,20 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
         if (e != cudaSuccess) return cuda_fail(e, "split-K GEMM launch");
         return MX_OK;
     }
-    return fail(MX_ERR_UNSUPPORTED, "GEMM path %d is not available", path);
+    if (path == 2) {
+        if (opts && opts->test_stall && !opts->status)
+            return fail(MX_ERR_INVALID_ARG, "test_stall needs a status word");
+        if (opts && opts->wait_timeout_us < 0) return fail(MX_ERR_INVALID_ARG, "wait_timeout_us < 0");
+        const uint64_t timeout_ns =
+            (opts && opts->wait_timeout_us > 0) ? uint64_t(opts->wait_timeout_us) * 1000u : 2000000000ull;
+        cudaError_t e = mx::launch_gemm_tc(*L, blob, Aq, s_a, M, Y, ldy,
+                                           opts ? opts->debug_partials : nullptr,
+                                           opts ? opts->status : nullptr, timeout_ns,
+                                           opts ? opts->test_stall : 0, s);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core GEMM launch");
+        return MX_OK;
+    }
+    return fail(MX_ERR_INVALID_ARG, "unknown GEMM path %d", path);
 }
 
 }  // extern "C"

@@ -68,4 +68,9 @@ cudaError_t launch_gemm_splitk(const mx_layout& L, const void* blob, const int8_
                                float* ws, const SplitPlan& plan, int32_t* debug_partials,
                                cudaStream_t s);
 
+cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* Aq,
+                           const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy,
+                           int32_t* debug_partials, int32_t* status, uint64_t timeout_ns,
+                           int stall_test, cudaStream_t s);
+
 }  // namespace mx

@@ -251,3 +251,62 @@ def test_gemm_rejects_bad_arguments(orc):
     with pytest.raises(mx.MXError) as e:
         mx.mx_quant_act(Xh, Aq, sa)
     assert e.value.status == 1
+
+
+# ------------------------------------------------------------------ tensor-core path
+@pytest.mark.parametrize("M", [1, 17, 128, 129, 300])
+@pytest.mark.parametrize("g", [64, 128])
+def test_gemm_tc_token_counts(orc, M, g):
+    rng = np.random.default_rng(M * 31 + g)
+    N, K = 300, 512
+    X = inputs.activations(rng, M, K, 5)
+    W = inputs.weights(rng, N, K, outlier_frac=0.001)
+    is8 = inputs.saliency_mask(np.abs(rng.standard_normal(N)), 37)
+    run_and_check(orc, X, W, is8, g, path=mx.PATH_TENSOR)
+
+
+@pytest.mark.parametrize("frac", [0.0, 1.0])
+def test_gemm_tc_degenerate_fractions(orc, frac):
+    rng = np.random.default_rng(int(frac * 10) + 7)
+    M, N, K = 130, 256, 2048
+    X = inputs.activations(rng, M, K, 20)
+    W = inputs.weights(rng, N, K, outlier_frac=0.001)
+    is8 = np.full(N, int(frac), np.uint8)
+    run_and_check(orc, X, W, is8, 128, path=mx.PATH_TENSOR)
+
+
+def test_paths_agree_bit_exact_partials(orc):
+    rng = np.random.default_rng(21)
+    M, N, K = 24, 400, 1024
+    X = inputs.activations(rng, M, K, 10)
+    W = inputs.weights(rng, N, K, outlier_frac=0.001)
+    is8 = inputs.saliency_mask(np.abs(rng.standard_normal(N)), 40)
+    Aq, sa = gpu_quant(X)
+    L, blob = gpu_pack(W, is8, 128)
+    Y1, P1, _ = gpu_gemm(L, blob, Aq, sa, path=mx.PATH_SPLITK, debug=True)
+    Y2, P2, _ = gpu_gemm(L, blob, Aq, sa, path=mx.PATH_TENSOR, debug=True)
+    assert torch.equal(P1, P2)
+    y1, y2 = Y1.float().cpu().numpy(), Y2.float().cpu().numpy()
+    assert np.abs(y1 - y2).max() <= 2 * 2e-3 * np.abs(y1).max()
+
+
+@pytest.mark.parametrize("M,K,N", [(256, 4096, 14336), (2048, 4096, 14336), (2048, 14336, 4096),
+                                   (4096, 8192, 28672)])
+def test_gemm_tc_llama_shapes_sampled(orc, M, K, N):
+    lay = inputs.llama_layer(M, K, N, seed=M + K + N)
+    Aq, sa, Aq_o, sa_o = check_quant(orc, lay.X)
+    L, blob = gpu_pack(lay.W, lay.is8, 128)
+    c = orc.pack(lay.W, lay.is8, 128)
+    assert mx.mx_gemm_select_path(L, M) == mx.PATH_TENSOR
+    Y, _, _ = gpu_gemm(L, blob, Aq, sa)
+    Yh = Y.cpu().numpy()
+    rng = np.random.default_rng(1)
+    y0 = orc.gemm(Aq_o, sa_o, c, pairs=(np.full(N, M - 1, np.int32), np.arange(N)))[1]
+    assert_y_close(Yh[M - 1], y0)
+    rows = rng.integers(0, N, 8)
+    ym = orc.gemm(Aq_o, sa_o, c, pairs=(np.repeat(np.arange(M), 8), np.tile(rows, M)))[1]
+    assert_y_close(Yh[:, rows].reshape(-1), ym, rows_rms=np.sqrt(np.mean(y0 ** 2)))
+    pm = rng.integers(0, M, 1024)
+    pn = rng.integers(0, N, 1024)
+    yr = orc.gemm(Aq_o, sa_o, c, pairs=(pm, pn))[1]
+    assert_y_close(Yh[pm, pn], yr, rows_rms=np.sqrt(np.mean(y0 ** 2)))
