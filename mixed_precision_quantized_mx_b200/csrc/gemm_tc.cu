@@ -3,27 +3,32 @@
 // Two-step dequantization (MixLLM section 3.3) on 5th-generation tensor cores:
 //   step 1: per quantization group, P = A_q . (W_q - z)^T with tcgen05.mma
 //           kind::i8 (int8 x int8 -> int32) into a TMEM accumulator that holds
-//           only that group's sum;
-//   step 2: the epilogue warps read P from TMEM, convert it with the fast
-//           int-to-float of section 3.3 (Figure 3) and accumulate
-//           acc += float(P) * s_w[row, group] in fp32 registers; at the end of
-//           the tile Y = fp16(acc * s_a[token]) is scattered to the original
-//           output columns (section 3.3, fused scatter epilogue).
+//           only that group's sum; the accumulator starts at the fast-I2F bias
+//           integer (section 3.3: the accumulator is initialised with the bias),
+//   step 2: the epilogue warps read bias + P from TMEM, subtract the float bias
+//           (section 3.3, Figure 3) and accumulate acc += float(P) * s_w[row, group]
+//           in fp32 registers; at the end of the tile Y = fp16(acc * s_a[token])
+//           is scattered to the original output columns (section 3.3, fused
+//           scatter epilogue).
 // The group tile of the paper's software pipeline (section 3.3, Figure 4)
-// becomes a pair of TMEM buffers: the MMA fills one group's accumulator while
-// the epilogue drains the other.
+// becomes a ring of four TMEM group accumulators: the MMA fills one while the
+// epilogue drains the others.
 //
 // Tile: 128 packed weight rows (UMMA M) x 128 tokens (UMMA N), the whole K.
+// A pipeline stage holds two k-blocks (256 columns of K): 32 KB of int8 weight
+// operand and 32 KB of activations.  Each stage is filled by exactly two copies
+// issued from two different warps -- one bulk copy of the pre-packed weight
+// blocks (int8 rows already in the 128-byte-swizzled operand layout, or the
+// uint4 codes, which land in the upper half of the operand buffer) and one 3-D
+// TMA box of activations -- because on sm_100a copies issued by one thread
+// complete one after another, so few large copies from several issuers are
+// what keeps the tensor cores fed.
 // Warp roles (512 threads):
-//   warp 0      loader: per k-block, one bulk copy of the pre-packed weight
-//               block (16 KB int8, already in the 128-byte-swizzled operand
-//               layout; or 8 KB of uint4 codes) and one TMA tile of
-//               activations (128 tokens x 128 bytes, hardware-swizzled)
-//   warp 1      MMA issuer (one thread)
-//   warp 2      TMEM allocator
+//   warp 0      weight copies           warp 3      activation copies
+//   warp 1      MMA issuer (one thread) warp 2      TMEM allocator
 //   warps 4-7   widening (step one for 4-bit rows): uint4 codes -> int8 (q - z)
-//               written in the swizzled operand layout, four codes per 32-bit
-//               operation (the vsub4 idea of section 3.3, done with a biased add)
+//               in place, four codes per 32-bit operation (the vsub4 idea of
+//               section 3.3, done with a biased add)
 //   warps 8-15  epilogue (two warps per TMEM lane quarter, 64 tokens each)
 // Persistent CTAs walk the (row tile, token tile) list; consecutive tiles share
 // a row tile, so CTAs running together read each weight block once from HBM.
@@ -41,24 +46,26 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int kStages = 4;
-constexpr int kABytes = BM * kKBlock;          // int8 weight operand per stage
-constexpr int kBBytes = BN * kKBlock;          // int8 activation operand per stage
-constexpr int kRawBytes = BM * kKBlock / 2;    // packed uint4 codes per stage
+constexpr int kKbPerStage = 2;                 // k-blocks per pipeline stage
+constexpr int kStages = 3;
+constexpr int kABytes = BM * kKBlock;          // int8 weight operand of one k-block
+constexpr int kBBytes = BN * kKBlock;          // int8 activation operand of one k-block
+constexpr int kRawBytes = BM * kKBlock / 2;    // uint4 codes of one k-block
 constexpr int kThreads = 512;
 constexpr int kWidenThreads = 128;
 constexpr int kEpiWarps = 8;
-constexpr uint32_t kTmemCols = 2 * BN;         // two int32 group accumulators
+constexpr int kAccBufs = 4;                     // int32 group accumulators in TMEM
+constexpr uint32_t kTmemCols = kAccBufs * BN;   // all 512 columns
+constexpr int kWidenBarrier = 1;                // named barrier of the widening warps
 
 struct __align__(1024) Smem {
-    uint8_t A[kStages][kABytes];
-    uint8_t B[kStages][kBBytes];
-    uint8_t Raw[kStages][kRawBytes];
-    uint64_t full[kStages];       // loader -> widen/MMA: stage bytes landed
-    uint64_t wdone[kStages];      // widen -> MMA: operand A ready
-    uint64_t empty[kStages];      // MMA -> loader: stage consumed
-    uint64_t acc_full[2];         // MMA -> epilogue: group accumulator complete
-    uint64_t acc_empty[2];        // epilogue -> MMA: accumulator drained
+    uint8_t A[kStages][kKbPerStage * kABytes];  // raw uint4 codes land at A + kABytes
+    uint8_t B[kStages][kKbPerStage * kBBytes];
+    uint64_t full[kStages];       // both copies of the stage landed (2 arrivals + bytes)
+    uint64_t wdone[kStages];      // widen -> MMA: weight operand ready
+    uint64_t empty[kStages];      // MMA -> loaders: stage consumed
+    uint64_t acc_full[kAccBufs];  // MMA -> epilogue: group accumulator complete
+    uint64_t acc_empty[kAccBufs]; // epilogue -> MMA: accumulator drained and re-armed
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort;
@@ -85,6 +92,16 @@ __device__ __forceinline__ uint32_t widen_hi(uint32_t w, uint32_t zc) {
     return (((w >> 4) & 0x0F0F0F0Fu) + zc) ^ 0x80808080u;
 }
 
+// Drain every issued stage (bounded) so that no copy targets this CTA's shared
+// memory after it exits.
+__device__ __forceinline__ void drain_stages(Smem& S, int issued, uint64_t timeout_ns) {
+    for (int j = max(0, issued - kStages); j < issued; ++j) {
+        int dummy = 0;
+        mbar_wait_bounded(&S.full[j % kStages], (j / kStages) & 1, &dummy, nullptr, timeout_ns);
+    }
+}
+
+template <bool DEBUG>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -93,15 +110,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     const Geom& g = a.g;
     const int gpk = kKBlock / g.group;            // groups per k-block (1 or 2)
     const int ksteps = g.group / 32;              // MMA k-steps per group
+    const int n_ss = (g.kblocks + kKbPerStage - 1) / kKbPerStage;   // stages per tile
     volatile int* abort = &S.abort;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&S.full[s], 1);
-            mbar_init(&S.wdone[s], kWidenThreads);
+            mbar_init(&S.full[s], 2);
+            mbar_init(&S.wdone[s], kWidenThreads / 32);
             mbar_init(&S.empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kAccBufs; ++b) {
             mbar_init(&S.acc_full[b], 1);
             mbar_init(&S.acc_empty[b], kEpiWarps);
         }
@@ -118,34 +136,48 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
+    if (warp >= 8) {
+        // every group accumulator starts at the fast-I2F bias, so all MMAs accumulate
+        const uint32_t la = tmem + (uint32_t((warp & 3) * 32) << 16) + ((warp - 8) >> 2) * 64;
+        for (int b = 0; b < kAccBufs; ++b)
+            for (int h = 0; h < 2; ++h) tmem_st_x32_splat(la + b * BN + h * 32, kI2FBiasBits);
+        tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ loader
+    if (warp == 0 || warp == 3) {
+        // ------------------------------------------------------------ loaders
         if (lane == 0 && !a.stall_test) {
+            const bool weights = warp == 0;
             int it = 0;
             for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
                 const int rt = t / a.n_tt, tt = t % a.n_tt;
                 const bool eight = rt < g.t8;
                 const int lt = eight ? rt : rt - g.t8;
-                const uint32_t wbytes = eight ? kABytes : kRawBytes;
-                const uint8_t* wsrc = eight
-                    ? reinterpret_cast<const uint8_t*>(g.codes8) + size_t(lt) * g.kblocks * kABytes
-                    : g.codes4 + size_t(lt) * g.kblocks * kRawBytes;
-                for (int kb = 0; kb < g.kblocks; ++kb, ++it) {
+                for (int sp = 0; sp < n_ss; ++sp, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
                     if (!mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, a.status, a.timeout_ns)) goto load_done;
-                    mbar_arrive_expect_tx(&S.full[s], wbytes + kBBytes);
-                    bulk_g2s(eight ? S.A[s] : S.Raw[s], wsrc + size_t(kb) * wbytes, wbytes, &S.full[s]);
-                    tma_load_2d(S.B[s], &amap, kb * kKBlock, tt * BN, &S.full[s]);
+                    const int kb0 = sp * kKbPerStage;
+                    if (weights) {
+                        const int nkb = min(kKbPerStage, g.kblocks - kb0);
+                        const uint32_t bytes = uint32_t(nkb * (eight ? kABytes : kRawBytes));
+                        const uint8_t* src =
+                            eight ? reinterpret_cast<const uint8_t*>(g.codes8) + (size_t(lt) * g.kblocks + kb0) * kABytes
+                                  : g.codes4 + (size_t(lt) * g.kblocks + kb0) * kRawBytes;
+                        mbar_arrive_expect_tx(&S.full[s], bytes);
+                        bulk_g2s(eight ? S.A[s] : S.A[s] + kABytes, src, bytes, &S.full[s]);
+                    } else {
+                        // the box always spans two k-blocks; a missing last one reads as zeros
+                        mbar_arrive_expect_tx(&S.full[s], kKbPerStage * kBBytes);
+                        tma_load_3d(S.B[s], &amap, 0, tt * BN, kb0, &S.full[s]);
+                    }
                 }
             }
         load_done:
-            // every issued copy must land before the CTA can exit
-            for (int j = max(0, it - kStages); j < it; ++j) {
-                int dummy = 0;
-                mbar_wait_bounded(&S.full[j % kStages], (j / kStages) & 1, &dummy, nullptr, a.timeout_ns);
-            }
+            drain_stages(S, it, a.timeout_ns);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -154,24 +186,28 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             int it = 0;
             uint32_t gc = 0;
             for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
-                for (int kb = 0; kb < g.kblocks; ++kb, ++it) {
+                for (int sp = 0; sp < n_ss; ++sp, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
                     if (!mbar_wait_bounded(&S.full[s], ph, abort, a.status, a.timeout_ns)) goto mma_out;
                     if (!mbar_wait_bounded(&S.wdone[s], ph, abort, a.status, a.timeout_ns)) goto mma_out;
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(S.A[s]), b0 = smem_u32(S.B[s]);
-                    for (int j = 0; j < gpk; ++j, ++gc) {
-                        const uint32_t b = gc & 1, u = gc >> 1;
-                        if (!mbar_wait_bounded(&S.acc_empty[b], (u & 1) ^ 1, abort, a.status, a.timeout_ns))
-                            goto mma_out;
-                        tc_fence_after();
-                        for (int kk = 0; kk < ksteps; ++kk) {
-                            const uint32_t off = uint32_t(j * g.group + kk * 32);
-                            mma_i8(tmem + b * BN, sw128_kmajor_desc(a0 + off), sw128_kmajor_desc(b0 + off),
-                                   idesc, kk > 0 ? 1u : 0u);
+                    const int nkb = min(kKbPerStage, g.kblocks - sp * kKbPerStage);
+                    for (int kbi = 0; kbi < nkb; ++kbi) {
+                        const uint32_t a0 = smem_u32(S.A[s] + kbi * kABytes);
+                        const uint32_t b0 = smem_u32(S.B[s] + kbi * kBBytes);
+                        for (int j = 0; j < gpk; ++j, ++gc) {
+                            const uint32_t b = gc % kAccBufs, u = gc / kAccBufs;
+                            if (!mbar_wait_bounded(&S.acc_empty[b], (u & 1) ^ 1, abort, a.status, a.timeout_ns))
+                                goto mma_out;
+                            tc_fence_after();
+                            for (int kk = 0; kk < ksteps; ++kk) {
+                                const uint32_t off = uint32_t(j * g.group + kk * 32);
+                                mma_i8(tmem + b * BN, sw128_kmajor_desc(a0 + off), sw128_kmajor_desc(b0 + off),
+                                       idesc, 1u);
+                            }
+                            mma_commit(&S.acc_full[b]);
                         }
-                        mma_commit(&S.acc_full[b]);
                     }
                     mma_commit(&S.empty[s]);
                 }
@@ -189,36 +225,65 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             const int rt = t / a.n_tt;
             const bool eight = rt < g.t8;
             const int lt = eight ? rt : rt - g.t8;
-            for (int kb = 0; kb < g.kblocks; ++kb, ++it) {
+            const uint8_t* zrow = g.zeros4 + size_t(lt) * g.G * kTileRows;
+            // zero points of this thread's four chunks in k-block kb, as (128 - z) per byte
+            auto load_z = [&](int kb, uint32_t (&zc)[4]) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = wt + kWidenThreads * j, r = i >> 2, c = i & 3;
+                    const int gi = (kb * kKBlock + c * 32) / g.group;
+                    zc[j] = (0x80u - uint32_t(zrow[size_t(gi) * kTileRows + r])) * 0x01010101u;
+                }
+            };
+            uint32_t z0[4] = {0, 0, 0, 0}, z1[4] = {0, 0, 0, 0};
+            if (!eight) {
+                load_z(0, z0);
+                if (g.kblocks > 1) load_z(1, z1);
+            }
+            for (int sp = 0; sp < n_ss; ++sp, ++it) {
                 const int s = it % kStages;
                 const uint32_t ph = (it / kStages) & 1;
-                uint32_t zc[4];
-                if (!eight) {
+                const int kb0 = sp * kKbPerStage;
+                const int nkb = min(kKbPerStage, g.kblocks - kb0);
+                uint32_t zc0[4], zc1[4];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int i = wt + kWidenThreads * j, r = i >> 2, c = i & 3;
-                        const int gi = (kb * kKBlock + c * 32) / g.group;
-                        const uint32_t z = g.zeros4[(size_t(lt) * g.G + gi) * kTileRows + r];
-                        zc[j] = (0x80u - z) * 0x01010101u;
-                    }
+                for (int j = 0; j < 4; ++j) { zc0[j] = z0[j]; zc1[j] = z1[j]; }
+                if (!eight) {                       // next stage's zero points, in flight now
+                    if (kb0 + 2 < g.kblocks) load_z(kb0 + 2, z0);
+                    if (kb0 + 3 < g.kblocks) load_z(kb0 + 3, z1);
                 }
-                if (!mbar_wait_bounded(&S.full[s], ph, abort, a.status, a.timeout_ns)) goto widen_done;
+                const bool ok = mbar_wait_bounded(&S.full[s], ph, abort, a.status, a.timeout_ns);
+                __syncwarp();   // the named barrier is warp-collective
+                // one decision for all 128 widening threads: the in-place conversion below
+                // needs every one of them at the named barrier
+                if (!named_bar_and(kWidenBarrier, kWidenThreads, ok)) goto widen_done;
                 if (!eight) {
+                    const uint8_t* raw = S.A[s] + kABytes;
+                    for (int kbi = 0; kbi < nkb; ++kbi) {
+                        uint4 w[4];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int i = wt + kWidenThreads * j, r = i >> 2, c = i & 3;
-                        const uint4 w = *reinterpret_cast<const uint4*>(S.Raw[s] + i * 16);
-                        uint4 o0, o1;
-                        o0.x = widen_lo(w.x, zc[j]); o0.y = widen_hi(w.x, zc[j]);
-                        o0.z = widen_lo(w.y, zc[j]); o0.w = widen_hi(w.y, zc[j]);
-                        o1.x = widen_lo(w.z, zc[j]); o1.y = widen_hi(w.z, zc[j]);
-                        o1.z = widen_lo(w.w, zc[j]); o1.w = widen_hi(w.w, zc[j]);
-                        *reinterpret_cast<uint4*>(S.A[s] + swz128_offset(r, 2 * c)) = o0;
-                        *reinterpret_cast<uint4*>(S.A[s] + swz128_offset(r, 2 * c + 1)) = o1;
+                        for (int j = 0; j < 4; ++j)
+                            w[j] = *reinterpret_cast<const uint4*>(raw + kbi * kRawBytes + (wt + kWidenThreads * j) * 16);
+                        // the second k-block overwrites the codes it reads: all reads first
+                        if (kbi == 1) named_bar_and(kWidenBarrier, kWidenThreads, true);
+                        uint8_t* out = S.A[s] + kbi * kABytes;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int i = wt + kWidenThreads * j, r = i >> 2, c = i & 3;
+                            const uint32_t z = kbi ? zc1[j] : zc0[j];
+                            uint4 o0, o1;
+                            o0.x = widen_lo(w[j].x, z); o0.y = widen_hi(w[j].x, z);
+                            o0.z = widen_lo(w[j].y, z); o0.w = widen_hi(w[j].y, z);
+                            o1.x = widen_lo(w[j].z, z); o1.y = widen_hi(w[j].z, z);
+                            o1.z = widen_lo(w[j].w, z); o1.w = widen_hi(w[j].w, z);
+                            *reinterpret_cast<uint4*>(out + swz128_offset(r, 2 * c)) = o0;
+                            *reinterpret_cast<uint4*>(out + swz128_offset(r, 2 * c + 1)) = o1;
+                        }
                     }
                     fence_proxy_async_smem();
                 }
-                mbar_arrive(&S.wdone[s]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.wdone[s]);
             }
         }
     widen_done:;
@@ -228,6 +293,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         const int row = q * 32 + lane;               // packed row within the tile
         const int cb = ((warp - 8) >> 2) * 64;       // first of this warp's 64 tokens
         const uint32_t lane_addr = tmem + (uint32_t(q * 32) << 16);
+        const float2 nbias = make_float2(-kI2FBias, -kI2FBias);
         uint32_t gc = 0;
         for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
             const int rt = t / a.n_tt, tt = t % a.n_tt;
@@ -235,45 +301,67 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             const int lt = eight ? rt : rt - g.t8;
             const __half* sc = (eight ? g.scales8 : g.scales4) + size_t(lt) * g.G * kTileRows + row;
             const int orig = g.rowmap[rt * kTileRows + row];
-            float acc[64];
+            float2 acc[32];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
+            for (int c = 0; c < 32; ++c) acc[c] = make_float2(0.0f, 0.0f);
+            // group scales are fetched two groups ahead of their use
+            float sw_n1 = __half2float(sc[0]);
+            float sw_n2 = g.G > 1 ? __half2float(sc[kTileRows]) : 0.0f;
             for (int gi = 0; gi < g.G; ++gi, ++gc) {
-                const float sw = __half2float(sc[size_t(gi) * kTileRows]);
-                const uint32_t b = gc & 1, u = gc >> 1;
+                const float sw = sw_n1;
+                sw_n1 = sw_n2;
+                sw_n2 = gi + 2 < g.G ? __half2float(sc[size_t(gi + 2) * kTileRows]) : 0.0f;
+                const float2 s2 = make_float2(sw, sw);
+                const uint32_t b = gc % kAccBufs, u = gc / kAccBufs;
                 // every lane waits; the warp leaves together if any lane gave up, because
                 // the TMEM loads below are warp-collective (.sync.aligned)
                 const bool ok = mbar_wait_bounded(&S.acc_full[b], u & 1, abort, a.status, a.timeout_ns);
                 if (!__all_sync(0xffffffffu, ok)) goto epi_done;
                 tc_fence_after();
+                // drain the group's 64 columns in four 16-column chunks, loading chunk
+                // h+1 while chunk h is converted; each chunk is re-armed with the bias
+                const uint32_t col0 = lane_addr + b * BN + cb;
+                uint32_t va[16], vb[16];
+                tmem_ld_x16(col0, va);
+                tmem_wait_ld();
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t v[32];
-                    tmem_ld_x32(lane_addr + b * BN + cb + h * 32, v);
-                    tmem_wait_ld();
-                    if (h == 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&S.acc_empty[b]);
+                for (int h = 0; h < 4; ++h) {
+                    uint32_t (&v)[16] = (h & 1) ? vb : va;
+                    uint32_t (&vn)[16] = (h & 1) ? va : vb;
+                    if (h < 3) tmem_ld_x16(col0 + (h + 1) * 16, vn);
+                    tmem_st_x16_splat(col0 + h * 16, kI2FBiasBits);
+                    // acc += (float(bias + P) - bias) * s_w, two columns per instruction
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float2 f = add2(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])),
+                                              nbias);
+                        acc[h * 8 + c] = fma2(f, s2, acc[h * 8 + c]);
                     }
+                    if (DEBUG && orig >= 0) {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        acc[h * 32 + c] = __fmaf_rn(i2f_biased(int32_t(v[c])), sw, acc[h * 32 + c]);
-                    if (a.debug != nullptr && orig >= 0) {
-                        for (int c = 0; c < 32; ++c) {
-                            const int m = tt * BN + cb + h * 32 + c;
-                            if (m < a.M) a.debug[(size_t(m) * g.N + orig) * g.G + gi] = int32_t(v[c]);
+                        for (int c = 0; c < 16; ++c) {
+                            const int m = tt * BN + cb + h * 16 + c;
+                            if (m < a.M)
+                                a.debug[(size_t(m) * g.N + orig) * g.G + gi] = int32_t(v[c] - kI2FBiasBits);
                         }
                     }
+                    if (h < 3) tmem_wait_ld();
                 }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.acc_empty[b]);
             }
             if (orig >= 0) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const int m = tt * BN + cb + c;
-                    if (m < a.M)
-                        a.Y[int64_t(m) * a.ldy + orig] =
-                            __float2half_rn(__fmul_rn(acc[c], __half2float(a.s_a[m])));
+                for (int c = 0; c < 32; ++c) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int m = tt * BN + cb + 2 * c + e;
+                        if (m < a.M)
+                            a.Y[int64_t(m) * a.ldy + orig] = __float2half_rn(
+                                __fmul_rn(e ? acc[c].y : acc[c].x, __half2float(a.s_a[m])));
+                    }
                 }
             }
         }
@@ -322,12 +410,14 @@ cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* A
     cudaError_t e;
     EncodeTiledFn enc = encode_fn(&e);
     if (e != cudaSuccess) return e;
+    // activations as a 3-D tensor [k-block][token][128 bytes], so one box brings
+    // two k-blocks of BN tokens, each landing as its own swizzled 128-byte-row block
     CUtensorMap map;
-    const cuuint64_t dims[2] = {cuuint64_t(L.K), cuuint64_t(M)};
-    const cuuint64_t strides[1] = {cuuint64_t(L.K)};
-    const cuuint32_t box[2] = {cuuint32_t(kKBlock), cuuint32_t(BN)};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(Aq), dims, strides,
+    const cuuint64_t dims[3] = {cuuint64_t(kKBlock), cuuint64_t(M), cuuint64_t(L.kblocks)};
+    const cuuint64_t strides[2] = {cuuint64_t(L.K), cuuint64_t(kKBlock)};
+    const cuuint32_t box[3] = {cuuint32_t(kKBlock), cuuint32_t(BN), cuuint32_t(kKbPerStage)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(Aq), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
@@ -337,7 +427,10 @@ cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* A
     static int sms[64] = {};
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (sms[dev] == 0) {
-        if ((e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((e = cudaFuncSetAttribute(gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(tc_smem_bytes()))) != cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(tc_smem_bytes()))) != cudaSuccess)
             return e;
         int n = 0;
@@ -357,7 +450,10 @@ cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* A
     a.timeout_ns = timeout_ns;
     a.stall_test = stall_test;
     const int grid = a.n_tiles < sms[dev] ? a.n_tiles : sms[dev];
-    gemm_tc_kernel<<<grid, kThreads, tc_smem_bytes(), s>>>(map, a);
+    if (debug_partials)
+        gemm_tc_kernel<true><<<grid, kThreads, tc_smem_bytes(), s>>>(map, a);
+    else
+        gemm_tc_kernel<false><<<grid, kThreads, tc_smem_bytes(), s>>>(map, a);
     return cudaGetLastError();
 }
 

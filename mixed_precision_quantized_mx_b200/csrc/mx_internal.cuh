@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/mx.h"
+#include "mx.h"
 
 namespace mx {
 
