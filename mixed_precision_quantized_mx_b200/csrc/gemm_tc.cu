@@ -25,7 +25,10 @@
 // what keeps the tensor cores fed.
 // Warp roles (512 threads):
 //   warp 0      weight copies           warp 3      activation copies
-//   warp 1      MMA issuer (one thread) warp 2      TMEM allocator
+//   warps 1, 2  MMA issuers, one thread each, taking alternate groups: a thread
+//               spends ~150 ns in every barrier wait or commit, about as long as
+//               one group's MMAs take, so two of them keep the tensor core busy
+//               (warp 2 also allocates TMEM)
 //   warps 4-7   widening (step one for 4-bit rows): uint4 codes -> int8 (q - z)
 //               in place, four codes per 32-bit operation (the vsub4 idea of
 //               section 3.3, done with a biased add)
@@ -57,16 +60,17 @@ constexpr int kEpiWarps = 8;
 constexpr int kAccBufs = 4;                     // int32 group accumulators in TMEM
 constexpr uint32_t kTmemCols = kAccBufs * BN;   // all 512 columns
 constexpr int kWidenBarrier = 1;                // named barrier of the widening warps
+constexpr int kMmaIssuers = 2;                  // MMA-issuing threads, alternating groups
 
 struct __align__(1024) Smem {
     uint8_t A[kStages][kKbPerStage * kABytes];  // raw uint4 codes land at A + kABytes
     uint8_t B[kStages][kKbPerStage * kBBytes];
     uint64_t full[kStages];       // both copies of the stage landed (2 arrivals + bytes)
     uint64_t wdone[kStages];      // widen -> MMA: weight operand ready
-    uint64_t empty[kStages];      // MMA -> loaders: stage consumed
+    uint64_t empty[kStages];      // MMA issuers -> loaders: stage consumed (one commit each)
     uint64_t acc_full[kAccBufs];  // MMA -> epilogue: group accumulator complete
     uint64_t acc_empty[kAccBufs]; // epilogue -> MMA: accumulator drained and re-armed
-    uint64_t mma_done;
+    uint64_t mma_done[kMmaIssuers];
     uint32_t tmem_base;
     int abort;
 };
@@ -117,13 +121,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&S.full[s], 2);
             mbar_init(&S.wdone[s], kWidenThreads / 32);
-            mbar_init(&S.empty[s], 1);
+            mbar_init(&S.empty[s], kMmaIssuers);
         }
         for (int b = 0; b < kAccBufs; ++b) {
             mbar_init(&S.acc_full[b], 1);
             mbar_init(&S.acc_empty[b], kEpiWarps);
         }
-        mbar_init(&S.mma_done, 1);
+        for (int m = 0; m < kMmaIssuers; ++m) mbar_init(&S.mma_done[m], 1);
         S.abort = 0;
         fence_mbar_init();
         prefetch_tensormap(&amap);
@@ -179,9 +183,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         load_done:
             drain_stages(S, it, a.timeout_ns);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 2) {
+        // ------------------------------------------------------------ MMA issuers
         if (lane == 0) {
+            const uint32_t mine = warp - 1;              // this issuer takes groups gc % 2 == mine
             const uint32_t idesc = idesc_i8(BM, BN);
             int it = 0;
             uint32_t gc = 0;
@@ -197,6 +202,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                         const uint32_t a0 = smem_u32(S.A[s] + kbi * kABytes);
                         const uint32_t b0 = smem_u32(S.B[s] + kbi * kBBytes);
                         for (int j = 0; j < gpk; ++j, ++gc) {
+                            if ((gc & 1) != mine) continue;
                             const uint32_t b = gc % kAccBufs, u = gc / kAccBufs;
                             if (!mbar_wait_bounded(&S.acc_empty[b], (u & 1) ^ 1, abort, a.status, a.timeout_ns))
                                 goto mma_out;
@@ -209,13 +215,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                             mma_commit(&S.acc_full[b]);
                         }
                     }
-                    mma_commit(&S.empty[s]);
+                    mma_commit(&S.empty[s]);   // arrives once this issuer's MMAs on the stage are done
                 }
             }
         mma_out:
-            mma_commit(&S.mma_done);      // all MMAs issued so far complete before teardown
+            mma_commit(&S.mma_done[mine]);  // all MMAs issued so far complete before teardown
             int dummy = 0;
-            mbar_wait_bounded(&S.mma_done, 0, &dummy, nullptr, a.timeout_ns);
+            mbar_wait_bounded(&S.mma_done[mine], 0, &dummy, nullptr, a.timeout_ns);
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ widening (4-bit rows)

@@ -310,3 +310,15 @@ def test_gemm_tc_llama_shapes_sampled(orc, M, K, N):
     pn = rng.integers(0, N, 1024)
     yr = orc.gemm(Aq_o, sa_o, c, pairs=(pm, pn))[1]
     assert_y_close(Yh[pm, pn], yr, rows_rms=np.sqrt(np.mean(y0 ** 2)))
+
+
+@pytest.mark.parametrize("K", [128, 384, 640])
+@pytest.mark.parametrize("g", [64, 128])
+def test_gemm_tc_odd_kblocks(orc, K, g):
+    # an odd number of 128-column k-blocks leaves the last pipeline stage half filled
+    rng = np.random.default_rng(K + g)
+    M, N = 150, 260
+    X = inputs.activations(rng, M, K, 3)
+    W = inputs.weights(rng, N, K, outlier_frac=0.002)
+    is8 = inputs.saliency_mask(np.abs(rng.standard_normal(N)), 30)
+    run_and_check(orc, X, W, is8, g, path=mx.PATH_TENSOR)
