@@ -382,7 +382,7 @@ def main():
             traffic = rec["dram_bytes_per_launch"]
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": "mx_gemm (split-K + reduce)" if path_used == 1 else "mx_gemm (tcgen05)",
+                "kernel": "gemm_decode_kernel (cluster split-K, CUDA cores)" if path_used == 1 else "gemm_tc_kernel (tcgen05)",
                 "algorithmic_per_launch": algo, "launch_ms": gemm_ms,
                 "peak_source": (f"{peaks['source']} HBM copy" if bound == "hbm" else
                                 f"{peaks['source']} bf16 cuBLAS burst x 2 (nominal int8/bf16 ratio)")}
@@ -428,7 +428,7 @@ def main():
         cpu = {"value": units_per_step * frac / sec, "unit": unit, "cores": 1, "kind": "oracle",
                "sample": f"{done} steps, each: quantize {M}x{K} activations + {desc}"}
 
-    kernels_per_step = 1 + (2 if path_used == 1 else 1)
+    kernels_per_step = 2                       # activation quantizer + GEMM
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K_steps,
         "warmup": a.warmup, "ms_per_step": ms / K_steps, "higher_is_better": True,

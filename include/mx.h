@@ -98,7 +98,8 @@ typedef struct mx_layout {
 /* Options of mx_gemm; pass NULL for the defaults (all fields zero). */
 typedef struct mx_gemm_opts {
     int32_t path;              /* 0 auto; 1 split-K CUDA-core path; 2 tensor-core path */
-    int32_t split;             /* split-K factor for 4-bit tiles (0 = auto); path 1 */
+    int32_t split;             /* path 1: CTAs (a thread-block cluster, 1..8) that split
+                                  the K range of each row unit (0 = auto) */
     int32_t* debug_partials;   /* device int32 [M][N][G] or NULL: every per-group
                                   int32 partial P[m][n][g] (original row order) */
     int32_t* status;           /* device int32 or NULL: kernel-side error code */
@@ -169,7 +170,9 @@ mx_status mx_quant_act(const void* X, mx_dtype xdtype, int M, int K, int64_t ldx
 
 /*
  * mx_gemm_workspace_size -- host only.  Bytes of device workspace mx_gemm
- * needs for this layer at M tokens with these options (0 if none).
+ * needs for this layer at M tokens with these options.  Both GEMM paths of this
+ * version run without scratch memory, so it reports 0; callers that size and
+ * pass a workspace stay correct if a later version needs one.
  */
 mx_status mx_gemm_workspace_size(const mx_layout* L, int M, const mx_gemm_opts* opts,
                                  size_t* bytes);
@@ -177,7 +180,9 @@ mx_status mx_gemm_workspace_size(const mx_layout* L, int M, const mx_gemm_opts* 
 /*
  * mx_gemm_select_path -- host only.  The GEMM path mx_gemm will take for this
  * layer at M tokens with these options: 1 = split-K CUDA-core path (decode-sized
- * M, HBM-bound), 2 = tensor-core path.  Negative mx_status on bad arguments.
+ * M <= 16, HBM-bound; the K split of each row unit is one thread-block cluster
+ * reduced through distributed shared memory), 2 = tensor-core path.  Negative
+ * mx_status on bad arguments.
  */
 int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts);
 
@@ -188,7 +193,8 @@ int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts);
  *   Aq      device int8 [M][K] row-major (dense); s_a device fp16 bits [M]
  *   Y       device fp16 [M][ldy], ldy >= N; column n is original row n of W
  *   workspace / ws_bytes: device scratch of at least
- *           mx_gemm_workspace_size(L, M, opts) bytes (may be NULL if 0)
+ *           mx_gemm_workspace_size(L, M, opts) bytes (may be NULL if 0; unused
+ *           by this version)
  * Per group g: P = sum_{k in g} Aq[m,k] (W_q[n,k] - z[n,g]) exactly in int32
  * (|P| <= 127*127*128 < 2^22), acc[m,n] = sum_g float(P) * s_w[n,g] in fp32,
  * then Y[m,n] = fp16_rn(acc * s_a[m]).  The fp32 summation order depends on the

@@ -166,9 +166,9 @@ mx_status mx_quant_act(const void* X, mx_dtype xdtype, int M, int K, int64_t ldx
 constexpr int kDecodeMaxM = 16;
 
 static int choose_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
-    (void)L;
     if (opts && opts->path) return opts->path;
-    return M <= kDecodeMaxM ? 1 : 2;
+    if (M <= kDecodeMaxM && mx::plan_decode(*L, M, 0).ok) return 1;
+    return 2;
 }
 
 int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
@@ -183,9 +183,8 @@ mx_status mx_gemm_workspace_size(const mx_layout* L, int M, const mx_gemm_opts* 
     if (st != MX_OK) return st;
     if (bytes == nullptr) return fail(MX_ERR_INVALID_ARG, "bytes is NULL");
     if (M < 0) return fail(MX_ERR_INVALID_ARG, "M=%d", M);
-    *bytes = 0;
-    if (M == 0) return MX_OK;
-    if (choose_path(L, M, opts) == 1) *bytes = mx::plan_splitk(*L, M, opts ? opts->split : 0).ws_bytes;
+    *bytes = 0;   // both paths run without scratch memory
+    (void)opts;
     return MX_OK;
 }
 
@@ -209,14 +208,14 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
     const int path = choose_path(L, M, opts);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (path == 1) {
-        mx::SplitPlan plan = mx::plan_splitk(*L, M, opts ? opts->split : 0);
-        if (ws_bytes < plan.ws_bytes || (plan.ws_bytes && workspace == nullptr))
-            return fail(MX_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.ws_bytes, ws_bytes);
-        if ((st = check_device_ptr(workspace, "workspace")) != MX_OK) return st;
-        if (!aligned16(workspace)) return fail(MX_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
-        cudaError_t e = mx::launch_gemm_splitk(*L, blob, Aq, s_a, M, Y, ldy, static_cast<float*>(workspace),
-                                               plan, opts ? opts->debug_partials : nullptr, s);
-        if (e != cudaSuccess) return cuda_fail(e, "split-K GEMM launch");
+        if (opts && opts->split > 8) return fail(MX_ERR_UNSUPPORTED, "split=%d above the cluster limit 8", opts->split);
+        mx::DecodePlan plan = mx::plan_decode(*L, M, opts ? opts->split : 0);
+        if (!plan.ok)
+            return fail(MX_ERR_UNSUPPORTED, "M=%d K=%d: activation slice too large for the decode path", M, L->K);
+        cudaError_t e = mx::launch_gemm_decode(*L, blob, Aq, s_a, M, Y, ldy, plan,
+                                               opts ? opts->debug_partials : nullptr,
+                                               opts ? opts->status : nullptr, s);
+        if (e != cudaSuccess) return cuda_fail(e, "decode GEMM launch");
         return MX_OK;
     }
     if (path == 2) {

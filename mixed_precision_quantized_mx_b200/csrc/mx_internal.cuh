@@ -52,20 +52,21 @@ cudaError_t launch_pack(const mx_layout& L, const void* W, mx_dtype wdt, int64_t
 cudaError_t launch_quant_act(const void* X, mx_dtype xdt, int M, int K, int64_t ldx,
                              int8_t* Aq, uint16_t* s_a, cudaStream_t s);
 
-struct SplitPlan {
+struct DecodePlan {
     int mt;             // tokens per CTA (1, 2, 4, 8, 16)
     int m_tiles;        // ceil(M / mt)
-    int kbu8, kbu4;     // k-blocks per unit in 8-bit / 4-bit tiles
-    int s8, s4;         // units per 8-bit / 4-bit tile
-    int units;          // t8 * s8 + t4 * s4
-    size_t ws_bytes;    // fp32 partial outputs
+    int units;          // 2 * t8 + t4: 64-row 8-bit units and 128-row 4-bit units
+    int S;              // CTAs per unit = cluster size (split of K)
+    int kbu;            // k-blocks per CTA
+    bool ok;            // the activation slice fits in shared memory
+    size_t smem;        // dynamic shared memory per CTA
 };
 
-SplitPlan plan_splitk(const mx_layout& L, int M, int split_hint);
+DecodePlan plan_decode(const mx_layout& L, int M, int split_hint);
 
-cudaError_t launch_gemm_splitk(const mx_layout& L, const void* blob, const int8_t* Aq,
+cudaError_t launch_gemm_decode(const mx_layout& L, const void* blob, const int8_t* Aq,
                                const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy,
-                               float* ws, const SplitPlan& plan, int32_t* debug_partials,
+                               const DecodePlan& plan, int32_t* debug_partials, int32_t* status,
                                cudaStream_t s);
 
 cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* Aq,

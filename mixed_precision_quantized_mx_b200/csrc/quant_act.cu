@@ -57,6 +57,12 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 quant_act_kernel(const T* __restrict__ X, int K, int64_t ldx, int8_t* __restrict__ Aq,
                  __half* __restrict__ s_a) {
+    // This grid may be launched as a programmatic dependent of the previous kernel
+    // (for example the GEMM that produced X): wait for it before reading anything.
+    // Then let the GEMM that consumes Aq launch and start streaming its weights; it
+    // waits for this grid to finish before reading Aq.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     const int m = blockIdx.x;
     const T* x = X + int64_t(m) * ldx;
     const int nvec = K / Vec<T>::kElems;
@@ -107,14 +113,19 @@ quant_act_kernel(const T* __restrict__ X, int K, int64_t ldx, int8_t* __restrict
 cudaError_t launch_quant_act(const void* X, mx_dtype xdt, int M, int K, int64_t ldx,
                              int8_t* Aq, uint16_t* s_a, cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    dim3 grid(M), block(kThreads);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(M);
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // resident early, waits in-kernel
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    __half* sa = reinterpret_cast<__half*>(s_a);
     if (xdt == MX_F16)
-        quant_act_kernel<__half><<<grid, block, 0, s>>>(static_cast<const __half*>(X), K, ldx,
-                                                        Aq, reinterpret_cast<__half*>(s_a));
-    else
-        quant_act_kernel<float><<<grid, block, 0, s>>>(static_cast<const float*>(X), K, ldx,
-                                                       Aq, reinterpret_cast<__half*>(s_a));
-    return cudaGetLastError();
+        return cudaLaunchKernelEx(&cfg, quant_act_kernel<__half>, static_cast<const __half*>(X), K, ldx, Aq, sa);
+    return cudaLaunchKernelEx(&cfg, quant_act_kernel<float>, static_cast<const float*>(X), K, ldx, Aq, sa);
 }
 
 }  // namespace mx

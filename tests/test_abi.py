@@ -119,8 +119,14 @@ def test_host_argument_checks_before_any_launch(lib):
     assert n.value == 0
 
 
-def test_split_workspace_is_sized_on_host(lib):
+def test_paths_need_no_workspace_and_dispatch_on_m(lib):
     L = mx.mx_layout_init(4096, 4096, 128, 410)
-    w1 = mx.mx_gemm_workspace_size(L, 1, path=mx.PATH_SPLITK)
-    w16 = mx.mx_gemm_workspace_size(L, 16, path=mx.PATH_SPLITK)
-    assert w1 > 0 and w16 == 16 * w1 and w1 % (128 * 4) == 0
+    for M in (1, 16, 17, 2048):
+        assert mx.mx_gemm_workspace_size(L, M) == 0
+    assert mx.mx_gemm_select_path(L, 1) == mx.PATH_SPLITK
+    assert mx.mx_gemm_select_path(L, 16) == mx.PATH_SPLITK
+    assert mx.mx_gemm_select_path(L, 17) == mx.PATH_TENSOR
+    assert mx.mx_gemm_select_path(L, 1, path=mx.PATH_TENSOR) == mx.PATH_TENSOR
+    # 16 tokens of a 64K-column activation slice cannot be staged per cluster: tensor cores
+    Lbig = mx.mx_layout_init(1024, 65536, 128, 102)
+    assert mx.mx_gemm_select_path(Lbig, 16) == mx.PATH_TENSOR

@@ -233,19 +233,18 @@ def test_gemm_rejects_bad_arguments(orc):
     Aq, sa = gpu_quant(X)
     L, blob = gpu_pack(W, is8, 128)
     Y = torch.empty((2, 140), dtype=torch.float16, device=dev())
-    need = mx.mx_gemm_workspace_size(L, 2, path=mx.PATH_SPLITK)
-    small = torch.empty(need - 16, dtype=torch.uint8, device=dev())
-    with pytest.raises(mx.MXError) as e:
-        mx.mx_gemm(L, blob, Aq, sa, Y, workspace=small, path=mx.PATH_SPLITK)
-    assert e.value.status == 7
-    ws = torch.empty(need, dtype=torch.uint8, device=dev())
+    assert mx.mx_gemm_workspace_size(L, 2, path=mx.PATH_SPLITK) == 0
+    ws = None
     with pytest.raises(mx.MXError) as e:                      # host memory is refused
-        mx.mx_gemm(L, blob, Aq.cpu(), sa, Y, workspace=ws, path=mx.PATH_SPLITK)
+        mx.mx_gemm(L, blob, Aq.cpu(), sa, Y, path=mx.PATH_SPLITK)
     assert e.value.status == 1
+    with pytest.raises(mx.MXError) as e:                      # cluster split above 8
+        mx.mx_gemm(L, blob, Aq, sa, Y, path=mx.PATH_SPLITK, split=9)
+    assert e.value.status == 2
     raw = torch.empty(2 * 256 + 16, dtype=torch.uint8, device=dev())
     Aq_mis = raw[1:1 + 512].view(torch.int8).view(2, 256)
     with pytest.raises(mx.MXError) as e:
-        mx.mx_gemm(L, blob, Aq_mis, sa, Y, workspace=ws, path=mx.PATH_SPLITK)
+        mx.mx_gemm(L, blob, Aq_mis, sa, Y, path=mx.PATH_SPLITK)
     assert e.value.status == 3
     Xh = torch.from_numpy(X)
     with pytest.raises(mx.MXError) as e:
