@@ -175,6 +175,25 @@ def time_oracle(lay, canonical, steps: int, min_seconds: float = 0.0):
     return (time.perf_counter() - t0) / done, desc, frac, done
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Largest value of x over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" \
+            else torch.device("cpu")
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own batch and layer (weak scaling: fixed work per GPU)."""
+    return seed + 1000003 * rank
+
+
 def step_units(M, K, N, g, n8, unit):
     from mixed_precision_quantized_mx_b200 import model
     if unit == "GB/s":
@@ -237,7 +256,7 @@ def main():
 
     M, K, N = WORKLOADS[a.workload]
     g = a.group
-    lay = inputs.llama_layer(M, K, N, a.frac8, g, seed=a.seed + rank)   # each rank its own batch
+    lay = inputs.llama_layer(M, K, N, a.frac8, g, seed=rank_seed(a.seed, rank))
     n8 = lay.n8
     L = mx.mx_layout_init(N, K, g, n8)
     unit = "GB/s" if M <= HBM_BOUND_MAX_M else "TOPS"
@@ -342,11 +361,7 @@ def main():
     if world > 1:
         dist.barrier()
     sampler.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     units_per_step = step_units(M, K, N, g, n8, unit)
     value = units_per_step * K_steps * world / (ms / 1e3)
 
@@ -406,11 +421,7 @@ def main():
         Ypin.copy_(layer(Xdev, path=a.path), non_blocking=True)
     f1.record()
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / Ke
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / Ke, dev)
     e2e = {"value": units_per_step * world / (e2e_ms / 1e3), "unit": unit,
            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
            "ms_per_step": e2e_ms, "api": "MixedPrecisionLinear.forward (eager, per-call launches)"}
