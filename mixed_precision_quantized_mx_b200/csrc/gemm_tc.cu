@@ -61,6 +61,7 @@ constexpr int kAccBufs = 4;                     // int32 group accumulators in T
 constexpr uint32_t kTmemCols = kAccBufs * BN;   // all 512 columns
 constexpr int kWidenBarrier = 1;                // named barrier of the widening warps
 constexpr int kMmaIssuers = 2;                  // MMA-issuing threads, alternating groups
+constexpr int kScaleRing = 4;                   // group scales in flight per epilogue thread
 
 struct __align__(1024) Smem {
     uint8_t A[kStages][kKbPerStage * kABytes];  // raw uint4 codes land at A + kABytes
@@ -232,37 +233,31 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             const bool eight = rt < g.t8;
             const int lt = eight ? rt : rt - g.t8;
             const uint8_t* zrow = g.zeros4 + size_t(lt) * g.G * kTileRows;
-            // zero points of this thread's four chunks in k-block kb, as (128 - z) per byte
-            auto load_z = [&](int kb, uint32_t (&zc)[4]) {
+            // zero points of this thread's four chunks in the two k-blocks of stage sp, as
+            // (128 - z) per byte; two register sets alternate between even and odd stages
+            // so each is loaded two stages before its use
+            auto load_z = [&](int sp, uint32_t (&zc)[2][4]) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int i = wt + kWidenThreads * j, r = i >> 2, c = i & 3;
-                    const int gi = (kb * kKBlock + c * 32) / g.group;
-                    zc[j] = (0x80u - uint32_t(zrow[size_t(gi) * kTileRows + r])) * 0x01010101u;
-                }
+                for (int kbi = 0; kbi < kKbPerStage; ++kbi)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int kb = sp * kKbPerStage + kbi;
+                        const int i = wt + kWidenThreads * j, r = i >> 2, c = i & 3;
+                        const int gi = (kb * kKBlock + c * 32) / g.group;
+                        zc[kbi][j] = kb < g.kblocks
+                            ? (0x80u - uint32_t(zrow[size_t(gi) * kTileRows + r])) * 0x01010101u : 0u;
+                    }
             };
-            uint32_t z0[4] = {0, 0, 0, 0}, z1[4] = {0, 0, 0, 0};
-            if (!eight) {
-                load_z(0, z0);
-                if (g.kblocks > 1) load_z(1, z1);
-            }
-            for (int sp = 0; sp < n_ss; ++sp, ++it) {
+            // one stage: wait for its copies, widen the uint4 codes in place, release it
+            auto widen_stage = [&](int sp, const uint32_t (&zc)[2][4]) -> bool {
                 const int s = it % kStages;
                 const uint32_t ph = (it / kStages) & 1;
-                const int kb0 = sp * kKbPerStage;
-                const int nkb = min(kKbPerStage, g.kblocks - kb0);
-                uint32_t zc0[4], zc1[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) { zc0[j] = z0[j]; zc1[j] = z1[j]; }
-                if (!eight) {                       // next stage's zero points, in flight now
-                    if (kb0 + 2 < g.kblocks) load_z(kb0 + 2, z0);
-                    if (kb0 + 3 < g.kblocks) load_z(kb0 + 3, z1);
-                }
+                const int nkb = min(kKbPerStage, g.kblocks - sp * kKbPerStage);
                 const bool ok = mbar_wait_bounded(&S.full[s], ph, abort, a.status, a.timeout_ns);
                 __syncwarp();   // the named barrier is warp-collective
                 // one decision for all 128 widening threads: the in-place conversion below
                 // needs every one of them at the named barrier
-                if (!named_bar_and(kWidenBarrier, kWidenThreads, ok)) goto widen_done;
+                if (!named_bar_and(kWidenBarrier, kWidenThreads, ok)) return false;
                 if (!eight) {
                     const uint8_t* raw = S.A[s] + kABytes;
                     for (int kbi = 0; kbi < nkb; ++kbi) {
@@ -276,7 +271,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const int i = wt + kWidenThreads * j, r = i >> 2, c = i & 3;
-                            const uint32_t z = kbi ? zc1[j] : zc0[j];
+                            const uint32_t z = kbi ? zc[1][j] : zc[0][j];
                             uint4 o0, o1;
                             o0.x = widen_lo(w[j].x, z); o0.y = widen_hi(w[j].x, z);
                             o0.z = widen_lo(w[j].y, z); o0.w = widen_hi(w[j].y, z);
@@ -290,6 +285,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.wdone[s]);
+                ++it;
+                return true;
+            };
+            uint32_t zA[2][4] = {}, zB[2][4] = {};
+            if (!eight) {
+                load_z(0, zA);
+                if (n_ss > 1) load_z(1, zB);
+            }
+            for (int sp = 0; sp < n_ss; sp += 2) {
+                if (!widen_stage(sp, zA)) goto widen_done;
+                if (!eight && sp + 2 < n_ss) load_z(sp + 2, zA);
+                if (sp + 1 < n_ss) {
+                    if (!widen_stage(sp + 1, zB)) goto widen_done;
+                    if (!eight && sp + 3 < n_ss) load_z(sp + 3, zB);
+                }
             }
         }
     widen_done:;
@@ -310,53 +320,62 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             float2 acc[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) acc[c] = make_float2(0.0f, 0.0f);
-            // group scales are fetched two groups ahead of their use
-            float sw_n1 = __half2float(sc[0]);
-            float sw_n2 = g.G > 1 ? __half2float(sc[kTileRows]) : 0.0f;
-            for (int gi = 0; gi < g.G; ++gi, ++gc) {
-                const float sw = sw_n1;
-                sw_n1 = sw_n2;
-                sw_n2 = gi + 2 < g.G ? __half2float(sc[size_t(gi + 2) * kTileRows]) : 0.0f;
-                const float2 s2 = make_float2(sw, sw);
-                const uint32_t b = gc % kAccBufs, u = gc / kAccBufs;
-                // every lane waits; the warp leaves together if any lane gave up, because
-                // the TMEM loads below are warp-collective (.sync.aligned)
-                const bool ok = mbar_wait_bounded(&S.acc_full[b], u & 1, abort, a.status, a.timeout_ns);
-                if (!__all_sync(0xffffffffu, ok)) goto epi_done;
-                tc_fence_after();
-                // drain the group's 64 columns in four 16-column chunks, loading chunk
-                // h+1 while chunk h is converted; each chunk is re-armed with the bias
-                const uint32_t col0 = lane_addr + b * BN + cb;
-                uint32_t va[16], vb[16];
-                tmem_ld_x16(col0, va);
-                tmem_wait_ld();
+            // group scales live in a ring of kScaleRing registers, each loaded kScaleRing
+            // groups before its use; the group loop is unrolled by kScaleRing so every
+            // ring slot is a fixed register and no instruction waits on a young load
+            float swr[kScaleRing];
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    uint32_t (&v)[16] = (h & 1) ? vb : va;
-                    uint32_t (&vn)[16] = (h & 1) ? va : vb;
-                    if (h < 3) tmem_ld_x16(col0 + (h + 1) * 16, vn);
-                    tmem_st_x16_splat(col0 + h * 16, kI2FBiasBits);
-                    // acc += (float(bias + P) - bias) * s_w, two columns per instruction
+            for (int j = 0; j < kScaleRing; ++j)
+                swr[j] = j < g.G ? __half2float(sc[size_t(j) * kTileRows]) : 0.0f;
+            for (int gi0 = 0; gi0 < g.G; gi0 += kScaleRing) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const float2 f = add2(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])),
-                                              nbias);
-                        acc[h * 8 + c] = fma2(f, s2, acc[h * 8 + c]);
-                    }
-                    if (DEBUG && orig >= 0) {
+                for (int j = 0; j < kScaleRing; ++j) {
+                    const int gi = gi0 + j;
+                    if (gi >= g.G) break;
+                    const float sw = swr[j];
+                    if (gi + kScaleRing < g.G) swr[j] = __half2float(sc[size_t(gi + kScaleRing) * kTileRows]);
+                    const float2 s2 = make_float2(sw, sw);
+                    const uint32_t b = gc % kAccBufs, u = gc / kAccBufs;
+                    // every lane waits; the warp leaves together if any lane gave up, because
+                    // the TMEM loads below are warp-collective (.sync.aligned)
+                    const bool ok = mbar_wait_bounded(&S.acc_full[b], u & 1, abort, a.status, a.timeout_ns);
+                    if (!__all_sync(0xffffffffu, ok)) goto epi_done;
+                    tc_fence_after();
+                    // drain the group's 64 columns in four 16-column chunks, loading chunk
+                    // h+1 while chunk h is converted; each chunk is re-armed with the bias
+                    const uint32_t col0 = lane_addr + b * BN + cb;
+                    uint32_t va[16], vb[16];
+                    tmem_ld_x16(col0, va);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const int m = tt * BN + cb + h * 16 + c;
-                            if (m < a.M)
-                                a.debug[(size_t(m) * g.N + orig) * g.G + gi] = int32_t(v[c] - kI2FBiasBits);
+                    for (int h = 0; h < 4; ++h) {
+                        uint32_t (&v)[16] = (h & 1) ? vb : va;
+                        uint32_t (&vn)[16] = (h & 1) ? va : vb;
+                        if (h < 3) tmem_ld_x16(col0 + (h + 1) * 16, vn);
+                        tmem_st_x16_splat(col0 + h * 16, kI2FBiasBits);
+                        // acc += (float(bias + P) - bias) * s_w, two columns per instruction
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const float2 f = add2(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])),
+                                                  nbias);
+                            acc[h * 8 + c] = fma2(f, s2, acc[h * 8 + c]);
                         }
+                        if (DEBUG && orig >= 0) {
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) {
+                                const int m = tt * BN + cb + h * 16 + c;
+                                if (m < a.M)
+                                    a.debug[(size_t(m) * g.N + orig) * g.G + gi] = int32_t(v[c] - kI2FBiasBits);
+                            }
+                        }
+                        if (h < 3) tmem_wait_ld();
                     }
-                    if (h < 3) tmem_wait_ld();
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.acc_empty[b]);
+                    ++gc;
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.acc_empty[b]);
             }
             if (orig >= 0) {
 #pragma unroll

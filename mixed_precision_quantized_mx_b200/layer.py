@@ -72,3 +72,50 @@ class MixedPrecisionLinear:
         return Y
 
     __call__ = forward
+
+    def graphed(self, x_host: torch.Tensor, y_host: torch.Tensor | None = None, path: int = 0) -> "GraphedLinear":
+        """Capture host-in / host-out calls for this input buffer (see GraphedLinear)."""
+        return GraphedLinear(self, x_host, y_host, path)
+
+
+class GraphedLinear:
+    """A MixedPrecisionLinear call captured once as a CUDA graph for a fixed M.
+
+    The graph copies the pinned host input into the device, quantizes, runs the
+    GEMM and copies Y back into the pinned host output, so one `replay()` per
+    step is the whole host-to-host pass with a single launch from the host.
+    The caller rewrites `x_host` between replays and reads `y_host` after the
+    stream is synchronised (or after an event recorded after `replay()`).
+    """
+
+    def __init__(self, layer: MixedPrecisionLinear, x_host: torch.Tensor, y_host: torch.Tensor | None = None,
+                 path: int = 0):
+        if not x_host.is_pinned():
+            raise ValueError("x_host must be pinned host memory")
+        M, K = x_host.shape
+        dev = layer.blob.device
+        self.layer = layer
+        self.x_host = x_host
+        self.y_host = y_host if y_host is not None else torch.empty((M, layer.N), dtype=torch.float16).pin_memory()
+        self.x_dev = torch.empty((M, K), dtype=x_host.dtype, device=dev)
+        self.aq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        self.sa = torch.empty((M,), dtype=torch.float16, device=dev)
+        self.y_dev = torch.empty((M, layer.N), dtype=torch.float16, device=dev)
+        ws = layer.workspace(M, path)
+        self.stream = torch.cuda.Stream(dev)
+
+        def body():
+            self.x_dev.copy_(self.x_host, non_blocking=True)
+            mx.mx_quant_act(self.x_dev, self.aq, self.sa)
+            mx.mx_gemm(layer.layout, layer.blob, self.aq, self.sa, self.y_dev, workspace=ws, path=path)
+            self.y_host.copy_(self.y_dev, non_blocking=True)
+
+        with torch.cuda.stream(self.stream):        # configure kernels outside capture
+            body()
+        self.stream.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=self.stream):
+            body()
+
+    def replay(self) -> None:
+        self.graph.replay()
