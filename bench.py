@@ -197,7 +197,7 @@ def rank_seed(seed: int, rank: int) -> int:
 def step_units(M, K, N, g, n8, unit):
     from mixed_precision_quantized_mx_b200 import model
     if unit == "GB/s":
-        return model.step_bytes(M, N, K, g, n8, 2) / 1e9
+        return model.linear_bytes(M, N, K, g, n8, 2) / 1e9
     return model.gemm_ops(M, N, K) / 1e12
 
 
@@ -282,7 +282,7 @@ def main():
 
     # ---- rotated copies beyond L2
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    per_step = model.step_bytes(M, N, K, g, n8, 2)
+    per_step = model.linear_bytes(M, N, K, g, n8, 2)
     R = int(min(64, max(2, math.ceil(4 * l2 / per_step))))
     R = max(2, min(R, int(20e9 // max(per_step, 1))))
     Xh = torch.from_numpy(lay.X)
@@ -291,16 +291,20 @@ def main():
     Aqs = [torch.empty((M, K), dtype=torch.int8, device=dev) for _ in range(R)]
     sas = [torch.empty((M,), dtype=torch.float16, device=dev) for _ in range(R)]
     Ys = [torch.empty((M, N), dtype=torch.float16, device=dev) for _ in range(R)]
-    ws_bytes = mx.mx_gemm_workspace_size(L, M, path=a.path)
-    ws = torch.empty(max(16, ws_bytes), dtype=torch.uint8, device=dev)
+    ws_bytes = mx.mx_linear_workspace_size(L, M, torch.float16, path=a.path)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+    fused = ws_bytes == 0                      # one kernel quantizes X and multiplies
     path_used = mx.mx_gemm_select_path(L, M, path=a.path)
 
     def step(i):
-        mx.mx_quant_act(Xs[i], Aqs[i], sas[i])
-        mx.mx_gemm(L, blobs[i], Aqs[i], sas[i], Ys[i], workspace=ws, path=a.path)
+        mx.mx_linear(L, blobs[i], Xs[i], Ys[i], workspace=ws, path=a.path)
 
     def gemm_only(i):
-        mx.mx_gemm(L, blobs[i], Aqs[i], sas[i], Ys[i], workspace=ws, path=a.path)
+        mx.mx_gemm(L, blobs[i], Aqs[i], sas[i], Ys[i], path=a.path)
+
+    dominant = step if fused else gemm_only
+    for i in range(R):                          # codes the GEMM-only timing reads
+        mx.mx_quant_act(Xs[i], Aqs[i], sas[i])
 
     s = torch.cuda.Stream(dev)
     torch.cuda.synchronize()
@@ -365,9 +369,10 @@ def main():
     units_per_step = step_units(M, K, N, g, n8, unit)
     value = units_per_step * K_steps * world / (ms / 1e3)
 
-    # ---- dominant kernel: the GEMM call alone, timed live on its stream
+    # ---- dominant kernel: the fused kernel (the whole step) or the GEMM call alone,
+    # timed live on its stream
     nd = max(R, min(4 * R, 400))
-    g_gemm = capture(gemm_only, nd)
+    g_gemm = capture(dominant, nd)
     g_gemm.replay()
     torch.cuda.synchronize()
     d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -380,7 +385,7 @@ def main():
     gemm_ms = d0.elapsed_time(d1) / (3 * nd)
     peaks = load_peaks()
     if bound == "hbm":
-        algo = model.gemm_bytes(M, N, K, g, n8)
+        algo = model.linear_bytes(M, N, K, g, n8, 2) if fused else model.gemm_bytes(M, N, K, g, n8)
         achieved = algo / (gemm_ms / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         r_unit = "GB/s"
@@ -393,11 +398,14 @@ def main():
     tfile = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if os.path.exists(tfile):
         rec = json.load(open(tfile)).get(a.workload)
-        if rec and rec.get("src_digest") == src_digest() and rec.get("path") == path_used:
+        if (rec and rec.get("src_digest") == src_digest() and rec.get("path") == path_used
+                and rec.get("fused", False) == fused):
             traffic = rec["dram_bytes_per_launch"]
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": "gemm_decode_kernel (cluster split-K, CUDA cores)" if path_used == 1 else "gemm_tc_kernel (tcgen05)",
+                "kernel": ("gemm_decode_kernel, activation quantizer fused (cluster split-K, CUDA cores)"
+                           if fused else "gemm_decode_kernel (cluster split-K, CUDA cores)" if path_used == 1
+                           else "gemm_tc_kernel (tcgen05)"),
                 "algorithmic_per_launch": algo, "launch_ms": gemm_ms,
                 "peak_source": (f"{peaks['source']} HBM copy" if bound == "hbm" else
                                 f"{peaks['source']} bf16 cuBLAS burst x 2 (nominal int8/bf16 ratio)")}
@@ -406,7 +414,7 @@ def main():
     layer = MixedPrecisionLinear.from_blob(blob0)
     Xpin = Xh.pin_memory()
     Ypin = torch.empty((M, N), dtype=torch.float16).pin_memory()
-    runner = layer.graphed(Xpin, Ypin, path=a.path)        # H2D, quantize, GEMM, D2H: one graph
+    runner = layer.graphed(Xpin, Ypin, path=a.path)        # H2D, mx_linear, D2H: one graph
     Ke = max(20, min(K_steps, 5000))
     for _ in range(3):
         runner.replay()
@@ -423,7 +431,7 @@ def main():
     e2e = {"value": units_per_step * world / (e2e_ms / 1e3), "unit": unit,
            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
            "ms_per_step": e2e_ms,
-           "api": "MixedPrecisionLinear.graphed: pinned X -> device, quantize, GEMM, Y -> pinned, one graph per step"}
+           "api": "MixedPrecisionLinear.graphed: pinned X -> device, mx_linear, Y -> pinned, one graph per step"}
 
     clocks = sampler.summary(t_time0, t_time1) or sampler.summary(t_load0, t_load1)
     if clocks is not None and "error" not in clocks:
@@ -438,20 +446,20 @@ def main():
         cpu = {"value": units_per_step * frac / sec, "unit": unit, "cores": 1, "kind": "oracle",
                "sample": f"{done} steps, each: quantize {M}x{K} activations + {desc}"}
 
-    kernels_per_step = 2                       # activation quantizer + GEMM
+    kernels_per_step = 1 if fused else 2       # fused kernel, or activation quantizer + GEMM
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K_steps,
         "warmup": a.warmup, "ms_per_step": ms / K_steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": a.workload, "M": M, "K": K, "N": N, "group": g, "frac8": a.frac8,
-                   "n8": n8, "path": path_used,
+                   "n8": n8, "path": path_used, "fused_quantizer": fused,
                    "l2": f"inputs rotate over {R} copies ({R * per_step / 1e6:.0f} MB >= 4x the "
                          f"{l2 / 1e6:.0f} MB L2); no flush",
                    "graphs": "timed steps replayed from CUDA graphs"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": kernels_per_step * K_steps, "clocks": clocks,
         "tops": model.gemm_ops(M, N, K) * K_steps * world / (ms / 1e3) / 1e12,
-        "gbs": model.step_bytes(M, N, K, g, n8, 2) * K_steps * world / (ms / 1e3) / 1e9,
+        "gbs": model.linear_bytes(M, N, K, g, n8, 2) * K_steps * world / (ms / 1e3) / 1e9,
         "pack": {"ms": pack_ms, "weights_gb_per_s": (N * K * 4) / (pack_ms / 1e3) / 1e9},
     }
     if rank == 0:

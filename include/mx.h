@@ -205,6 +205,35 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
                   int M, uint16_t* Y, int64_t ldy, void* workspace, size_t ws_bytes,
                   const mx_gemm_opts* opts, void* stream);
 
+/*
+ * mx_linear_workspace_size -- host only.  Bytes of device scratch mx_linear
+ * needs at M tokens of activations of type xdtype: 0 when the call is served by
+ * the decode kernel that quantizes X itself, else room for Aq (M*K bytes) and
+ * s_a (2*M bytes), each rounded up to 16 bytes.
+ */
+mx_status mx_linear_workspace_size(const mx_layout* L, int M, mx_dtype xdtype,
+                                   const mx_gemm_opts* opts, size_t* bytes);
+
+/*
+ * mx_linear -- Y = X W^T for a packed layer in one call: per-token 8-bit
+ * quantization of X (MixLLM section 3.1.2) followed by the two-step
+ * dequantized GEMM (section 3.3).
+ *   X       device [M][ldx] fp32 or fp16 (xdtype), rows 16-byte aligned, ldx >= K
+ *   Y       device fp16 [M][ldy], ldy >= N; column n is original row n of W
+ *   workspace / ws_bytes: device scratch of at least mx_linear_workspace_size
+ *           bytes (may be NULL when that is 0)
+ * When the decode path serves the call (mx_gemm_select_path == 1), M <= 4 and
+ * the activation rows take at most 64 KB, one kernel does both steps: each CTA
+ * takes the absmax of the whole token row and quantizes only its own K slice,
+ * with the same operations as mx_quant_act, so the codes -- and Y -- are
+ * identical to mx_quant_act followed by mx_gemm.  Otherwise mx_quant_act and
+ * mx_gemm run back to back on `stream` with Aq and s_a in the workspace.
+ * Returns MX_ERR_WORKSPACE if the workspace is missing or too small.
+ */
+mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtype xdtype, int M,
+                    int64_t ldx, uint16_t* Y, int64_t ldy, void* workspace, size_t ws_bytes,
+                    const mx_gemm_opts* opts, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,7 @@ PATH_AUTO, PATH_SPLITK, PATH_TENSOR = 0, 1, 2
 
 EXPORTED = ("mx_version", "mx_last_error", "mx_layout_init", "mx_layout_from_header",
             "mx_pack_weights", "mx_quant_act", "mx_gemm_workspace_size", "mx_gemm_select_path",
-            "mx_gemm")
+            "mx_gemm", "mx_linear_workspace_size", "mx_linear")
 
 
 class MXError(RuntimeError):
@@ -76,8 +76,12 @@ def lib() -> ctypes.CDLL:
     L.mx_gemm_select_path.restype = I
     L.mx_gemm.argtypes = [ctypes.POINTER(Layout), P, P, P, I, P, I64, P, Z,
                           ctypes.POINTER(GemmOpts), P]
+    L.mx_linear_workspace_size.argtypes = [ctypes.POINTER(Layout), I, I, ctypes.POINTER(GemmOpts),
+                                           ctypes.POINTER(Z)]
+    L.mx_linear.argtypes = [ctypes.POINTER(Layout), P, P, I, I, I64, P, I64, P, Z,
+                            ctypes.POINTER(GemmOpts), P]
     for n in ("mx_layout_init", "mx_layout_from_header", "mx_pack_weights", "mx_quant_act",
-              "mx_gemm_workspace_size", "mx_gemm"):
+              "mx_gemm_workspace_size", "mx_gemm", "mx_linear_workspace_size", "mx_linear"):
         getattr(L, n).restype = I
     _lib = L
     return L
@@ -173,3 +177,25 @@ def mx_gemm(L: Layout, blob: torch.Tensor, Aq: torch.Tensor, s_a: torch.Tensor, 
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().mx_gemm(ctypes.byref(L), _ptr(blob), _ptr(Aq), _ptr(s_a), M, _ptr(Y), Y.stride(0),
                          _ptr(workspace), ws_bytes, ctypes.byref(o), _stream(stream)), "mx_gemm")
+
+
+def mx_linear_workspace_size(L: Layout, M: int, xdtype=torch.float16, path: int = 0, split: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    o = _opts(path, split)
+    code = MX_F16 if xdtype == torch.float16 else MX_F32
+    _check(lib().mx_linear_workspace_size(ctypes.byref(L), M, code, ctypes.byref(o), ctypes.byref(n)),
+           "mx_linear_workspace_size")
+    return n.value
+
+
+def mx_linear(L: Layout, blob: torch.Tensor, X: torch.Tensor, Y: torch.Tensor,
+              workspace: torch.Tensor | None = None, path: int = 0, split: int = 0,
+              debug_partials: torch.Tensor | None = None, status: torch.Tensor | None = None,
+              stream=None) -> None:
+    assert X.dim() == 2 and X.stride(1) == 1
+    M = X.shape[0]
+    o = _opts(path, split, debug_partials, status)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().mx_linear(ctypes.byref(L), _ptr(blob), _ptr(X), _dtype_code(X), M, X.stride(0),
+                           _ptr(Y), Y.stride(0), _ptr(workspace), ws_bytes, ctypes.byref(o),
+                           _stream(stream)), "mx_linear")

@@ -26,6 +26,7 @@
 // resident (and waiting) when this kernel finishes.
 #include <algorithm>
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "mx_internal.cuh"
 
@@ -42,8 +43,10 @@ constexpr int kMaxCluster = 8;             // portable cluster size
 
 struct DecArgs {
     Geom g;
-    const int8_t* Aq;
+    const int8_t* Aq;      // quantized activations (when the kernel is not fed X)
     const __half* s_a;
+    const void* X;         // raw activations fp16 / fp32 (when it quantizes them itself)
+    int64_t ldx;
     __half* Y;
     int64_t ldy;
     int M;
@@ -112,8 +115,12 @@ __host__ __device__ constexpr int decode_ctas_per_sm(int mt, int nb) {
 }
 
 // NB: register buffers of kBatch k-blocks (2 = the next batch streams while one
-// is computed; 1 when a CTA's whole K range is a single batch)
-template <int MT, int NB, bool DEBUG>
+// is computed; 1 when a CTA's whole K range is a single batch).
+// XT: void -- read Aq and s_a produced by the activation quantizer; __half or
+// float -- read X and quantize in-kernel: each CTA takes the absmax of the whole
+// row (the scale needs all K) and quantizes only its own K slice into shared
+// memory, with the quantizer's own device code, so the codes are identical.
+template <int MT, int NB, bool DEBUG, typename XT>
 __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(MT, NB))
 gemm_decode_kernel(const __grid_constant__ DecArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -179,19 +186,63 @@ gemm_decode_kernel(const __grid_constant__ DecArgs a) {
     cluster.sync();
     griddep_wait();
 
-    // ---- stage Aq[m0 .. m0+MT)[kb0*128 .. kb1*128) (zero rows beyond M)
     const int rowb = a.kbu * kKBlock;
     int8_t* act = reinterpret_cast<int8_t*>(smem);
     int32_t* sa64 = reinterpret_cast<int32_t*>(smem + size_t(MT) * rowb);
     // partial sums of every rank, [S][MT][128]; only rank 0's copy is used
     float* part = reinterpret_cast<float*>(smem + size_t(MT) * rowb + size_t(MT) * 2 * a.kbu * 4);
-    const int chunks = nkb * (kKBlock / 16);
-    for (int i = tid; i < MT * chunks; i += kThreads) {
-        const int j = i / chunks, c = i % chunks;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (m0 + j < a.M)
-            v = __ldg(reinterpret_cast<const uint4*>(a.Aq + int64_t(m0 + j) * g.K + kb0 * kKBlock) + c);
-        *reinterpret_cast<uint4*>(act + j * rowb + c * 16) = v;
+    __shared__ float sa_loc[MT];              // token scales quantized in-kernel
+    if constexpr (std::is_void_v<XT>) {
+        // ---- stage Aq[m0 .. m0+MT)[kb0*128 .. kb1*128) (zero rows beyond M)
+        const int chunks = nkb * (kKBlock / 16);
+        for (int i = tid; i < MT * chunks; i += kThreads) {
+            const int j = i / chunks, c = i % chunks;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (m0 + j < a.M)
+                v = __ldg(reinterpret_cast<const uint4*>(a.Aq + int64_t(m0 + j) * g.K + kb0 * kKBlock) + c);
+            *reinterpret_cast<uint4*>(act + j * rowb + c * 16) = v;
+        }
+    } else {
+        // ---- per-token absmax over the whole row, then this CTA's slice quantized
+        const XT* X = static_cast<const XT*>(a.X);
+        __shared__ float red[kThreads / 32][MT];
+        float am[MT];
+#pragma unroll
+        for (int j = 0; j < MT; ++j) {
+            am[j] = 0.0f;
+            if (m0 + j < a.M) {
+                const XT* x = X + int64_t(m0 + j) * a.ldx;
+                for (int v = tid; v < g.K / 8; v += kThreads) {
+                    float f[8];
+                    load8(x + v * 8, f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) am[j] = fmaxf(am[j], fabsf(f[e]));
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) am[j] = fmaxf(am[j], __shfl_xor_sync(0xffffffffu, am[j], o));
+            if ((tid & 31) == 0) red[tid >> 5][j] = am[j];
+        }
+        __syncthreads();
+        if (tid < MT) {
+            float m = red[0][tid];
+#pragma unroll
+            for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w][tid]);
+            sa_loc[tid] = __half2float(act_scale(m));
+        }
+        __syncthreads();
+        const int units8 = nkb * (kKBlock / 8);
+        for (int i = tid; i < MT * units8; i += kThreads) {
+            const int j = i / units8, c = i % units8;
+            uint2 o = make_uint2(0, 0);
+            if (m0 + j < a.M) {
+                float f[8];
+                load8(X + int64_t(m0 + j) * a.ldx + kb0 * kKBlock + c * 8, f);
+                o.x = quant4(f, sa_loc[j]);
+                o.y = quant4(f + 4, sa_loc[j]);
+            }
+            *reinterpret_cast<uint2*>(act + j * rowb + c * 8) = o;
+        }
     }
     __syncthreads();
     if (!eight) {
@@ -343,16 +394,18 @@ gemm_decode_kernel(const __grid_constant__ DecArgs a) {
         for (int q = 0; q < a.S; ++q) sum = __fadd_rn(sum, part[(size_t(q) * MT + j) * 128 + rr]);
         const int sl = eight ? tile * kTileRows + row0 + rr : (g.t8 + tile) * kTileRows + rr;
         const int o = g.rowmap[sl];
-        if (o >= 0)
-            a.Y[int64_t(m0 + j) * a.ldy + o] = __float2half_rn(__fmul_rn(sum, __half2float(a.s_a[m0 + j])));
+        float sa;
+        if constexpr (std::is_void_v<XT>) sa = __half2float(a.s_a[m0 + j]);
+        else sa = sa_loc[j];
+        if (o >= 0) a.Y[int64_t(m0 + j) * a.ldy + o] = __float2half_rn(__fmul_rn(sum, sa));
     }
 }
 
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-template <int MT, int NB, bool DEBUG>
+template <int MT, int NB, bool DEBUG, typename XT>
 cudaError_t launch_t(const DecArgs& args, int units, int m_tiles, size_t smem, cudaStream_t s) {
-    auto k = gemm_decode_kernel<MT, NB, DEBUG>;
+    auto k = gemm_decode_kernel<MT, NB, DEBUG, XT>;
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -380,20 +433,31 @@ cudaError_t launch_t(const DecArgs& args, int units, int m_tiles, size_t smem, c
     return cudaLaunchKernelEx(&cfg, k, args);
 }
 
-template <int MT, bool DEBUG>
+template <int MT, bool DEBUG, typename XT>
 cudaError_t launch_nb(const DecArgs& a, int units, int m_tiles, size_t smem, cudaStream_t s) {
-    return a.kbu <= kBatch ? launch_t<MT, 1, DEBUG>(a, units, m_tiles, smem, s)
-                           : launch_t<MT, 2, DEBUG>(a, units, m_tiles, smem, s);
+    return a.kbu <= kBatch ? launch_t<MT, 1, DEBUG, XT>(a, units, m_tiles, smem, s)
+                           : launch_t<MT, 2, DEBUG, XT>(a, units, m_tiles, smem, s);
 }
 
 template <bool DEBUG>
 cudaError_t launch_mt(const DecArgs& a, int mt, int units, int m_tiles, size_t smem, cudaStream_t s) {
     switch (mt) {
-        case 1: return launch_nb<1, DEBUG>(a, units, m_tiles, smem, s);
-        case 2: return launch_nb<2, DEBUG>(a, units, m_tiles, smem, s);
-        case 4: return launch_nb<4, DEBUG>(a, units, m_tiles, smem, s);
-        case 8: return launch_nb<8, DEBUG>(a, units, m_tiles, smem, s);
-        default: return launch_nb<16, DEBUG>(a, units, m_tiles, smem, s);
+        case 1: return launch_nb<1, DEBUG, void>(a, units, m_tiles, smem, s);
+        case 2: return launch_nb<2, DEBUG, void>(a, units, m_tiles, smem, s);
+        case 4: return launch_nb<4, DEBUG, void>(a, units, m_tiles, smem, s);
+        case 8: return launch_nb<8, DEBUG, void>(a, units, m_tiles, smem, s);
+        default: return launch_nb<16, DEBUG, void>(a, units, m_tiles, smem, s);
+    }
+}
+
+// in-kernel quantization of X: up to four tokens per CTA
+template <bool DEBUG, typename XT>
+cudaError_t launch_mt_fused(const DecArgs& a, int mt, int units, int m_tiles, size_t smem, cudaStream_t s) {
+    switch (mt) {
+        case 1: return launch_nb<1, DEBUG, XT>(a, units, m_tiles, smem, s);
+        case 2: return launch_nb<2, DEBUG, XT>(a, units, m_tiles, smem, s);
+        case 4: return launch_nb<4, DEBUG, XT>(a, units, m_tiles, smem, s);
+        default: return cudaErrorInvalidValue;
     }
 }
 
@@ -450,6 +514,35 @@ cudaError_t launch_gemm_decode(const mx_layout& L, const void* blob, const int8_
     a.status = status;
     return debug_partials ? launch_mt<true>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s)
                           : launch_mt<false>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s);
+}
+
+bool decode_can_fuse(const mx_layout& L, int M, mx_dtype xdt) {
+    // every CTA reads whole activation rows for the scales: keep that to 64 KB
+    return M >= 1 && M <= kMaxFusedTokens &&
+           size_t(M) * L.K * (xdt == MX_F16 ? 2 : 4) <= size_t(64) * 1024;
+}
+
+cudaError_t launch_gemm_decode_fused(const mx_layout& L, const void* blob, const void* X, mx_dtype xdt,
+                                     int64_t ldx, int M, uint16_t* Y, int64_t ldy, const DecodePlan& plan,
+                                     int32_t* debug_partials, int32_t* status, cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    if (plan.mt > kMaxFusedTokens) return cudaErrorInvalidValue;
+    DecArgs a{};
+    a.g = make_geom(L, blob);
+    a.X = X;
+    a.ldx = ldx;
+    a.Y = reinterpret_cast<__half*>(Y);
+    a.ldy = ldy;
+    a.M = M;
+    a.S = plan.S;
+    a.kbu = plan.kbu;
+    a.debug = debug_partials;
+    a.status = status;
+    if (xdt == MX_F16)
+        return debug_partials ? launch_mt_fused<true, __half>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s)
+                              : launch_mt_fused<false, __half>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s);
+    return debug_partials ? launch_mt_fused<true, float>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s)
+                          : launch_mt_fused<false, float>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s);
 }
 
 }  // namespace mx

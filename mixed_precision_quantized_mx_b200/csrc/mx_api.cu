@@ -234,4 +234,68 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
     return fail(MX_ERR_INVALID_ARG, "unknown GEMM path %d", path);
 }
 
+namespace {
+
+size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
+
+bool linear_fused(const mx_layout* L, int M, mx_dtype xdt, const mx_gemm_opts* opts) {
+    return choose_path(L, M, opts) == 1 && mx::decode_can_fuse(*L, M, xdt) &&
+           mx::plan_decode(*L, M, opts ? opts->split : 0).mt <= mx::kMaxFusedTokens;
+}
+
+}  // namespace
+
+mx_status mx_linear_workspace_size(const mx_layout* L, int M, mx_dtype xdtype, const mx_gemm_opts* opts,
+                                   size_t* bytes) {
+    mx_status st = check_layout(L);
+    if (st != MX_OK) return st;
+    if (bytes == nullptr) return fail(MX_ERR_INVALID_ARG, "bytes is NULL");
+    if (M < 0) return fail(MX_ERR_INVALID_ARG, "M=%d", M);
+    if (xdtype != MX_F32 && xdtype != MX_F16) return fail(MX_ERR_INVALID_ARG, "bad xdtype %d", int(xdtype));
+    *bytes = (M == 0 || linear_fused(L, M, xdtype, opts)) ? 0
+             : align16(size_t(M) * L->K) + align16(size_t(2) * M);
+    return MX_OK;
+}
+
+mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtype xdtype, int M,
+                    int64_t ldx, uint16_t* Y, int64_t ldy, void* workspace, size_t ws_bytes,
+                    const mx_gemm_opts* opts, void* stream) {
+    mx_status st = check_layout(L);
+    if (st != MX_OK) return st;
+    if (xdtype != MX_F32 && xdtype != MX_F16) return fail(MX_ERR_INVALID_ARG, "bad xdtype %d", int(xdtype));
+    if (M < 0) return fail(MX_ERR_INVALID_ARG, "M=%d", M);
+    if (ldx < L->K) return fail(MX_ERR_INVALID_ARG, "ldx=%lld < K=%d", (long long)ldx, L->K);
+    if (ldy < L->N) return fail(MX_ERR_INVALID_ARG, "ldy=%lld < N=%d", (long long)ldy, L->N);
+    if (M == 0) return MX_OK;
+    if (M > 65535) return fail(MX_ERR_UNSUPPORTED, "M=%d above 65535", M);
+    const int esz = xdtype == MX_F16 ? 2 : 4;
+    if ((st = check_device_ptr(X, "X")) != MX_OK) return st;
+    if (!aligned16(X) || (ldx * esz) % 16 != 0) return fail(MX_ERR_ALIGNMENT, "X and every X row must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (linear_fused(L, M, xdtype, opts)) {
+        if ((st = check_device_ptr(blob, "blob")) != MX_OK) return st;
+        if ((st = check_device_ptr(Y, "Y")) != MX_OK) return st;
+        if (!aligned16(blob)) return fail(MX_ERR_ALIGNMENT, "blob must be 16-byte aligned");
+        if (opts && opts->debug_partials && (st = check_device_ptr(opts->debug_partials, "debug_partials")) != MX_OK)
+            return st;
+        if (opts && opts->status && (st = check_device_ptr(opts->status, "status")) != MX_OK) return st;
+        if (opts && opts->split > 8) return fail(MX_ERR_UNSUPPORTED, "split=%d above the cluster limit 8", opts->split);
+        mx::DecodePlan plan = mx::plan_decode(*L, M, opts ? opts->split : 0);
+        cudaError_t e = mx::launch_gemm_decode_fused(*L, blob, X, xdtype, ldx, M, Y, ldy, plan,
+                                                     opts ? opts->debug_partials : nullptr,
+                                                     opts ? opts->status : nullptr, s);
+        if (e != cudaSuccess) return cuda_fail(e, "fused decode GEMM launch");
+        return MX_OK;
+    }
+    const size_t need = align16(size_t(M) * L->K) + align16(size_t(2) * M);
+    if (workspace == nullptr || ws_bytes < need)
+        return fail(MX_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace ? ws_bytes : size_t(0));
+    if ((st = check_device_ptr(workspace, "workspace")) != MX_OK) return st;
+    if (!aligned16(workspace)) return fail(MX_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+    int8_t* Aq = static_cast<int8_t*>(workspace);
+    uint16_t* s_a = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + align16(size_t(M) * L->K));
+    if ((st = mx_quant_act(X, xdtype, M, L->K, ldx, Aq, s_a, stream)) != MX_OK) return st;
+    return mx_gemm(L, blob, Aq, s_a, M, Y, ldy, nullptr, 0, opts, stream);
+}
+
 }  // extern "C"

@@ -25,6 +25,48 @@ __device__ __forceinline__ float i2f_biased(int32_t v) {
     return __fsub_rn(__int_as_float(int32_t(kI2FBiasBits) + v), kI2FBias);
 }
 
+// ---- 8-bit symmetric activation quantizer (MixLLM section 3.1.2; the symmetric
+// quantizer of section 2.1 with range +-127).  Shared by the standalone
+// quantizer and the GEMM that quantizes its own activation slice, so both take
+// every decision with the same IEEE operations.
+
+// eight consecutive elements as fp32 (16-byte aligned)
+__device__ __forceinline__ void load8(const __half* p, float (&v)[8]) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
+    const __half2* h = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// s_a = fp16(amax / 127), saturated at the largest finite fp16, 0 -> 1
+__device__ __forceinline__ __half act_scale(float amax) {
+    __half h = __float2half_rn(fminf(__fdiv_rn(amax, 127.0f), 65504.0f));
+    if (__half2float(h) == 0.0f) h = __float2half_rn(1.0f);
+    return h;
+}
+
+// four codes clamp(round_half_even(x / s), -127, 127) packed little-endian
+__device__ __forceinline__ uint32_t quant4(const float* v, float s) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float q = rintf(__fdiv_rn(v[i], s));
+        q = fminf(fmaxf(q, -127.0f), 127.0f);
+        w |= (uint32_t(int32_t(q)) & 0xFFu) << (8 * i);
+    }
+    return w;
+}
+
 // Byte offset of the 16-byte chunk holding k = 16c..16c+15 of row r inside a
 // 128-row x 128-byte block stored with the 128-byte swizzle.
 __device__ __forceinline__ int swz128_offset(int r, int c) {
@@ -68,6 +110,13 @@ cudaError_t launch_gemm_decode(const mx_layout& L, const void* blob, const int8_
                                const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy,
                                const DecodePlan& plan, int32_t* debug_partials, int32_t* status,
                                cudaStream_t s);
+
+// decode GEMM that quantizes X itself (M <= kMaxFusedTokens): one launch per call
+constexpr int kMaxFusedTokens = 4;
+bool decode_can_fuse(const mx_layout& L, int M, mx_dtype xdt);
+cudaError_t launch_gemm_decode_fused(const mx_layout& L, const void* blob, const void* X, mx_dtype xdt,
+                                     int64_t ldx, int M, uint16_t* Y, int64_t ldy, const DecodePlan& plan,
+                                     int32_t* debug_partials, int32_t* status, cudaStream_t s);
 
 cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* Aq,
                            const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy,

@@ -18,41 +18,6 @@ namespace {
 
 constexpr int kThreads = 256;
 
-template <typename T> struct Vec;
-template <> struct Vec<__half> {
-    static constexpr int kElems = 8;   // 16 bytes
-    __device__ static void load(const __half* p, float (&v)[8]) {
-        uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
-        const __half2* h = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float2 f = __half22float2(h[i]);
-            v[2 * i] = f.x;
-            v[2 * i + 1] = f.y;
-        }
-    }
-};
-template <> struct Vec<float> {
-    static constexpr int kElems = 8;   // two 16-byte loads
-    __device__ static void load(const float* p, float (&v)[8]) {
-        float4 a = __ldg(reinterpret_cast<const float4*>(p));
-        float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    }
-};
-
-__device__ __forceinline__ uint32_t quant4(const float* v, float s) {
-    uint32_t w = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float q = rintf(__fdiv_rn(v[i], s));
-        q = fminf(fmaxf(q, -127.0f), 127.0f);
-        w |= (uint32_t(int32_t(q)) & 0xFFu) << (8 * i);
-    }
-    return w;
-}
-
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 quant_act_kernel(const T* __restrict__ X, int K, int64_t ldx, int8_t* __restrict__ Aq,
@@ -65,12 +30,12 @@ quant_act_kernel(const T* __restrict__ X, int K, int64_t ldx, int8_t* __restrict
     asm volatile("griddepcontrol.launch_dependents;");
     const int m = blockIdx.x;
     const T* x = X + int64_t(m) * ldx;
-    const int nvec = K / Vec<T>::kElems;
+    const int nvec = K / 8;
 
     float amax = 0.0f;
     for (int i = threadIdx.x; i < nvec; i += kThreads) {
         float v[8];
-        Vec<T>::load(x + i * 8, v);
+        load8(x + i * 8, v);
 #pragma unroll
         for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
     }
@@ -84,15 +49,9 @@ quant_act_kernel(const T* __restrict__ X, int K, int64_t ldx, int8_t* __restrict
         float a = red[0];
 #pragma unroll
         for (int w = 1; w < kThreads / 32; ++w) a = fmaxf(a, red[w]);
-        // fp16 scale; values above the largest finite fp16 saturate to 65504
-        __half h = __float2half_rn(fminf(__fdiv_rn(a, 127.0f), 65504.0f));
-        float s = __half2float(h);
-        if (s == 0.0f) {
-            s = 1.0f;
-            h = __float2half_rn(1.0f);
-        }
+        const __half h = act_scale(a);
         s_a[m] = h;
-        s_shared = s;
+        s_shared = __half2float(h);
     }
     __syncthreads();
     const float s = s_shared;
@@ -100,7 +59,7 @@ quant_act_kernel(const T* __restrict__ X, int K, int64_t ldx, int8_t* __restrict
     int8_t* q = Aq + int64_t(m) * K;
     for (int i = threadIdx.x; i < nvec; i += kThreads) {
         float v[8];
-        Vec<T>::load(x + i * 8, v);
+        load8(x + i * 8, v);
         uint2 out;
         out.x = quant4(v, s);
         out.y = quant4(v + 4, s);

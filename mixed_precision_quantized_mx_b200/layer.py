@@ -1,8 +1,8 @@
 """MixedPrecisionLinear: the user-facing object around the C ABI.
 
 It owns the packed weight blob (torch device memory), sizes the workspace, and
-runs one forward pass as quantize-activations -> mixed-precision GEMM on the
-current CUDA stream.  All arithmetic happens in libmx.so's kernels.
+runs one forward pass with mx_linear (quantize activations, mixed-precision
+GEMM) on the current CUDA stream.  All arithmetic happens in libmx.so's kernels.
 """
 from __future__ import annotations
 
@@ -52,23 +52,20 @@ class MixedPrecisionLinear:
         if st != 0:
             raise mx.MXError(st, "mx_pack_weights", "device-side error while packing")
 
-    def workspace(self, M: int, path: int = 0) -> torch.Tensor | None:
-        key = (M, path)
+    def workspace(self, M: int, xdtype=torch.float16, path: int = 0) -> torch.Tensor | None:
+        """Device scratch for mx_linear at M tokens (None when it needs none); cached."""
+        key = (M, xdtype, path)
         if key not in self._ws:
-            n = mx.mx_gemm_workspace_size(self.layout, M, path=path)
-            self._ws[key] = torch.empty(max(n, 16), dtype=torch.uint8, device=self.blob.device) if n else None
+            n = mx.mx_linear_workspace_size(self.layout, M, xdtype, path=path)
+            self._ws[key] = torch.empty(n, dtype=torch.uint8, device=self.blob.device) if n else None
         return self._ws[key]
 
     def forward(self, X: torch.Tensor, out: torch.Tensor | None = None, path: int = 0) -> torch.Tensor:
         M, K = X.shape
         if K != self.K:
             raise ValueError(f"X has K={K}, layer expects {self.K}")
-        dev = self.blob.device
-        Aq = torch.empty((M, K), dtype=torch.int8, device=dev)
-        sa = torch.empty((M,), dtype=torch.float16, device=dev)
-        Y = out if out is not None else torch.empty((M, self.N), dtype=torch.float16, device=dev)
-        mx.mx_quant_act(X, Aq, sa)
-        mx.mx_gemm(self.layout, self.blob, Aq, sa, Y, workspace=self.workspace(M, path), path=path)
+        Y = out if out is not None else torch.empty((M, self.N), dtype=torch.float16, device=self.blob.device)
+        mx.mx_linear(self.layout, self.blob, X, Y, workspace=self.workspace(M, X.dtype, path), path=path)
         return Y
 
     __call__ = forward
@@ -81,8 +78,9 @@ class MixedPrecisionLinear:
 class GraphedLinear:
     """A MixedPrecisionLinear call captured once as a CUDA graph for a fixed M.
 
-    The graph copies the pinned host input into the device, quantizes, runs the
-    GEMM and copies Y back into the pinned host output, so one `replay()` per
+    The graph copies the pinned host input into the device, runs mx_linear
+    (quantize + GEMM, one kernel for decode-sized M) and copies Y back into the
+    pinned host output, so one `replay()` per
     step is the whole host-to-host pass with a single launch from the host.
     The caller rewrites `x_host` between replays and reads `y_host` after the
     stream is synchronised (or after an event recorded after `replay()`).
@@ -98,16 +96,13 @@ class GraphedLinear:
         self.x_host = x_host
         self.y_host = y_host if y_host is not None else torch.empty((M, layer.N), dtype=torch.float16).pin_memory()
         self.x_dev = torch.empty((M, K), dtype=x_host.dtype, device=dev)
-        self.aq = torch.empty((M, K), dtype=torch.int8, device=dev)
-        self.sa = torch.empty((M,), dtype=torch.float16, device=dev)
         self.y_dev = torch.empty((M, layer.N), dtype=torch.float16, device=dev)
-        ws = layer.workspace(M, path)
+        ws = layer.workspace(M, x_host.dtype, path)
         self.stream = torch.cuda.Stream(dev)
 
         def body():
             self.x_dev.copy_(self.x_host, non_blocking=True)
-            mx.mx_quant_act(self.x_dev, self.aq, self.sa)
-            mx.mx_gemm(layer.layout, layer.blob, self.aq, self.sa, self.y_dev, workspace=ws, path=path)
+            mx.mx_linear(layer.layout, layer.blob, self.x_dev, self.y_dev, workspace=ws, path=path)
             self.y_host.copy_(self.y_dev, non_blocking=True)
 
         with torch.cuda.stream(self.stream):        # configure kernels outside capture

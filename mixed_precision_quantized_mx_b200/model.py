@@ -13,6 +13,8 @@ fractions.  The counts are the minimum traffic of the method, not of any kernel:
     activations = M K + 2 M            int8 codes + fp16 per-token scales
     output      = 2 M N                fp16 Y
 * quantize-activation bytes = (2 or 4) M K in + M K + 2 M out
+* linear bytes (the layer as a whole, quantized activations being an
+  intermediate) = weights + (2 or 4) M K of X + 2 M N of Y
 
 The compute-intensity form I = 2MNK / (M K B_act + K N B_weight) is the one the
 MixLLM paper uses to argue for 8-bit activations and 4-bit weights (section 3.1.2).
@@ -46,3 +48,8 @@ def quant_act_bytes(M: int, K: int, in_bytes: int = 2) -> float:
 def step_bytes(M: int, N: int, K: int, group: int, n8: int, in_bytes: int = 2) -> float:
     """quantize activations + GEMM: X in, Aq/s_a round trip through HBM, Y out."""
     return quant_act_bytes(M, K, in_bytes) + gemm_bytes(M, N, K, group, n8)
+
+
+def linear_bytes(M: int, N: int, K: int, group: int, n8: int, in_bytes: int = 2) -> float:
+    """The layer end to end: X in, packed weights, Y out."""
+    return weight_bytes(N, K, group, n8) + float(in_bytes) * M * K + 2.0 * M * N

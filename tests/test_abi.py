@@ -130,3 +130,38 @@ def test_paths_need_no_workspace_and_dispatch_on_m(lib):
     # 16 tokens of a 64K-column activation slice cannot be staged per cluster: tensor cores
     Lbig = mx.mx_layout_init(1024, 65536, 128, 102)
     assert mx.mx_gemm_select_path(Lbig, 16) == mx.PATH_TENSOR
+
+
+def test_linear_workspace_follows_the_fused_decode_rule(lib):
+    L = mx.mx_layout_init(4096, 4096, 128, 410)
+    import torch
+    # decode-sized M with a small activation row: one fused kernel, no scratch
+    for M in (1, 2, 3, 4):
+        assert mx.mx_linear_workspace_size(L, M, torch.float16) == 0
+        assert mx.mx_linear_workspace_size(L, M, torch.float32) == 0
+    assert mx.mx_linear_workspace_size(L, 0, torch.float16) == 0
+    # more tokens, the tensor-core path, or a forced path: Aq + s_a, 16-byte rounded
+    a16 = lambda v: (v + 15) // 16 * 16
+    for M in (5, 16, 17, 2048):
+        assert mx.mx_linear_workspace_size(L, M, torch.float16) == a16(M * 4096) + a16(2 * M)
+    assert mx.mx_linear_workspace_size(L, 1, torch.float16, path=mx.PATH_TENSOR) == 4096 + 16
+    # 4 fp32 rows of 8192 columns exceed the 64 KB the fused kernel stages
+    Lw = mx.mx_layout_init(1024, 8192, 128, 102)
+    assert mx.mx_linear_workspace_size(Lw, 2, torch.float32) == 0
+    assert mx.mx_linear_workspace_size(Lw, 4, torch.float32) == a16(4 * 8192) + 16
+
+
+def test_linear_host_argument_checks(lib):
+    L = mx.mx_layout_init(256, 256, 128, 10)
+    o = mx.GemmOpts(0, 0, None, None)
+    n = ctypes.c_size_t(0)
+    assert lib.mx_linear_workspace_size(ctypes.byref(L), 1, 5, ctypes.byref(o), ctypes.byref(n)) == 1
+    assert lib.mx_linear_workspace_size(ctypes.byref(L), -1, 1, ctypes.byref(o), ctypes.byref(n)) == 1
+    assert lib.mx_linear_workspace_size(ctypes.byref(L), 1, 1, ctypes.byref(o), None) == 1
+    args = lambda M, ldx, ldy, xdt=1: (ctypes.byref(L), None, None, xdt, M, ldx, None, ldy, None, 0,
+                                       ctypes.byref(o), None)
+    assert lib.mx_linear(*args(1, 100, 256)) == 1           # ldx < K
+    assert lib.mx_linear(*args(1, 256, 100)) == 1           # ldy < N
+    assert lib.mx_linear(*args(1, 256, 256, xdt=9)) == 1    # bad dtype
+    assert lib.mx_linear(*args(-2, 256, 256)) == 1
+    assert lib.mx_linear(*args(0, 256, 256)) == 0           # M = 0: no-op
