@@ -234,6 +234,37 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
                     int64_t ldx, uint16_t* Y, int64_t ldy, void* workspace, size_t ws_bytes,
                     const mx_gemm_opts* opts, void* stream);
 
+/*
+ * MX_NOALLOC_SCRATCH_BYTES -- size of the fixed device array (one per device)
+ * that mx_linear_noalloc uses as its scratch: 4 MiB.
+ */
+#define MX_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * mx_linear_noalloc -- mx_linear with no workspace argument and no allocation.
+ * The method has no counterpart of this call; it exists for callers that
+ * cannot hand out device memory.  Where mx_linear needs scratch (the
+ * two-kernel path: Aq of M*K bytes and s_a of 2*M bytes, each rounded up to 16
+ * bytes, as mx_linear_workspace_size reports), this call uses a file-scope
+ * device array of MX_NOALLOC_SCRATCH_BYTES bytes instead.  Its address on the
+ * calling thread's current device is looked up with cudaGetSymbolAddress on
+ * the first call that needs it on that device and kept for later calls.
+ *   Arguments as mx_linear, less workspace and ws_bytes.
+ * Nothing in the array has to start at zero: the quantizer writes every byte
+ * of it that the GEMM then reads.  The call never allocates or frees device
+ * or host memory.
+ * Returns MX_ERR_WORKSPACE, before anything is launched, when the scratch
+ * needed exceeds MX_NOALLOC_SCRATCH_BYTES; MX_ERR_CUDA when the address
+ * lookup fails; otherwise what mx_linear returns.
+ * All calls on one device share the one array, so two calls whose kernels can
+ * run at the same time (streams with no order between them, or several host
+ * threads) race on it; calls in one stream are ordered and safe.  Make the
+ * first call on each device outside any stream capture.
+ */
+mx_status mx_linear_noalloc(const mx_layout* L, const void* blob, const void* X, mx_dtype xdtype, int M,
+                            int64_t ldx, uint16_t* Y, int64_t ldy, const mx_gemm_opts* opts,
+                            void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,7 @@ PATH_AUTO, PATH_SPLITK, PATH_TENSOR = 0, 1, 2
 
 EXPORTED = ("mx_version", "mx_last_error", "mx_layout_init", "mx_layout_from_header",
             "mx_pack_weights", "mx_quant_act", "mx_gemm_workspace_size", "mx_gemm_select_path",
-            "mx_gemm", "mx_linear_workspace_size", "mx_linear")
+            "mx_gemm", "mx_linear_workspace_size", "mx_linear", "mx_linear_noalloc")
 
 
 class MXError(RuntimeError):
@@ -80,8 +80,11 @@ def lib() -> ctypes.CDLL:
                                            ctypes.POINTER(Z)]
     L.mx_linear.argtypes = [ctypes.POINTER(Layout), P, P, I, I, I64, P, I64, P, Z,
                             ctypes.POINTER(GemmOpts), P]
+    L.mx_linear_noalloc.argtypes = [ctypes.POINTER(Layout), P, P, I, I, I64, P, I64,
+                                    ctypes.POINTER(GemmOpts), P]
     for n in ("mx_layout_init", "mx_layout_from_header", "mx_pack_weights", "mx_quant_act",
-              "mx_gemm_workspace_size", "mx_gemm", "mx_linear_workspace_size", "mx_linear"):
+              "mx_gemm_workspace_size", "mx_gemm", "mx_linear_workspace_size", "mx_linear",
+              "mx_linear_noalloc"):
         getattr(L, n).restype = I
     _lib = L
     return L
@@ -199,3 +202,16 @@ def mx_linear(L: Layout, blob: torch.Tensor, X: torch.Tensor, Y: torch.Tensor,
     _check(lib().mx_linear(ctypes.byref(L), _ptr(blob), _ptr(X), _dtype_code(X), M, X.stride(0),
                            _ptr(Y), Y.stride(0), _ptr(workspace), ws_bytes, ctypes.byref(o),
                            _stream(stream)), "mx_linear")
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20      # MX_NOALLOC_SCRATCH_BYTES
+
+
+def mx_linear_noalloc(L: Layout, blob: torch.Tensor, X: torch.Tensor, Y: torch.Tensor, path: int = 0,
+                      split: int = 0, debug_partials: torch.Tensor | None = None,
+                      status: torch.Tensor | None = None, stream=None) -> None:
+    assert X.dim() == 2 and X.stride(1) == 1
+    o = _opts(path, split, debug_partials, status)
+    _check(lib().mx_linear_noalloc(ctypes.byref(L), _ptr(blob), _ptr(X), _dtype_code(X), X.shape[0],
+                                   X.stride(0), _ptr(Y), Y.stride(0), ctypes.byref(o), _stream(stream)),
+           "mx_linear_noalloc")

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "mx_internal.cuh"
@@ -296,6 +297,60 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
     uint16_t* s_a = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + align16(size_t(M) * L->K));
     if ((st = mx_quant_act(X, xdtype, M, L->K, ldx, Aq, s_a, stream)) != MX_OK) return st;
     return mx_gemm(L, blob, Aq, s_a, M, Y, ldy, nullptr, 0, opts, stream);
+}
+
+// ---------------------------------------------------------------------------
+// mx_linear_noalloc: the scratch of mx_linear's two-kernel path in a fixed
+// device array instead of a caller workspace.
+
+}  // extern "C"
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MX_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocDevices = 64;
+void* g_noalloc_addr[kNoAllocDevices] = {};
+std::mutex g_noalloc_mu;
+
+// the array's address on the current device, looked up once per device
+mx_status noalloc_scratch(void** addr) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kNoAllocDevices)
+        return fail(MX_ERR_UNSUPPORTED, "device %d beyond the %d this call tracks", dev, kNoAllocDevices);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_fail(e, "cudaGetSymbolAddress of the scratch array");
+        }
+        g_noalloc_addr[dev] = p;
+    }
+    *addr = g_noalloc_addr[dev];
+    return MX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mx_status mx_linear_noalloc(const mx_layout* L, const void* blob, const void* X, mx_dtype xdtype, int M,
+                            int64_t ldx, uint16_t* Y, int64_t ldy, const mx_gemm_opts* opts,
+                            void* stream) {
+    size_t need = 0;
+    mx_status st = mx_linear_workspace_size(L, M, xdtype, opts, &need);
+    if (st != MX_OK) return st;
+    if (need > MX_NOALLOC_SCRATCH_BYTES)
+        return fail(MX_ERR_WORKSPACE, "%zu bytes of scratch needed, the fixed array holds %u", need,
+                    MX_NOALLOC_SCRATCH_BYTES);
+    void* ws = nullptr;
+    if (need > 0 && (st = noalloc_scratch(&ws)) != MX_OK) return st;
+    return mx_linear(L, blob, X, xdtype, M, ldx, Y, ldy, ws, need > 0 ? size_t(MX_NOALLOC_SCRATCH_BYTES) : 0,
+                     opts, stream);
 }
 
 }  // extern "C"

@@ -165,3 +165,19 @@ def test_linear_host_argument_checks(lib):
     assert lib.mx_linear(*args(1, 256, 256, xdt=9)) == 1    # bad dtype
     assert lib.mx_linear(*args(-2, 256, 256)) == 1
     assert lib.mx_linear(*args(0, 256, 256)) == 0           # M = 0: no-op
+
+
+def test_noalloc_scratch_limit_is_checked_before_any_launch(lib):
+    text = open(os.path.join(ROOT, "include", "mx.h")).read()
+    m = re.search(r"#define MX_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == mx.NOALLOC_SCRATCH_BYTES
+    L = mx.mx_layout_init(4096, 4096, 128, 410)
+    o = mx.GemmOpts(0, 0, None, None)
+    # 1025 tokens of 4096 codes need 4 MiB + 16 B + 2064 B: refused with no pointer touched
+    M = mx.NOALLOC_SCRATCH_BYTES // 4096 + 1
+    assert mx.mx_linear_workspace_size(L, M) > mx.NOALLOC_SCRATCH_BYTES
+    assert lib.mx_linear_noalloc(ctypes.byref(L), None, None, 1, M, 4096, None, 4096,
+                                 ctypes.byref(o), None) == 7
+    assert "fixed array" in lib.mx_last_error().decode()
+    assert lib.mx_linear_noalloc(ctypes.byref(L), None, None, 1, 0, 4096, None, 4096,
+                                 ctypes.byref(o), None) == 0          # M = 0: no-op
