@@ -13,33 +13,60 @@
 // Work split.  A "unit" is 128 packed 4-bit rows, or 64 packed 8-bit rows (an
 // 8-bit tile is two units), so every unit streams 8 KB of codes per 128-column
 // k-block.  The S CTAs that split one unit's K range form a thread-block
-// cluster: each streams its k-blocks, leaves its per-row partial sums in shared
-// memory, and after a cluster barrier rank 0 adds the S partials in rank order
+// cluster; S is chosen so that the whole grid is resident at once (one wave).
+// Each CTA streams its k-blocks -- codes, group scales and zero points --
+// through a ring of shared-memory slots of up to four k-blocks each, filled by
+// asynchronous copies that one producer warp issues (one copy per operand per
+// slot: a bulk copy for the contiguous 4-bit codes, scales and zero points, a
+// 4-D tensor copy for the half-tile rows of 8-bit codes), so the eight consumer
+// warps spend their issue slots on shared-memory reads and dp4a only.  Consumers leave per-row partial sums in
+// shared memory; rank 0 of the cluster adds the S partials in rank order
 // (deterministic) through distributed shared memory, applies s_a and scatters
 // the rows to their original columns of Y (section 3.3, fused scatter).  No
 // workspace and no second kernel.
 //
-// The kernel is launched as a programmatic dependent of the activation
-// quantizer: its weight, scale and zero-point loads are in flight before
-// griddepcontrol.wait, which it passes only once the quantized activations exist.
-// It lets its own dependents launch at once, so the next step's quantizer is
-// resident (and waiting) when this kernel finishes.
+// The kernel is launched as a programmatic dependent of whatever precedes it on
+// the stream: the weight stream starts at once, and only the activation reads
+// wait (griddepcontrol.wait).  It lets its own dependents launch at once.
+//
+// Activations come either quantized (Aq, s_a from the activation quantizer) or
+// raw (X in fp16/fp32, up to four tokens): then each CTA stages its own K slice
+// of X, the cluster exchanges the slice maxima (the row absmax is their max,
+// exactly), and each CTA quantizes its slice with the quantizer's own device
+// functions, so the codes are identical to the two-kernel path.
 #include <algorithm>
 #include <cooperative_groups.h>
+#include <cstring>
 #include <type_traits>
 
 #include "mx_internal.cuh"
+#include "sm100.cuh"
 
 namespace mx {
 namespace {
 
 namespace cg = cooperative_groups;
+using namespace sm100;
 
-constexpr int kThreads = 256;
-constexpr int kBatch = 4;                  // k-blocks whose code loads are in flight together
-constexpr int kMaxActSmem = 64 * 1024;     // activation slice staged in shared memory
-constexpr int kMaxSmem = 200 * 1024;       // activation slice + partial sums of all ranks
-constexpr int kMaxCluster = 8;             // portable cluster size
+constexpr int kConsumers = 256;               // 8 warps: thread -> (row, 32-byte slice)
+constexpr int kThreads = kConsumers + 32;     // + one producer warp
+constexpr int kProducerWarp = kConsumers / 32;
+// per k-block of a slot: one unit's codes, <= 2 groups x 128 rows of fp16
+// scales, <= 2 groups x 128 rows of uint8 zero points
+constexpr int kKbCodes = 8192;
+constexpr int kKbScales = 2 * kTileRows * 2;
+constexpr int kKbZeros = 2 * kTileRows;
+constexpr int kKbSlotBytes = kKbCodes + kKbScales + kKbZeros;
+constexpr int kMaxKps = 4;                    // k-blocks per slot
+constexpr int kMaxSlots = 4;
+constexpr int kMaxActSmem = 64 * 1024;        // activation slice staged in shared memory
+constexpr int kMaxSmem = 200 * 1024;
+constexpr int kMaxCluster = 8;                // portable cluster size
+constexpr int kFullRowBytes = 16 * 1024;      // X rows staged whole up to this size
+constexpr int kConsumerBar = 1;               // named barrier of the consumer warps
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+static_assert(kKbSlotBytes % 128 == 0, "tensor copies need 128-byte aligned slots");
 
 struct DecArgs {
     Geom g;
@@ -52,28 +79,39 @@ struct DecArgs {
     int M;
     int S;            // CTAs per unit (cluster size)
     int kbu;          // k-blocks per CTA
+    int kps;          // k-blocks per slot
+    int ns;           // ring slots
+    int off_act, off_sa64, off_part, off_raw;   // dynamic shared-memory layout
+    int xfull;        // in-kernel quantization stages whole X rows (no exchange)
     int32_t* debug;
-    int32_t* status;  // MX_ERR_TIMEOUT if the reduction wait ran out (never expected)
+    int32_t* status;  // MX_ERR_TIMEOUT if a bounded wait ran out (never expected)
 };
-
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
 
 __device__ __forceinline__ int dp4a(uint32_t a, uint32_t b, int c) {
     return __dp4a(int(a), int(b), c);
+}
+
+// unsigned bytes of a times signed bytes of b, accumulated into c
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
 }
 
 __device__ __forceinline__ void griddep_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+__device__ __forceinline__ void consumer_sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(kConsumerBar), "n"(kConsumers) : "memory");
+}
+
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
 
 // the same shared-memory address in CTA `rank` of this cluster
@@ -83,14 +121,12 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
     return r;
 }
 
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-
-// arrive on an mbarrier of another CTA of the cluster, releasing this CTA's
-// earlier writes to the cluster
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+// asynchronous store into another CTA's shared memory that counts its 4 bytes
+// on that CTA's mbarrier (complete_tx), so the receiver's wait covers every
+// writer thread's data
+__device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+                 ::"r"(remote_addr), "r"(__float_as_uint(v)), "r"(remote_bar) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
@@ -99,34 +135,90 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
     return ok != 0;
 }
 
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
+// bounded wait on a cluster-scope phase (remote arrivals); false after the limit
+__device__ __forceinline__ bool cluster_phase_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (globaltimer_ns() - t0 > kTimeoutNs) {
+            if (status) atomicExch(status, MX_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// bounded wait for copies to land, ignoring the abort flag (used before exit)
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > kTimeoutNs) return;
+}
+
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// eight staged activations from shared memory, widened to fp32
+__device__ __forceinline__ void smem8(const __half* p, float (&v)[8]) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(p);
+    const __half2* h = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void smem8(const float* p, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void smem4(const __half* p, float (&v)[4]) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+__device__ __forceinline__ void smem4(const float* p, float (&v)[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
 }
 
 // resident CTAs per SM each variant is compiled for (register budget)
-__host__ __device__ constexpr int decode_ctas_per_sm(int mt, int nb) {
-    return mt >= 16 ? 1 : (mt <= 2 && nb == 1) ? 3 : 2;
+__host__ __device__ constexpr int decode_ctas_per_sm(int mt) {
+    return mt <= 2 ? 3 : mt <= 8 ? 2 : 1;
 }
 
-// NB: register buffers of kBatch k-blocks (2 = the next batch streams while one
-// is computed; 1 when a CTA's whole K range is a single batch).
 // XT: void -- read Aq and s_a produced by the activation quantizer; __half or
-// float -- read X and quantize in-kernel: each CTA takes the absmax of the whole
-// row (the scale needs all K) and quantizes only its own K slice into shared
-// memory, with the quantizer's own device code, so the codes are identical.
-template <int MT, int NB, bool DEBUG, typename XT>
-__global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(MT, NB))
-gemm_decode_kernel(const __grid_constant__ DecArgs a) {
-    extern __shared__ __align__(16) uint8_t smem[];
+// float -- read X and quantize in-kernel (see the file comment).
+template <int MT, bool DEBUG, typename XT>
+__global__ void __launch_bounds__(kThreads, decode_ctas_per_sm(MT))
+gemm_decode_kernel(const __grid_constant__ CUtensorMap codes8_map, const __grid_constant__ DecArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    // tensor copies land on 128-byte boundaries: align the base (the plan adds 128 bytes)
+    uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
     const Geom& g = a.g;
-    cg::cluster_group cluster = cg::this_cluster();
-    const int rank = int(cluster.block_rank());
+    const int rank = int(cg::this_cluster().block_rank());
     const int unit = blockIdx.x / a.S;
     const bool eight = unit < 2 * g.t8;
     const int tile = eight ? unit >> 1 : unit - 2 * g.t8;
@@ -137,65 +229,94 @@ gemm_decode_kernel(const __grid_constant__ DecArgs a) {
     const int nkb = max(kb1 - kb0, 0);
     const int m0 = blockIdx.y * MT;
     const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int gpk = kKBlock / g.group;                     // groups per k-block: 1 or 2
 
-    // thread -> (row, 32-byte slice of a k-block row)
-    int r, sub;
-    if (eight) { r = row0 + (tid >> 2); sub = tid & 3; }   // 4 slices of 32 B per 128-B row
-    else { r = tid >> 1; sub = tid & 1; }                   // 2 slices of 32 B per 64-B row
-    const uint8_t* wbase = eight
-        ? reinterpret_cast<const uint8_t*>(g.codes8) + size_t(tile) * g.kblocks * kBlock8Bytes + r * 128 + sub * 32
-        : g.codes4 + size_t(tile) * g.kblocks * kBlock4Bytes + r * 64 + sub * 32;
-    const size_t wstride = eight ? kBlock8Bytes : kBlock4Bytes;
-    // logical 16-column chunks held by this thread (the 8-bit rows are stored swizzled)
-    const int lc0 = eight ? (2 * sub) ^ (r & 7) : 4 * sub;
-    const int lc1 = eight ? (2 * sub + 1) ^ (r & 7) : 4 * sub + 2;   // 4-bit: second 32 codes
-    const size_t meta_base = size_t(tile) * g.G * kTileRows + r;
-    const __half* scales = eight ? g.scales8 : g.scales4;
-
-    // the next kernel (the following step's activation quantizer) may become
-    // resident now; it waits for this grid to complete before it reads anything
-    asm volatile("griddepcontrol.launch_dependents;");
-
-    // ---- loads that do not depend on the previous kernel: codes, scales, zeros.
-    // Two register buffers of kBatch k-blocks: batch i+1 is in flight while batch i
-    // is computed.
-    uint4 w[NB][kBatch][2];
-    __half sw[NB][kBatch];
-    uint8_t zw[NB][kBatch];
-    auto load_batch = [&](int buf, int kbb) {
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-            if (kbb + u < kb1) {
-                const int kb = kbb + u;
-                w[buf][u][0] = ldg_stream(wbase + size_t(kb) * wstride);
-                w[buf][u][1] = ldg_stream(wbase + size_t(kb) * wstride + 16);
-                const size_t gi = size_t((kb * kKBlock + lc0 * 16) / g.group);
-                sw[buf][u] = scales[meta_base + gi * kTileRows];
-                zw[buf][u] = eight ? uint8_t(0) : g.zeros4[meta_base + gi * kTileRows];
-            }
-    };
-    load_batch(0, kb0);
-    if (NB > 1 && kb0 + kBatch < kb1) load_batch(NB - 1, kb0 + kBatch);
-
-    // rank 0 collects the partial sums: its barrier must exist before anyone arrives
-    __shared__ uint64_t red_bar;
+    __shared__ uint64_t full[kMaxSlots], empty[kMaxSlots];
+    __shared__ uint64_t red_bar, x_bar;
+    __shared__ int abort_flag;
     if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&red_bar)), "r"(max(a.S - 1, 1)));
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int i = 0; i < a.ns; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kConsumers / 32);
+        }
+        mbar_init(&red_bar, 1);      // completes on rank 0's expect_tx + the peers' stores
+        mbar_init(&x_bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
     }
-    cluster.sync();
-    griddep_wait();
+    __syncthreads();
+    // Peers store into this CTA's exchange slots (counted on red_bar / x_bar)
+    // only after every CTA of the cluster has initialized its barriers: each
+    // thread's arrive here is matched by its wait before its first remote access
+    // (or before it exits).
+    cluster_arrive();
+    asm volatile("griddepcontrol.launch_dependents;");
+    uint8_t* ring = smem;
 
+    if (warp == kProducerWarp) {
+        // ---- producer: slot use c carries k-blocks kb0 + c*kps .. (codes, scales,
+        // zero points). These do not depend on the previous kernel: they start at once.
+        const uint8_t* codes4 = g.codes4 + size_t(tile) * g.kblocks * kBlock4Bytes;
+        const uint32_t sbytes = uint32_t(gpk) * kTileRows * 2;          // per k-block
+        const uint32_t zbytes = eight ? 0u : uint32_t(gpk) * kTileRows;
+        const uint8_t* scl = reinterpret_cast<const uint8_t*>(eight ? g.scales8 : g.scales4) +
+                             size_t(tile) * g.G * kTileRows * 2;
+        const uint8_t* zer = g.zeros4 + size_t(tile) * g.G * kTileRows;   // read for 4-bit units only
+        const int kps = a.kps;
+        const int uses = (nkb + kps - 1) / kps;
+        int issued = 0;
+        for (int c = 0; c < uses; ++c) {
+            const int s = c % a.ns;
+            if (c >= a.ns) {
+                bool ok = true;
+                if (lane == 0)
+                    ok = mbar_wait_bounded(&empty[s], uint32_t((c / a.ns - 1) & 1), &abort_flag, a.status, kTimeoutNs);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            }
+            const int kb = kb0 + c * kps;
+            const int nk = min(kps, kb1 - kb);
+            uint8_t* slot = ring + size_t(s) * kps * kKbSlotBytes;
+            // an 8-bit box always spans kps k-blocks (beyond K it is zero-filled)
+            const uint32_t cbytes = eight ? uint32_t(kps) * kKbCodes : uint32_t(nk) * kKbCodes;
+            const int l0 = (c % 10) * 3;        // consecutive slots from different lanes
+            if (lane == l0) mbar_arrive_expect_tx(&full[s], cbytes + nk * (sbytes + zbytes));
+            __syncwarp();
+            if (lane == l0) {
+                if (eight) tma_load_4d(slot, &codes8_map, 0, row0, kb, tile, &full[s]);
+                else bulk_g2s(slot, codes4 + size_t(kb) * kBlock4Bytes, cbytes, &full[s]);
+            } else if (lane == l0 + 1) {
+                bulk_g2s(slot + kps * kKbCodes, scl + size_t(kb) * sbytes, nk * sbytes, &full[s]);
+            } else if (lane == l0 + 2 && !eight) {
+                bulk_g2s(slot + kps * (kKbCodes + kKbScales), zer + size_t(kb) * zbytes, nk * zbytes, &full[s]);
+            }
+            issued = c + 1;
+        }
+        // every copy has landed before the CTA may exit
+        if (lane == 0)
+            for (int c = max(0, issued - a.ns); c < issued; ++c)
+                drain_wait(&full[c % a.ns], uint32_t((c / a.ns) & 1));
+        __syncwarp();
+        cluster_wait();
+        return;
+    }
+
+    // ---- consumers (warps 0-7)
+    // rank 0 scatters rows tid % rows (rows divides the thread count): their
+    // columns of Y come from the row map, which does not depend on the previous kernel
+    const int y_slot = eight ? tile * kTileRows + row0 + tid % rows : (g.t8 + tile) * kTileRows + tid % rows;
+    const int y_col = rank == 0 ? g.rowmap[y_slot] : -1;
     const int rowb = a.kbu * kKBlock;
-    int8_t* act = reinterpret_cast<int8_t*>(smem);
-    int32_t* sa64 = reinterpret_cast<int32_t*>(smem + size_t(MT) * rowb);
-    // partial sums of every rank, [S][MT][128]; only rank 0's copy is used
-    float* part = reinterpret_cast<float*>(smem + size_t(MT) * rowb + size_t(MT) * 2 * a.kbu * 4);
-    __shared__ float sa_loc[MT];              // token scales quantized in-kernel
+    int8_t* act = reinterpret_cast<int8_t*>(smem + a.off_act);
+    int32_t* sa64 = reinterpret_cast<int32_t*>(smem + a.off_sa64);
+    float* part = reinterpret_cast<float*>(smem + a.off_part);   // [S][MT][128], rank 0's is used
+    __shared__ float sa_loc[MT];                                  // token scales quantized in-kernel
+    bool cluster_waited = false;                                  // (the wait matching the arrive)
+    griddep_wait();
     if constexpr (std::is_void_v<XT>) {
         // ---- stage Aq[m0 .. m0+MT)[kb0*128 .. kb1*128) (zero rows beyond M)
         const int chunks = nkb * (kKBlock / 16);
-        for (int i = tid; i < MT * chunks; i += kThreads) {
+        for (int i = tid; i < MT * chunks; i += kConsumers) {
             const int j = i / chunks, c = i % chunks;
             uint4 v = make_uint4(0, 0, 0, 0);
             if (m0 + j < a.M)
@@ -203,50 +324,96 @@ gemm_decode_kernel(const __grid_constant__ DecArgs a) {
             *reinterpret_cast<uint4*>(act + j * rowb + c * 16) = v;
         }
     } else {
-        // ---- per-token absmax over the whole row, then this CTA's slice quantized
+        // ---- in-kernel quantization of X.  Short rows (xfull): every CTA stages the
+        // whole rows and takes the absmax itself.  Long rows: every CTA stages its own
+        // K slice and the cluster exchanges the slice maxima (their max is the row
+        // absmax, exactly).  Either way the CTA then quantizes its own slice with the
+        // quantizer's device functions.
         const XT* X = static_cast<const XT*>(a.X);
-        __shared__ float red[kThreads / 32][MT];
-        float am[MT];
+        const int xrow = a.xfull ? g.K : a.kbu * kKBlock;   // elements per staged row
+        const int xoff = a.xfull ? 0 : kb0 * kKBlock;       // first staged column
+        const int ncols = a.xfull ? g.K : nkb * kKBlock;    // columns staged per row
+        uint8_t* raw = smem + a.off_raw;
+        const int chunks = ncols * int(sizeof(XT)) / 16;
+        for (int i = tid; i < MT * chunks; i += kConsumers) {
+            const int j = i / chunks, c = i % chunks;
+            if (m0 + j < a.M)
+                cp_async16(raw + (size_t(j) * xrow) * sizeof(XT) + size_t(c) * 16,
+                           reinterpret_cast<const uint8_t*>(X + int64_t(m0 + j) * a.ldx + xoff) + size_t(c) * 16);
+        }
+        cp_async_wait_all();
+        consumer_sync();
+        const XT* xs = reinterpret_cast<const XT*>(raw);
+        const int units8 = ncols / 8;
+        __shared__ float red[kConsumers / 32][MT];
+        __shared__ float xmax[kMaxCluster][MT];
 #pragma unroll
         for (int j = 0; j < MT; ++j) {
-            am[j] = 0.0f;
+            float am = 0.0f;
             if (m0 + j < a.M) {
-                const XT* x = X + int64_t(m0 + j) * a.ldx;
-                for (int v = tid; v < g.K / 8; v += kThreads) {
+                for (int c = tid; c < units8; c += kConsumers) {
                     float f[8];
-                    load8(x + v * 8, f);
+                    smem8(xs + size_t(j) * xrow + c * 8, f);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) am[j] = fmaxf(am[j], fabsf(f[e]));
+                    for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(f[e]));
                 }
             }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) am[j] = fmaxf(am[j], __shfl_xor_sync(0xffffffffu, am[j], o));
-            if ((tid & 31) == 0) red[tid >> 5][j] = am[j];
+            for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+            if (lane == 0) red[warp][j] = am;
         }
-        __syncthreads();
+        consumer_sync();
+        const bool exchange = !a.xfull && a.S > 1;
+        if (exchange) {
+            cluster_wait();
+            cluster_waited = true;
+        }
         if (tid < MT) {
             float m = red[0][tid];
 #pragma unroll
-            for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w][tid]);
-            sa_loc[tid] = __half2float(act_scale(m));
-        }
-        __syncthreads();
-        const int units8 = nkb * (kKBlock / 8);
-        for (int i = tid; i < MT * units8; i += kThreads) {
-            const int j = i / units8, c = i % units8;
-            uint2 o = make_uint2(0, 0);
-            if (m0 + j < a.M) {
-                float f[8];
-                load8(X + int64_t(m0 + j) * a.ldx + kb0 * kKBlock + c * 8, f);
-                o.x = quant4(f, sa_loc[j]);
-                o.y = quant4(f + 4, sa_loc[j]);
+            for (int w = 1; w < kConsumers / 32; ++w) m = fmaxf(m, red[w][tid]);
+            xmax[rank][tid] = m;
+            if (exchange) {
+                const uint32_t slot = smem_u32(&xmax[rank][tid]), bar = smem_u32(&x_bar);
+                for (int q = 0; q < a.S; ++q)
+                    if (q != rank) st_async_f32(map_rank(slot, q), m, map_rank(bar, q));
             }
-            *reinterpret_cast<uint2*>(act + j * rowb + c * 8) = o;
+        }
+        if (exchange && tid == 0) {
+            mbar_arrive_expect_tx(&x_bar, uint32_t(a.S - 1) * MT * 4);
+            cluster_phase_wait(&x_bar, 0, a.status);
+        }
+        consumer_sync();
+        float sc[MT];
+#pragma unroll
+        for (int j = 0; j < MT; ++j) {
+            float m = xmax[rank][j];
+            if (exchange)
+                for (int q = 0; q < a.S; ++q) m = fmaxf(m, xmax[q][j]);
+            sc[j] = __half2float(act_scale(m));
+            if (tid == j) sa_loc[j] = sc[j];
+        }
+        // the slice, four values to one word of codes per item, over all threads
+        const int sbase = a.xfull ? kb0 * kKBlock : 0;       // slice start in the staged row
+        const int words = nkb * (kKBlock / 4);
+        for (int i = tid; i < MT * words; i += kConsumers) {
+            const int j = i / words, c = i % words;
+            float sj = sc[0];
+#pragma unroll
+            for (int t = 1; t < MT; ++t)
+                if (j == t) sj = sc[t];
+            uint32_t o = 0;
+            if (m0 + j < a.M) {
+                float f[4];
+                smem4(xs + size_t(j) * xrow + sbase + c * 4, f);
+                o = quant4(f, sj);
+            }
+            *reinterpret_cast<uint32_t*>(act + j * rowb + c * 4) = o;
         }
     }
-    __syncthreads();
+    consumer_sync();
     if (!eight) {
-        for (int i = tid; i < MT * nkb * 2; i += kThreads) {
+        for (int i = tid; i < MT * nkb * 2; i += kConsumers) {
             const int j = i / (nkb * 2), hb = i % (nkb * 2);
             const uint4* p = reinterpret_cast<const uint4*>(act + j * rowb + hb * 64);
             int s = 0;
@@ -260,93 +427,112 @@ gemm_decode_kernel(const __grid_constant__ DecArgs a) {
             }
             sa64[j * 2 * a.kbu + hb] = s;
         }
-        __syncthreads();
+        consumer_sync();
     }
 
-    const int slot = eight ? tile * kTileRows + r : (g.t8 + tile) * kTileRows + r;
-    const int orig = DEBUG ? g.rowmap[slot] : 0;
+    // thread -> (row, 32-byte slice of a k-block row)
+    int r, sub;
+    if (eight) { r = row0 + (tid >> 2); sub = tid & 3; }   // 4 slices of 32 B per 128-B row
+    else { r = tid >> 1; sub = tid & 1; }                   // 2 slices of 32 B per 64-B row
+    const int coff = eight ? (r - row0) * kKBlock + sub * 32 : r * 64 + sub * 32;
+    // logical 16-column chunks held by this thread (the 8-bit rows are stored swizzled)
+    const int lc0 = eight ? (2 * sub) ^ (r & 7) : 4 * sub;
+    const int lc1 = eight ? (2 * sub + 1) ^ (r & 7) : 4 * sub + 2;   // 4-bit: second 32 codes
+    const int gl = lc0 * 16 / g.group;                    // this thread's group within a k-block
+    const int slot_row = eight ? tile * kTileRows + r : (g.t8 + tile) * kTileRows + r;
+    const int orig = DEBUG ? g.rowmap[slot_row] : 0;
     float out[MT];
 #pragma unroll
     for (int j = 0; j < MT; ++j) out[j] = 0.0f;
 
-    auto compute_batch = [&](int buf, int kbb) {
+    bool ok = true;
+    const int kps = a.kps;
+    // one k-block of a landed slot: codes, scale and zero point from the slot,
+    // activations and their 64-column sums from shared memory
+    auto kblock = [&](const uint8_t* sl, int u, int kl) {
+        const uint8_t* cw = sl + u * kKbCodes + coff;
+        const uint4 w[2] = {*reinterpret_cast<const uint4*>(cw), *reinterpret_cast<const uint4*>(cw + 16)};
+        const int gs = (u * gpk + gl) * kTileRows + r;     // (group, row) within the slot
+        const float sw = __half2float(reinterpret_cast<const __half*>(sl + kps * kKbCodes)[gs]);
+        const int kb = kb0 + kl;
+        const int gi = kb * gpk + gl;
+        int acc[MT];
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int kb = kbb + u;
-            if (kb >= kb1) break;
-            const int kl = kb - kb0;
-            const int gi = (kb * kKBlock + lc0 * 16) / g.group;
-            const float s = __half2float(sw[buf][u]);
-            int acc[MT];
+        for (int j = 0; j < MT; ++j) acc[j] = 0;
+        if (eight) {
 #pragma unroll
-            for (int j = 0; j < MT; ++j) acc[j] = 0;
-            if (eight) {
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int lc = i ? lc1 : lc0;
-#pragma unroll
-                    for (int j = 0; j < MT; ++j) {
-                        const uint4 av = *reinterpret_cast<const uint4*>(act + j * rowb + kl * kKBlock + lc * 16);
-                        acc[j] = dp4a(w[buf][u][i].x, av.x, acc[j]);
-                        acc[j] = dp4a(w[buf][u][i].y, av.y, acc[j]);
-                        acc[j] = dp4a(w[buf][u][i].z, av.z, acc[j]);
-                        acc[j] = dp4a(w[buf][u][i].w, av.w, acc[j]);
-                    }
-                }
-                // threads holding the same group: the 4 slices of a row (g = 128) or the two
-                // slices of one logical half (g = 64)
+            for (int i = 0; i < 2; ++i) {
+                const int lc = i ? lc1 : lc0;
 #pragma unroll
                 for (int j = 0; j < MT; ++j) {
-                    acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 1);
-                    if (g.group == 128) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 2);
-                }
-            } else {
-                const int z = zw[buf][u];
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const uint32_t wd[4] = {w[buf][u][i].x, w[buf][u][i].y, w[buf][u][i].z, w[buf][u][i].w};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t lo = wd[q] & 0x0F0F0F0Fu;          // k = 8w .. 8w+3
-                        const uint32_t hi = (wd[q] >> 4) & 0x0F0F0F0Fu;   // k = 8w+4 .. 8w+7
-                        const int koff = sub * 64 + i * 32 + q * 8;
-#pragma unroll
-                        for (int j = 0; j < MT; ++j) {
-                            const uint2 av = *reinterpret_cast<const uint2*>(act + j * rowb + kl * kKBlock + koff);
-                            acc[j] = dp4a(lo, av.x, acc[j]);
-                            acc[j] = dp4a(hi, av.y, acc[j]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < MT; ++j) {
-                    acc[j] -= z * sa64[j * 2 * a.kbu + kl * 2 + sub];
-                    if (g.group == 128) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 1);
+                    const uint4 av = *reinterpret_cast<const uint4*>(act + j * rowb + kl * kKBlock + lc * 16);
+                    acc[j] = dp4a(w[i].x, av.x, acc[j]);
+                    acc[j] = dp4a(w[i].y, av.y, acc[j]);
+                    acc[j] = dp4a(w[i].z, av.z, acc[j]);
+                    acc[j] = dp4a(w[i].w, av.w, acc[j]);
                 }
             }
+            // threads holding the same group: the 4 slices of a row (g = 128) or the two
+            // slices of one logical half (g = 64)
 #pragma unroll
-            for (int j = 0; j < MT; ++j) out[j] = __fmaf_rn(i2f_biased(acc[j]), s, out[j]);
-            if (DEBUG && orig >= 0) {
-                const bool writer = eight ? (g.group == 128 ? sub == 0 : (sub & 1) == 0)
-                                          : (g.group == 128 ? sub == 0 : true);
-                if (writer) {
+            for (int j = 0; j < MT; ++j) {
+                acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 1);
+                if (g.group == 128) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 2);
+            }
+        } else {
+            const int z = sl[kps * (kKbCodes + kKbScales) + gs];
+            // word q of the thread's 32 bytes holds k = 8q .. 8q+7 of its 64 columns: the
+            // low nibbles pair with k = 8q .. 8q+3 and the high nibbles, left in place
+            // (16 x code, an unsigned byte), with k = 8q+4 .. 8q+7
+            const uint32_t wd[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
 #pragma unroll
-                    for (int j = 0; j < MT; ++j)
-                        if (m0 + j < a.M) a.debug[(size_t(m0 + j) * g.N + orig) * g.G + gi] = acc[j];
+            for (int j = 0; j < MT; ++j) {
+                const uint4* ap = reinterpret_cast<const uint4*>(act + j * rowb + kl * kKBlock + sub * 64);
+                int lo = 0, hi16 = 0;
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const uint4 av = ap[h];                  // k = 16h .. 16h+15
+                    lo = dp4a(wd[2 * h] & 0x0F0F0F0Fu, av.x, lo);
+                    hi16 = dp4a_us(wd[2 * h] & 0xF0F0F0F0u, av.y, hi16);
+                    lo = dp4a(wd[2 * h + 1] & 0x0F0F0F0Fu, av.z, lo);
+                    hi16 = dp4a_us(wd[2 * h + 1] & 0xF0F0F0F0u, av.w, hi16);
                 }
+                acc[j] = lo + (hi16 >> 4);                   // exact: hi16 is 16 x the sum
+            }
+#pragma unroll
+            for (int j = 0; j < MT; ++j) {
+                acc[j] -= z * sa64[j * 2 * a.kbu + kl * 2 + sub];
+                if (g.group == 128) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 1);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < MT; ++j) out[j] = __fmaf_rn(i2f_biased(acc[j]), sw, out[j]);
+        if (DEBUG && orig >= 0) {                       // padding rows have no column
+            const bool writer = eight ? (g.group == 128 ? sub == 0 : (sub & 1) == 0)
+                                      : (g.group == 128 ? sub == 0 : true);
+            if (writer) {
+#pragma unroll
+                for (int j = 0; j < MT; ++j)
+                    if (m0 + j < a.M) a.debug[(size_t(m0 + j) * g.N + orig) * g.G + gi] = acc[j];
             }
         }
     };
-    if (NB == 1) {
-        compute_batch(0, kb0);                  // the whole range is one batch
-    } else {
-        // unrolled by two so both register buffers are indexed with constants
-        for (int kbb = kb0; kbb < kb1; kbb += 2 * kBatch) {
-            compute_batch(0, kbb);
-            if (kbb + 2 * kBatch < kb1) load_batch(0, kbb + 2 * kBatch);
-            if (kbb + kBatch < kb1) compute_batch(NB - 1, kbb + kBatch);
-            if (kbb + 3 * kBatch < kb1) load_batch(NB - 1, kbb + 3 * kBatch);
+    const int uses = (nkb + kps - 1) / kps;
+    for (int c = 0; c < uses; ++c) {
+        const int s = c % a.ns;
+        if (ok) ok = mbar_wait_bounded(&full[s], uint32_t((c / a.ns) & 1), &abort_flag, a.status, kTimeoutNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            const uint8_t* sl = ring + size_t(s) * kps * kKbSlotBytes;
+            const int nk = min(kps, nkb - c * kps);
+            // the slot's k-blocks are independent dot products: unrolled, their loads
+            // and dp4a chains interleave
+#pragma unroll
+            for (int u = 0; u < kMaxKps; ++u)
+                if (u < nk) kblock(sl, u, c * kps + u);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);     // this warp is done with the slot
     }
     // with g = 64 the slices of a row hold different groups: add them up
     if (g.group == 64) {
@@ -356,15 +542,15 @@ gemm_decode_kernel(const __grid_constant__ DecArgs a) {
     }
     const bool lead = sub == 0;
     const int rl = r - row0;                       // row within the unit
+    if (!cluster_waited) cluster_wait();
     if (rank != 0) {
-        // push this CTA's partials into rank 0's slot `rank`, then arrive there
+        // push this CTA's partials into rank 0's slot `rank`, counted on its red_bar
         if (lead) {
-            const uint32_t dst = map_rank(smem_addr(part + (size_t(rank) * MT) * 128 + rl), 0);
+            const uint32_t dst = map_rank(smem_u32(part + (size_t(rank) * MT) * 128 + rl), 0);
+            const uint32_t bar = map_rank(smem_u32(&red_bar), 0);
 #pragma unroll
-            for (int j = 0; j < MT; ++j) st_cluster_f32(dst + j * 128 * 4, out[j]);
+            for (int j = 0; j < MT; ++j) st_async_f32(dst + j * 128 * 4, out[j], bar);
         }
-        __syncthreads();
-        if (tid == 0) mbar_arrive_remote(map_rank(smem_addr(&red_bar), 0));
         return;
     }
     if (lead) {
@@ -372,28 +558,19 @@ gemm_decode_kernel(const __grid_constant__ DecArgs a) {
         for (int j = 0; j < MT; ++j) part[j * 128 + rl] = out[j];
     }
     // rank 0: wait (bounded) for the S-1 other partials, then add them in rank order
-    bool ok = true;
-    if (a.S > 1) {
-        if (tid == 0) {
-            const uint64_t t0 = globaltimer();
-            while (!mbar_try_wait_cluster(&red_bar, 0)) {
-                if (globaltimer() - t0 > 2000000000ull) {
-                    ok = false;
-                    if (a.status) atomicExch(a.status, MX_ERR_TIMEOUT);
-                    break;
-                }
-            }
-        }
+    bool okr = true;
+    if (a.S > 1 && tid == 0) {
+        mbar_arrive_expect_tx(&red_bar, uint32_t(a.S - 1) * MT * rows * 4);
+        okr = cluster_phase_wait(&red_bar, 0, a.status);
     }
-    ok = __syncthreads_and(ok);
-    if (!ok) return;
-    for (int i = tid; i < MT * rows; i += kThreads) {
+    okr = named_bar_and(kConsumerBar, kConsumers, okr);
+    if (!okr) return;
+    for (int i = tid; i < MT * rows; i += kConsumers) {
         const int j = i / rows, rr = i % rows;
         if (m0 + j >= a.M) continue;
         float sum = 0.0f;
         for (int q = 0; q < a.S; ++q) sum = __fadd_rn(sum, part[(size_t(q) * MT + j) * 128 + rr]);
-        const int sl = eight ? tile * kTileRows + row0 + rr : (g.t8 + tile) * kTileRows + rr;
-        const int o = g.rowmap[sl];
+        const int o = y_col;                      // rr == tid % rows
         float sa;
         if constexpr (std::is_void_v<XT>) sa = __half2float(a.s_a[m0 + j]);
         else sa = sa_loc[j];
@@ -402,10 +579,12 @@ gemm_decode_kernel(const __grid_constant__ DecArgs a) {
 }
 
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
+size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
 
-template <int MT, int NB, bool DEBUG, typename XT>
-cudaError_t launch_t(const DecArgs& args, int units, int m_tiles, size_t smem, cudaStream_t s) {
-    auto k = gemm_decode_kernel<MT, NB, DEBUG, XT>;
+template <int MT, bool DEBUG, typename XT>
+cudaError_t launch_t(const CUtensorMap& map, const DecArgs& args, int units, int m_tiles, size_t smem,
+                     cudaStream_t s) {
+    auto k = gemm_decode_kernel<MT, DEBUG, XT>;
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -413,6 +592,9 @@ cudaError_t launch_t(const DecArgs& args, int units, int m_tiles, size_t smem, c
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!configured[dev]) {
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+        if (e != cudaSuccess) return e;
+        // the ring of every resident CTA must fit: ask for the largest shared-memory carveout
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
@@ -430,69 +612,131 @@ cudaError_t launch_t(const DecArgs& args, int units, int m_tiles, size_t smem, c
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, k, args);
-}
-
-template <int MT, bool DEBUG, typename XT>
-cudaError_t launch_nb(const DecArgs& a, int units, int m_tiles, size_t smem, cudaStream_t s) {
-    return a.kbu <= kBatch ? launch_t<MT, 1, DEBUG, XT>(a, units, m_tiles, smem, s)
-                           : launch_t<MT, 2, DEBUG, XT>(a, units, m_tiles, smem, s);
+    return cudaLaunchKernelEx(&cfg, k, map, args);
 }
 
 template <bool DEBUG>
-cudaError_t launch_mt(const DecArgs& a, int mt, int units, int m_tiles, size_t smem, cudaStream_t s) {
+cudaError_t launch_mt(const CUtensorMap& m, const DecArgs& a, int mt, int units, int m_tiles, size_t smem,
+                      cudaStream_t s) {
     switch (mt) {
-        case 1: return launch_nb<1, DEBUG, void>(a, units, m_tiles, smem, s);
-        case 2: return launch_nb<2, DEBUG, void>(a, units, m_tiles, smem, s);
-        case 4: return launch_nb<4, DEBUG, void>(a, units, m_tiles, smem, s);
-        case 8: return launch_nb<8, DEBUG, void>(a, units, m_tiles, smem, s);
-        default: return launch_nb<16, DEBUG, void>(a, units, m_tiles, smem, s);
+        case 1: return launch_t<1, DEBUG, void>(m, a, units, m_tiles, smem, s);
+        case 2: return launch_t<2, DEBUG, void>(m, a, units, m_tiles, smem, s);
+        case 4: return launch_t<4, DEBUG, void>(m, a, units, m_tiles, smem, s);
+        case 8: return launch_t<8, DEBUG, void>(m, a, units, m_tiles, smem, s);
+        default: return launch_t<16, DEBUG, void>(m, a, units, m_tiles, smem, s);
     }
 }
 
 // in-kernel quantization of X: up to four tokens per CTA
 template <bool DEBUG, typename XT>
-cudaError_t launch_mt_fused(const DecArgs& a, int mt, int units, int m_tiles, size_t smem, cudaStream_t s) {
+cudaError_t launch_mt_fused(const CUtensorMap& m, const DecArgs& a, int mt, int units, int m_tiles, size_t smem,
+                            cudaStream_t s) {
     switch (mt) {
-        case 1: return launch_nb<1, DEBUG, XT>(a, units, m_tiles, smem, s);
-        case 2: return launch_nb<2, DEBUG, XT>(a, units, m_tiles, smem, s);
-        case 4: return launch_nb<4, DEBUG, XT>(a, units, m_tiles, smem, s);
+        case 1: return launch_t<1, DEBUG, XT>(m, a, units, m_tiles, smem, s);
+        case 2: return launch_t<2, DEBUG, XT>(m, a, units, m_tiles, smem, s);
+        case 4: return launch_t<4, DEBUG, XT>(m, a, units, m_tiles, smem, s);
         default: return cudaErrorInvalidValue;
     }
 }
 
+// 8-bit codes as a 4-D tensor [tile][k-block][row][128 bytes]: one box brings
+// kps k-blocks of one 64-row half tile, k-block after k-block, into a slot
+cudaError_t codes8_map(const mx_layout& L, const void* blob, int kps, CUtensorMap* map) {
+    memset(map, 0, sizeof *map);
+    if (L.t8 == 0) return cudaSuccess;                 // no 8-bit units: never read
+    cudaError_t e;
+    EncodeTiledFn enc = encode_fn(&e);
+    if (e != cudaSuccess) return e;
+    const cuuint64_t dims[4] = {cuuint64_t(kKBlock), cuuint64_t(kTileRows), cuuint64_t(L.kblocks), cuuint64_t(L.t8)};
+    const cuuint64_t strides[3] = {cuuint64_t(kKBlock), cuuint64_t(kBlock8Bytes),
+                                   cuuint64_t(kBlock8Bytes) * uint64_t(L.kblocks)};
+    const cuuint32_t box[4] = {cuuint32_t(kKBlock), cuuint32_t(kTileRows / 2), cuuint32_t(kps), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    void* base = const_cast<uint8_t*>(static_cast<const uint8_t*>(blob) + L.off_codes8);
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+DecArgs base_args(const mx_layout& L, const void* blob, int M, uint16_t* Y, int64_t ldy, const DecodePlan& p,
+                  int32_t* debug_partials, int32_t* status) {
+    DecArgs a{};
+    a.g = make_geom(L, blob);
+    a.Y = reinterpret_cast<__half*>(Y);
+    a.ldy = ldy;
+    a.M = M;
+    a.S = p.S;
+    a.kbu = p.kbu;
+    a.kps = p.kps;
+    a.ns = p.ns;
+    a.off_act = p.off_act;
+    a.off_sa64 = p.off_sa64;
+    a.off_part = p.off_part;
+    a.off_raw = p.off_raw;
+    a.xfull = p.xfull;
+    a.debug = debug_partials;
+    a.status = status;
+    return a;
+}
+
 }  // namespace
 
-DecodePlan plan_decode(const mx_layout& L, int M, int split_hint) {
+DecodePlan plan_decode(const mx_layout& L, int M, int split_hint, int x_bytes) {
     DecodePlan p{};
     p.mt = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
     p.m_tiles = std::max(1, ceil_div(M, p.mt));
     p.units = 2 * L.t8 + L.t4;
     const int kb = L.kblocks;
+    const int cps = decode_ctas_per_sm(p.mt);
     // at least as many CTAs per unit as the activation slice needs to fit in shared memory
     const int s_min = ceil_div(kb * p.mt * kKBlock, kMaxActSmem);
-    // fill the resident capacity of a 148-SM B200 once (clusters of up to 8 CTAs
-    // must also pack into GPCs, so aim a little below it); the single-batch
-    // variant keeps three CTAs per SM resident
     int S = split_hint;
     if (S <= 0) {
+        // the whole grid resident at once on a 148-SM B200 (clusters of up to 8
+        // CTAs must also pack into GPCs, so aim a little below the capacity)
         const int work = std::max(1, p.units * p.m_tiles);
-        const int s1 = ceil_div(decode_ctas_per_sm(p.mt, 1) * 148 * 7 / 8, work);
-        if (ceil_div(kb, s1) <= kBatch) {
-            S = s1;
-        } else {
-            // long K ranges: at most ~32 k-blocks per CTA, so several waves of CTAs
-            // keep enough loads in flight
-            S = std::max(ceil_div(decode_ctas_per_sm(p.mt, 2) * 148 * 7 / 8, work), ceil_div(kb, 32));
-        }
+        S = std::max(1, cps * 148 * 7 / 8 / work);
     }
     S = std::max(S, s_min);
     S = std::min(S, std::min(kMaxCluster, kb));
     p.S = S;
     p.kbu = ceil_div(kb, S);
-    p.ok = S >= s_min && p.kbu * p.mt * kKBlock <= kMaxActSmem;
-    p.smem = size_t(p.mt) * p.kbu * kKBlock + size_t(p.mt) * 2 * p.kbu * 4 + size_t(S) * p.mt * 128 * 4;
-    p.ok = p.ok && p.smem <= size_t(kMaxSmem);
+    // shared memory: ring | staged activations | 64-column activation sums |
+    // partial sums of every rank | raw X slice (in-kernel quantization)
+    const size_t act = align16(size_t(p.mt) * p.kbu * kKBlock);
+    const size_t sa64 = align16(size_t(p.mt) * 2 * p.kbu * 4);
+    const size_t part = size_t(S) * p.mt * kTileRows * 4;
+    // in-kernel quantization: whole rows when they are short (no cluster exchange of
+    // the row maxima), else this CTA's slice
+    p.xfull = x_bytes > 0 && S > 1 && size_t(p.mt) * L.K * x_bytes <= size_t(kFullRowBytes);
+    const size_t raw = align16(size_t(p.mt) * (p.xfull ? L.K : p.kbu * kKBlock) * x_bytes);
+    const size_t rest = act + sa64 + part + raw;
+    // resident CTAs per SM the grid needs (at most what the registers allow)
+    const int ctas = p.units * p.m_tiles * S;
+    const int need = std::max(1, std::min(cps, ceil_div(ctas, 148 * 7 / 8)));
+    // per-SM shared memory / resident CTAs, less the 1 KB the hardware reserves per
+    // CTA, the static shared memory and the alignment pad
+    const size_t budget = size_t(233472) / need - 2560;
+    // the largest slots (fewest copies) that leave room for two of them, or one
+    // when a single slot holds the whole K range
+    int kps = 1, ns = 1;
+    for (int k = std::min(kMaxKps, p.kbu); k >= 1; k = k > 2 ? 2 : k - 1) {
+        const int uses = ceil_div(p.kbu, k);
+        int n = std::min(uses, kMaxSlots);
+        while (n > std::min(uses, 2) && size_t(n) * k * kKbSlotBytes + rest > budget) --n;
+        kps = k;
+        ns = n;
+        if (size_t(n) * k * kKbSlotBytes + rest <= budget) break;
+    }
+    p.kps = kps;
+    p.ns = ns;
+    p.off_act = ns * kps * kKbSlotBytes;
+    p.off_sa64 = int(p.off_act + act);
+    p.off_part = int(p.off_sa64 + sa64);
+    p.off_raw = int(p.off_part + part);
+    p.smem = size_t(p.off_raw) + raw + 128;        // + room to align the base
+    p.ok = S >= s_min && size_t(p.kbu) * p.mt * kKBlock <= size_t(kMaxActSmem) && p.smem <= size_t(kMaxSmem);
     return p;
 }
 
@@ -501,23 +745,18 @@ cudaError_t launch_gemm_decode(const mx_layout& L, const void* blob, const int8_
                                const DecodePlan& plan, int32_t* debug_partials, int32_t* status,
                                cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    DecArgs a{};
-    a.g = make_geom(L, blob);
+    DecArgs a = base_args(L, blob, M, Y, ldy, plan, debug_partials, status);
     a.Aq = Aq;
     a.s_a = reinterpret_cast<const __half*>(s_a);
-    a.Y = reinterpret_cast<__half*>(Y);
-    a.ldy = ldy;
-    a.M = M;
-    a.S = plan.S;
-    a.kbu = plan.kbu;
-    a.debug = debug_partials;
-    a.status = status;
-    return debug_partials ? launch_mt<true>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s)
-                          : launch_mt<false>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s);
+    CUtensorMap map;
+    cudaError_t e = codes8_map(L, blob, plan.kps, &map);
+    if (e != cudaSuccess) return e;
+    return debug_partials ? launch_mt<true>(map, a, plan.mt, plan.units, plan.m_tiles, plan.smem, s)
+                          : launch_mt<false>(map, a, plan.mt, plan.units, plan.m_tiles, plan.smem, s);
 }
 
 bool decode_can_fuse(const mx_layout& L, int M, mx_dtype xdt) {
-    // every CTA reads whole activation rows for the scales: keep that to 64 KB
+    // each CTA stages its slice of the X rows: keep whole rows to 64 KB
     return M >= 1 && M <= kMaxFusedTokens &&
            size_t(M) * L.K * (xdt == MX_F16 ? 2 : 4) <= size_t(64) * 1024;
 }
@@ -526,23 +765,23 @@ cudaError_t launch_gemm_decode_fused(const mx_layout& L, const void* blob, const
                                      int64_t ldx, int M, uint16_t* Y, int64_t ldy, const DecodePlan& plan,
                                      int32_t* debug_partials, int32_t* status, cudaStream_t s) {
     if (M == 0) return cudaSuccess;
-    if (plan.mt > kMaxFusedTokens) return cudaErrorInvalidValue;
-    DecArgs a{};
-    a.g = make_geom(L, blob);
+    if (plan.mt > kMaxFusedTokens || !plan.ok) return cudaErrorInvalidValue;
+    // the plan must have room for the raw slice of this input type
+    const size_t cols = plan.xfull ? size_t(L.K) : size_t(plan.kbu) * kKBlock;
+    if (size_t(plan.smem) < size_t(plan.off_raw) + 128 + size_t(plan.mt) * cols * (xdt == MX_F16 ? 2 : 4))
+        return cudaErrorInvalidValue;
+    DecArgs a = base_args(L, blob, M, Y, ldy, plan, debug_partials, status);
     a.X = X;
     a.ldx = ldx;
-    a.Y = reinterpret_cast<__half*>(Y);
-    a.ldy = ldy;
-    a.M = M;
-    a.S = plan.S;
-    a.kbu = plan.kbu;
-    a.debug = debug_partials;
-    a.status = status;
+    CUtensorMap m;
+    cudaError_t e = codes8_map(L, blob, plan.kps, &m);
+    if (e != cudaSuccess) return e;
+    const int u = plan.units, t = plan.m_tiles;
     if (xdt == MX_F16)
-        return debug_partials ? launch_mt_fused<true, __half>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s)
-                              : launch_mt_fused<false, __half>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s);
-    return debug_partials ? launch_mt_fused<true, float>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s)
-                          : launch_mt_fused<false, float>(a, plan.mt, plan.units, plan.m_tiles, plan.smem, s);
+        return debug_partials ? launch_mt_fused<true, __half>(m, a, plan.mt, u, t, plan.smem, s)
+                              : launch_mt_fused<false, __half>(m, a, plan.mt, u, t, plan.smem, s);
+    return debug_partials ? launch_mt_fused<true, float>(m, a, plan.mt, u, t, plan.smem, s)
+                          : launch_mt_fused<false, float>(m, a, plan.mt, u, t, plan.smem, s);
 }
 
 }  // namespace mx

@@ -402,12 +402,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     }
 }
 
-// ---------------------------------------------------------------- host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+}  // namespace
 
+// ---------------------------------------------------------------- host side
 EncodeTiledFn encode_fn(cudaError_t* err) {
     static EncodeTiledFn fn = nullptr;
     static cudaError_t status = cudaSuccess;
@@ -422,8 +419,6 @@ EncodeTiledFn encode_fn(cudaError_t* err) {
     *err = status;
     return fn;
 }
-
-}  // namespace
 
 size_t tc_smem_bytes() { return sizeof(Smem) + 1024; }
 

@@ -239,9 +239,12 @@ namespace {
 
 size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
 
+int x_bytes(mx_dtype xdt) { return xdt == MX_F16 ? 2 : 4; }
+
 bool linear_fused(const mx_layout* L, int M, mx_dtype xdt, const mx_gemm_opts* opts) {
-    return choose_path(L, M, opts) == 1 && mx::decode_can_fuse(*L, M, xdt) &&
-           mx::plan_decode(*L, M, opts ? opts->split : 0).mt <= mx::kMaxFusedTokens;
+    if (choose_path(L, M, opts) != 1 || !mx::decode_can_fuse(*L, M, xdt)) return false;
+    const mx::DecodePlan p = mx::plan_decode(*L, M, opts ? opts->split : 0, x_bytes(xdt));
+    return p.ok && p.mt <= mx::kMaxFusedTokens;
 }
 
 }  // namespace
@@ -281,7 +284,7 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
             return st;
         if (opts && opts->status && (st = check_device_ptr(opts->status, "status")) != MX_OK) return st;
         if (opts && opts->split > 8) return fail(MX_ERR_UNSUPPORTED, "split=%d above the cluster limit 8", opts->split);
-        mx::DecodePlan plan = mx::plan_decode(*L, M, opts ? opts->split : 0);
+        mx::DecodePlan plan = mx::plan_decode(*L, M, opts ? opts->split : 0, x_bytes(xdtype));
         cudaError_t e = mx::launch_gemm_decode_fused(*L, blob, X, xdtype, ldx, M, Y, ldy, plan,
                                                      opts ? opts->debug_partials : nullptr,
                                                      opts ? opts->status : nullptr, s);

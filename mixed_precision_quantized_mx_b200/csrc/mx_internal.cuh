@@ -2,6 +2,7 @@
 // library's translation units (never by the CPU oracle).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -94,17 +95,29 @@ cudaError_t launch_pack(const mx_layout& L, const void* W, mx_dtype wdt, int64_t
 cudaError_t launch_quant_act(const void* X, mx_dtype xdt, int M, int K, int64_t ldx,
                              int8_t* Aq, uint16_t* s_a, cudaStream_t s);
 
+// cuTensorMapEncodeTiled, looked up once through the runtime (no -lcuda)
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn(cudaError_t* err);
+
 struct DecodePlan {
     int mt;             // tokens per CTA (1, 2, 4, 8, 16)
     int m_tiles;        // ceil(M / mt)
     int units;          // 2 * t8 + t4: 64-row 8-bit units and 128-row 4-bit units
     int S;              // CTAs per unit = cluster size (split of K)
     int kbu;            // k-blocks per CTA
-    bool ok;            // the activation slice fits in shared memory
+    int kps;            // k-blocks per ring slot (one copy per operand per slot)
+    int ns;             // weight ring slots per CTA
+    bool ok;            // the activation slice and the ring fit in shared memory
     size_t smem;        // dynamic shared memory per CTA
+    int off_act, off_sa64, off_part, off_raw;   // its layout
+    bool xfull;         // in-kernel quantization stages whole X rows
 };
 
-DecodePlan plan_decode(const mx_layout& L, int M, int split_hint);
+// x_bytes: 0 when the kernel reads Aq, else 2 / 4 (it stages and quantizes fp16 / fp32 X)
+DecodePlan plan_decode(const mx_layout& L, int M, int split_hint, int x_bytes = 0);
 
 cudaError_t launch_gemm_decode(const mx_layout& L, const void* blob, const int8_t* Aq,
                                const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy,

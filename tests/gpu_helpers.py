@@ -51,9 +51,16 @@ def gpu_gemm(L, blob, Aq, sa, path=0, split=0, debug=False, ldy=None):
     Y = Yfull[:, :L.N]
     ws_bytes = mx.mx_gemm_workspace_size(L, M, path=path, split=split)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev())
-    P = torch.zeros((M, L.N, L.G), dtype=torch.int32, device=dev()) if debug else None
+    P = None
+    if debug:                      # guard zones on both sides catch writes outside P
+        pad = 64
+        Pbig = torch.full((M * L.N * L.G + 2 * pad,), -12345, dtype=torch.int32, device=dev())
+        P = Pbig[pad:pad + M * L.N * L.G].view(M, L.N, L.G)
+        P.zero_()
     mx.mx_gemm(L, blob, Aq, sa, Y, workspace=ws, path=path, split=split, debug_partials=P)
     torch.cuda.synchronize()
+    if debug:
+        assert (Pbig[:pad] == -12345).all() and (Pbig[-pad:] == -12345).all()
     return Y, P, Yfull
 
 

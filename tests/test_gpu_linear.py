@@ -31,9 +31,16 @@ def run_linear(L, blob, Xd, path=0, split=0, debug=False, ws_pad=0):
     Y = torch.full((M, L.N), float("nan"), dtype=torch.float16, device=dev())
     n = mx.mx_linear_workspace_size(L, M, Xd.dtype, path=path, split=split)
     ws = torch.empty(n + ws_pad, dtype=torch.uint8, device=dev()) if n + ws_pad else None
-    P = torch.zeros((M, L.N, L.G), dtype=torch.int32, device=dev()) if debug else None
+    P = None
+    if debug:                      # guard zones on both sides catch writes outside P
+        pad = 64
+        Pbig = torch.full((M * L.N * L.G + 2 * pad,), -12345, dtype=torch.int32, device=dev())
+        P = Pbig[pad:pad + M * L.N * L.G].view(M, L.N, L.G)
+        P.zero_()
     mx.mx_linear(L, blob, Xd, Y, workspace=ws, path=path, split=split, debug_partials=P)
     torch.cuda.synchronize()
+    if debug:
+        assert (Pbig[:pad] == -12345).all() and (Pbig[-pad:] == -12345).all()
     return Y, P, n
 
 
