@@ -166,24 +166,6 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// eight staged activations from shared memory, widened to fp32
-__device__ __forceinline__ void smem8(const __half* p, float (&v)[8]) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(p);
-    const __half2* h = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = __half22float2(h[i]);
-        v[2 * i] = f.x;
-        v[2 * i + 1] = f.y;
-    }
-}
-__device__ __forceinline__ void smem8(const float* p, float (&v)[8]) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    const float4 b = *reinterpret_cast<const float4*>(p + 4);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
                                             uint64_t* bar) {
     asm volatile(
@@ -193,6 +175,7 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// four staged activations from shared memory, widened to fp32
 __device__ __forceinline__ void smem4(const __half* p, float (&v)[4]) {
     const uint2 raw = *reinterpret_cast<const uint2*>(p);
     const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
@@ -351,12 +334,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap codes8_map, const __grid_
         for (int j = 0; j < MT; ++j) {
             float am = 0.0f;
             if (m0 + j < a.M) {
-                for (int c = tid; c < units8; c += kConsumers) {
-                    float f[8];
-                    smem8(xs + size_t(j) * xrow + c * 8, f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(f[e]));
-                }
+                for (int c = tid; c < units8; c += kConsumers) am = absmax8(xs + size_t(j) * xrow + c * 8, am);
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
@@ -384,13 +362,14 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap codes8_map, const __grid_
             cluster_phase_wait(&x_bar, 0, a.status);
         }
         consumer_sync();
-        float sc[MT];
+        float sc[MT], rsc[MT];
 #pragma unroll
         for (int j = 0; j < MT; ++j) {
             float m = xmax[rank][j];
             if (exchange)
                 for (int q = 0; q < a.S; ++q) m = fmaxf(m, xmax[q][j]);
             sc[j] = __half2float(act_scale(m));
+            rsc[j] = __frcp_rn(sc[j]);
             if (tid == j) sa_loc[j] = sc[j];
         }
         // the slice, four values to one word of codes per item, over all threads
@@ -398,15 +377,18 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap codes8_map, const __grid_
         const int words = nkb * (kKBlock / 4);
         for (int i = tid; i < MT * words; i += kConsumers) {
             const int j = i / words, c = i % words;
-            float sj = sc[0];
+            float sj = sc[0], rj = rsc[0];
 #pragma unroll
             for (int t = 1; t < MT; ++t)
-                if (j == t) sj = sc[t];
+                if (j == t) {
+                    sj = sc[t];
+                    rj = rsc[t];
+                }
             uint32_t o = 0;
             if (m0 + j < a.M) {
                 float f[4];
                 smem4(xs + size_t(j) * xrow + sbase + c * 4, f);
-                o = quant4(f, sj);
+                o = quant4(f, sj, rj);
             }
             *reinterpret_cast<uint32_t*>(act + j * rowb + c * 4) = o;
         }

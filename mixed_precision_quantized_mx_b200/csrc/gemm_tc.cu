@@ -16,15 +16,14 @@
 //
 // Tile: 128 packed weight rows (UMMA M) x 128 tokens (UMMA N), the whole K.
 // A pipeline stage holds two k-blocks (256 columns of K): 32 KB of int8 weight
-// operand and 32 KB of activations.  Each stage is filled by exactly two copies
-// issued from two different warps -- one bulk copy of the pre-packed weight
-// blocks (int8 rows already in the 128-byte-swizzled operand layout, or the
-// uint4 codes, which land in the upper half of the operand buffer) and one 3-D
-// TMA box of activations -- because on sm_100a copies issued by one thread
-// complete one after another, so few large copies from several issuers are
-// what keeps the tensor cores fed.
+// operand and 32 KB of activations.  Each k-block of a stage is brought by its
+// own copies from its own lane -- a bulk copy of the pre-packed weight block
+// (int8 rows already in the 128-byte-swizzled operand layout, or the uint4 codes,
+// which land in the upper half of the operand buffer) and a 3-D TMA box of
+// activations -- because on sm_100a copies issued by one thread complete one
+// after another, while copies from different lanes and warps overlap.
 // Warp roles (512 threads):
-//   warp 0      weight copies           warp 3      activation copies
+//   warp 0      weight copies (lanes 0, 1) warp 3  activation copies (lanes 0, 1)
 //   warps 1, 2  MMA issuers, one thread each, taking alternate groups: a thread
 //               spends ~150 ns in every barrier wait or commit, about as long as
 //               one group's MMAs take, so two of them keep the tensor core busy
@@ -154,7 +153,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 
     if (warp == 0 || warp == 3) {
         // ------------------------------------------------------------ loaders
-        if (lane == 0 && !a.stall_test) {
+        // lane kbi copies k-block kbi of each stage: copies from one thread complete
+        // one after another, copies from different lanes overlap
+        if (lane < kKbPerStage && !a.stall_test) {
             const bool weights = warp == 0;
             int it = 0;
             for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
@@ -164,25 +165,32 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 for (int sp = 0; sp < n_ss; ++sp, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
-                    if (!mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, a.status, a.timeout_ns)) goto load_done;
+                    bool ok = true;
+                    if (lane == 0) ok = mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, a.status, a.timeout_ns);
+                    if (!__shfl_sync(0x3u, ok, 0)) goto load_done;
                     const int kb0 = sp * kKbPerStage;
+                    const int nkb = min(kKbPerStage, g.kblocks - kb0);
                     if (weights) {
-                        const int nkb = min(kKbPerStage, g.kblocks - kb0);
-                        const uint32_t bytes = uint32_t(nkb * (eight ? kABytes : kRawBytes));
-                        const uint8_t* src =
-                            eight ? reinterpret_cast<const uint8_t*>(g.codes8) + (size_t(lt) * g.kblocks + kb0) * kABytes
-                                  : g.codes4 + (size_t(lt) * g.kblocks + kb0) * kRawBytes;
-                        mbar_arrive_expect_tx(&S.full[s], bytes);
-                        bulk_g2s(eight ? S.A[s] : S.A[s] + kABytes, src, bytes, &S.full[s]);
+                        const uint32_t per = uint32_t(eight ? kABytes : kRawBytes);
+                        if (lane == 0) mbar_arrive_expect_tx(&S.full[s], uint32_t(nkb) * per);
+                        __syncwarp(0x3u);
+                        if (lane < nkb) {
+                            const uint8_t* src =
+                                eight ? reinterpret_cast<const uint8_t*>(g.codes8) +
+                                            (size_t(lt) * g.kblocks + kb0 + lane) * kABytes
+                                      : g.codes4 + (size_t(lt) * g.kblocks + kb0 + lane) * kRawBytes;
+                            bulk_g2s((eight ? S.A[s] : S.A[s] + kABytes) + lane * per, src, per, &S.full[s]);
+                        }
                     } else {
-                        // the box always spans two k-blocks; a missing last one reads as zeros
-                        mbar_arrive_expect_tx(&S.full[s], kKbPerStage * kBBytes);
-                        tma_load_3d(S.B[s], &amap, 0, tt * BN, kb0, &S.full[s]);
+                        // one box per k-block; a missing last one reads as zeros
+                        if (lane == 0) mbar_arrive_expect_tx(&S.full[s], kKbPerStage * kBBytes);
+                        __syncwarp(0x3u);
+                        tma_load_3d(S.B[s] + lane * kBBytes, &amap, 0, tt * BN, kb0 + lane, &S.full[s]);
                     }
                 }
             }
         load_done:
-            drain_stages(S, it, a.timeout_ns);
+            if (lane == 0) drain_stages(S, it, a.timeout_ns);
         }
     } else if (warp == 1 || warp == 2) {
         // ------------------------------------------------------------ MMA issuers
@@ -341,34 +349,34 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     const bool ok = mbar_wait_bounded(&S.acc_full[b], u & 1, abort, a.status, a.timeout_ns);
                     if (!__all_sync(0xffffffffu, ok)) goto epi_done;
                     tc_fence_after();
-                    // drain the group's 64 columns in four 16-column chunks, loading chunk
+                    // drain the group's 64 columns in eight 8-column chunks, loading chunk
                     // h+1 while chunk h is converted; each chunk is re-armed with the bias
                     const uint32_t col0 = lane_addr + b * BN + cb;
-                    uint32_t va[16], vb[16];
-                    tmem_ld_x16(col0, va);
+                    uint32_t va[8], vb[8];
+                    tmem_ld_x8(col0, va);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        uint32_t (&v)[16] = (h & 1) ? vb : va;
-                        uint32_t (&vn)[16] = (h & 1) ? va : vb;
-                        if (h < 3) tmem_ld_x16(col0 + (h + 1) * 16, vn);
-                        tmem_st_x16_splat(col0 + h * 16, kI2FBiasBits);
+                    for (int h = 0; h < 8; ++h) {
+                        uint32_t (&v)[8] = (h & 1) ? vb : va;
+                        uint32_t (&vn)[8] = (h & 1) ? va : vb;
+                        if (h < 7) tmem_ld_x8(col0 + (h + 1) * 8, vn);
+                        tmem_st_x8_splat(col0 + h * 8, kI2FBiasBits);
                         // acc += (float(bias + P) - bias) * s_w, two columns per instruction
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
+                        for (int c = 0; c < 4; ++c) {
                             const float2 f = add2(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])),
                                                   nbias);
-                            acc[h * 8 + c] = fma2(f, s2, acc[h * 8 + c]);
+                            acc[h * 4 + c] = fma2(f, s2, acc[h * 4 + c]);
                         }
                         if (DEBUG && orig >= 0) {
 #pragma unroll
-                            for (int c = 0; c < 16; ++c) {
-                                const int m = tt * BN + cb + h * 16 + c;
+                            for (int c = 0; c < 8; ++c) {
+                                const int m = tt * BN + cb + h * 8 + c;
                                 if (m < a.M)
                                     a.debug[(size_t(m) * g.N + orig) * g.G + gi] = int32_t(v[c] - kI2FBiasBits);
                             }
                         }
-                        if (h < 3) tmem_wait_ld();
+                        if (h < 7) tmem_wait_ld();
                     }
                     tmem_wait_st();
                     tc_fence_before();
@@ -430,12 +438,12 @@ cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* A
     cudaError_t e;
     EncodeTiledFn enc = encode_fn(&e);
     if (e != cudaSuccess) return e;
-    // activations as a 3-D tensor [k-block][token][128 bytes], so one box brings
-    // two k-blocks of BN tokens, each landing as its own swizzled 128-byte-row block
+    // activations as a 3-D tensor [k-block][token][128 bytes]: one box brings one
+    // k-block of BN tokens as a swizzled 128-byte-row block
     CUtensorMap map;
     const cuuint64_t dims[3] = {cuuint64_t(kKBlock), cuuint64_t(M), cuuint64_t(L.kblocks)};
     const cuuint64_t strides[2] = {cuuint64_t(L.K), cuuint64_t(kKBlock)};
-    const cuuint32_t box[3] = {cuuint32_t(kKBlock), cuuint32_t(BN), cuuint32_t(kKbPerStage)};
+    const cuuint32_t box[3] = {cuuint32_t(kKBlock), cuuint32_t(BN), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(Aq), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

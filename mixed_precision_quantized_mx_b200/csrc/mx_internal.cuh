@@ -56,16 +56,65 @@ __device__ __forceinline__ __half act_scale(float amax) {
     return h;
 }
 
-// four codes clamp(round_half_even(x / s), -127, 127) packed little-endian
-__device__ __forceinline__ uint32_t quant4(const float* v, float s) {
-    uint32_t w = 0;
+// One code clamp(round_half_even(fl(x / s)), -127, 127), with fl the IEEE fp32
+// division.  t = fl(x * fl(1/s)) is within 1.5 * 2^-23 |t| of fl(x / s) (two
+// roundings of at most 2^-24 each), so wherever t is farther than that from a
+// half-integer, round(t) is the code; only values closer than 1e-4 to a rounding
+// boundary (and NaN) take the IEEE division.  Beyond |t| = 200 both round past
+// 127 and clamp alike.  round(t) is t + 1.5 * 2^23 in fp32 (round-half-even to an
+// integer for |t| < 2^22), read back from the sum's bits, so no conversion
+// instruction is needed on the fast path.
+__device__ __forceinline__ int32_t quant_code_exact(float x, float s) {
+    return int32_t(fminf(fmaxf(rintf(__fdiv_rn(x, s)), -127.0f), 127.0f));
+}
+
+// The fast path without branches; *slow is set when x needs quant_code_exact.
+__device__ __forceinline__ int32_t quant_code_fast(float x, float rs, bool* slow) {
+    constexpr float kMagic = 12582912.0f;            // 1.5 * 2^23
+    const float t = __fmul_rn(x, rs);
+    const float tb = __fadd_rn(t, kMagic);
+    const float gap = __fsub_rn(0.5f, fabsf(__fsub_rn(t, __fsub_rn(tb, kMagic))));
+    const bool big = fabsf(t) > 200.0f;               // false for NaN
+    const int32_t q = min(max(__float_as_int(tb) - __float_as_int(kMagic), -127), 127);
+    *slow = !big && !(gap > 1.0e-4f);                 // near a boundary, or NaN
+    return big ? (t > 0.0f ? 127 : -127) : q;
+}
+
+__device__ __forceinline__ int32_t quant_code(float x, float s, float rs) {
+    bool slow;
+    const int32_t q = quant_code_fast(x, rs, &slow);
+    return slow ? quant_code_exact(x, s) : q;
+}
+
+// |x| maximum of eight values (exact in the input type; fp16 stays packed)
+__device__ __forceinline__ float absmax8(const __half* p, float m) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(p);
+    const __half2* h = reinterpret_cast<const __half2*>(&raw);
+    __half2 a = __hmax2(__habs2(h[0]), __habs2(h[1]));
+    a = __hmax2(a, __hmax2(__habs2(h[2]), __habs2(h[3])));
+    return fmaxf(m, fmaxf(__low2float(a), __high2float(a)));
+}
+__device__ __forceinline__ float absmax8(const float* p, float m) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+    return fmaxf(m, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
+}
+
+// four codes packed little-endian; rs = __frcp_rn(s).  One branch for all four,
+// taken only when one of them lies at a rounding boundary.
+__device__ __forceinline__ uint32_t quant4(const float* v, float s, float rs) {
+    bool sl[4];
+    int32_t q[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float q = rintf(__fdiv_rn(v[i], s));
-        q = fminf(fmaxf(q, -127.0f), 127.0f);
-        w |= (uint32_t(int32_t(q)) & 0xFFu) << (8 * i);
+    for (int i = 0; i < 4; ++i) q[i] = quant_code_fast(v[i], rs, &sl[i]);
+    if (sl[0] | sl[1] | sl[2] | sl[3]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (sl[i]) q[i] = quant_code_exact(v[i], s);
     }
-    return w;
+    return (uint32_t(q[0]) & 0xFFu) | ((uint32_t(q[1]) & 0xFFu) << 8) | ((uint32_t(q[2]) & 0xFFu) << 16) |
+           (uint32_t(q[3]) << 24);
 }
 
 // Byte offset of the 16-byte chunk holding k = 16c..16c+15 of row r inside a
@@ -123,6 +172,21 @@ cudaError_t launch_gemm_decode(const mx_layout& L, const void* blob, const int8_
                                const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy,
                                const DecodePlan& plan, int32_t* debug_partials, int32_t* status,
                                cudaStream_t s);
+
+// decode GEMM for short K (<= 8192) and M <= 4: every CTA owns whole rows (16 4-bit
+// or 8 8-bit), no split of K.  Reads Aq / s_a, or quantizes X (fp16 / fp32) itself.
+struct RowsPlan {
+    bool ok;            // shape served (K, M, one wave, shared memory)
+    int mt, m_tiles;    // tokens per CTA (1, 2, 4); ceil(M / mt)
+    int n8u, units;     // 8-bit units; all units
+    size_t smem;
+    int off_sc, off_z, off_act, off_sa64, off_raw, off_red;
+};
+// x_bytes: 0 when the kernel reads Aq, else 2 / 4 (fp16 / fp32 X staged in shared memory)
+RowsPlan plan_rows(const mx_layout& L, int M, int x_bytes);
+cudaError_t launch_gemm_rows(const mx_layout& L, const void* blob, const int8_t* Aq, const uint16_t* s_a,
+                             const void* X, mx_dtype xdt, int64_t ldx, int M, uint16_t* Y, int64_t ldy,
+                             const RowsPlan& p, int32_t* debug_partials, int32_t* status, cudaStream_t s);
 
 // decode GEMM that quantizes X itself (M <= kMaxFusedTokens): one launch per call
 constexpr int kMaxFusedTokens = 4;

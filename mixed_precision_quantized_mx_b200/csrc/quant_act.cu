@@ -33,12 +33,7 @@ quant_act_kernel(const T* __restrict__ X, int K, int64_t ldx, int8_t* __restrict
     const int nvec = K / 8;
 
     float amax = 0.0f;
-    for (int i = threadIdx.x; i < nvec; i += kThreads) {
-        float v[8];
-        load8(x + i * 8, v);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
-    }
+    for (int i = threadIdx.x; i < nvec; i += kThreads) amax = absmax8(x + i * 8, amax);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     __shared__ float red[kThreads / 32];
@@ -54,15 +49,15 @@ quant_act_kernel(const T* __restrict__ X, int K, int64_t ldx, int8_t* __restrict
         s_shared = __half2float(h);
     }
     __syncthreads();
-    const float s = s_shared;
+    const float s = s_shared, rs = __frcp_rn(s);
 
     int8_t* q = Aq + int64_t(m) * K;
     for (int i = threadIdx.x; i < nvec; i += kThreads) {
         float v[8];
         load8(x + i * 8, v);
         uint2 out;
-        out.x = quant4(v, s);
-        out.y = quant4(v + 4, s);
+        out.x = quant4(v, s, rs);
+        out.y = quant4(v + 4, s, rs);
         *reinterpret_cast<uint2*>(q + i * 8) = out;
     }
 }

@@ -75,6 +75,29 @@ def test_quant_act_special_rows(orc):
     check_quant(orc, X[[0, 1, 2, 4, 5]].astype(np.float16))       # rows that fp16 can hold
 
 
+def test_quant_act_rounding_boundaries(orc):
+    """Values at and one ulp either side of every half-integer multiple of the scale:
+    the codes are decided by fl(x / s), the IEEE fp32 quotient, then round-half-even."""
+    K = 1024
+    rng = np.random.default_rng(21)
+    rows = []
+    for amax in (127.0, 100.0, 3.0, 0.37, 1.0e-3):
+        s = np.float32(np.float16(np.float32(amax) / np.float32(127.0)))   # the fp16 scale
+        k = rng.integers(-127, 127, K).astype(np.float32)
+        x = (k + np.float32(0.5)) * s                                     # near ties
+        nudge = rng.integers(-1, 2, K)                                    # -1, 0, +1 ulp
+        x = np.where(nudge > 0, np.nextafter(x, np.float32(np.inf)),
+                     np.where(nudge < 0, np.nextafter(x, np.float32(-np.inf)), x)).astype(np.float32)
+        x = np.clip(x, -amax, amax)
+        x[0] = amax                                                       # pins the scale
+        rows.append(x)
+    X = np.stack(rows).astype(np.float32)
+    Aq, sa, Aq_o, sa_o = check_quant(orc, X)
+    # the rows hit every kind of decision: exact ties and both neighbours
+    q = Aq_o.astype(np.float64)
+    assert (np.abs(q) == 127).any() and len(np.unique(q)) > 200
+
+
 def test_quant_act_strided_rows(orc):
     rng = np.random.default_rng(3)
     Xbig = inputs.activations(rng, 9, 640, 6)
