@@ -403,9 +403,10 @@ def main():
             traffic = rec["dram_bytes_per_launch"]
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": ("gemm_decode_kernel, activation quantizer fused (cluster split-K, CUDA cores)"
-                           if fused else "gemm_decode_kernel (cluster split-K, CUDA cores)" if path_used == 1
-                           else "gemm_tc_kernel (tcgen05)"),
+                "kernel": {1: "gemm_decode_kernel (cluster split-K, CUDA cores)",
+                           2: "gemm_tc_kernel (tcgen05)",
+                           3: "gemm_rows_kernel (whole rows per CTA, CUDA cores)"}[path_used]
+                          + (", activation quantizer fused" if fused else ""),
                 "algorithmic_per_launch": algo, "launch_ms": gemm_ms,
                 "peak_source": (f"{peaks['source']} HBM copy" if bound == "hbm" else
                                 f"{peaks['source']} bf16 cuBLAS burst x 2 (nominal int8/bf16 ratio)")}

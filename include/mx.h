@@ -97,9 +97,11 @@ typedef struct mx_layout {
 
 /* Options of mx_gemm; pass NULL for the defaults (all fields zero). */
 typedef struct mx_gemm_opts {
-    int32_t path;              /* 0 auto; 1 split-K CUDA-core path; 2 tensor-core path */
+    int32_t path;              /* 0 auto; 1 split-K CUDA-core path; 2 tensor-core path;
+                                  3 row CUDA-core path (whole rows per CTA) */
     int32_t split;             /* path 1: CTAs (a thread-block cluster, 1..8) that split
-                                  the K range of each row unit (0 = auto) */
+                                  the K range of each row unit (0 = auto); a split
+                                  asked for under auto selects path 1 */
     int32_t* debug_partials;   /* device int32 [M][N][G] or NULL: every per-group
                                   int32 partial P[m][n][g] (original row order) */
     int32_t* status;           /* device int32 or NULL: kernel-side error code */
@@ -179,10 +181,14 @@ mx_status mx_gemm_workspace_size(const mx_layout* L, int M, const mx_gemm_opts* 
 
 /*
  * mx_gemm_select_path -- host only.  The GEMM path mx_gemm will take for this
- * layer at M tokens with these options: 1 = split-K CUDA-core path (decode-sized
- * M <= 16, HBM-bound; the K split of each row unit is one thread-block cluster
- * reduced through distributed shared memory), 2 = tensor-core path.  Negative
- * mx_status on bad arguments.
+ * layer at M tokens with these options.  The decode-sized paths are HBM-bound
+ * and run on CUDA cores:
+ *   3 = row path: M <= 4, K <= 4096 and one wave of CTAs; every CTA owns 32
+ *       4-bit (or 16 8-bit) rows over the whole K, no reduction between CTAs;
+ *   1 = split-K path: M <= 16; the K split of each row unit is one thread-block
+ *       cluster reduced through distributed shared memory;
+ *   2 = tensor-core path (larger M).
+ * Auto selection tries them in that order.  Negative mx_status on bad arguments.
  */
 int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts);
 
@@ -222,12 +228,13 @@ mx_status mx_linear_workspace_size(const mx_layout* L, int M, mx_dtype xdtype,
  *   Y       device fp16 [M][ldy], ldy >= N; column n is original row n of W
  *   workspace / ws_bytes: device scratch of at least mx_linear_workspace_size
  *           bytes (may be NULL when that is 0)
- * When the decode path serves the call (mx_gemm_select_path == 1), M <= 4 and
- * the activation rows take at most 64 KB, one kernel does both steps: each CTA
- * takes the absmax of the whole token row and quantizes only its own K slice,
- * with the same operations as mx_quant_act, so the codes -- and Y -- are
- * identical to mx_quant_act followed by mx_gemm.  Otherwise mx_quant_act and
- * mx_gemm run back to back on `stream` with Aq and s_a in the workspace.
+ * One kernel does both steps on the row path (mx_gemm_select_path == 3: each CTA
+ * quantizes the whole token rows it needs) and on the split-K path when M <= 4
+ * and the activation rows take at most 64 KB (each CTA takes the row absmax from
+ * its cluster and quantizes only its own K slice).  Both use the operations of
+ * mx_quant_act, so the codes -- and Y -- are identical to mx_quant_act followed
+ * by mx_gemm.  Otherwise mx_quant_act and mx_gemm run back to back on `stream`
+ * with Aq and s_a in the workspace.
  * Returns MX_ERR_WORKSPACE if the workspace is missing or too small.
  */
 mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtype xdtype, int M,

@@ -166,16 +166,13 @@ mx_status mx_quant_act(const void* X, mx_dtype xdtype, int M, int K, int64_t ldx
 // weights with enough CTAs; from 17 tokens on, the tensor-core path.
 constexpr int kDecodeMaxM = 16;
 
+// Short K and M <= 4 take the row kernel (whole rows per CTA) unless a cluster
+// split is asked for.
 static int choose_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
     if (opts && opts->path) return opts->path;
+    if (!(opts && opts->split > 0) && mx::plan_rows(*L, M, 0).ok) return 3;
     if (M <= kDecodeMaxM && mx::plan_decode(*L, M, 0).ok) return 1;
     return 2;
-}
-
-// On the decode path, short K and M <= 4 go to the row kernel (whole rows per
-// CTA) unless a cluster split is asked for explicitly.
-static bool rows_serves(const mx_layout* L, int M, const mx_gemm_opts* opts) {
-    return !(opts && opts->split > 0) && mx::plan_rows(*L, M, 0).ok;
 }
 
 int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
@@ -214,15 +211,16 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
     if (opts && opts->status && (st = check_device_ptr(opts->status, "status")) != MX_OK) return st;
     const int path = choose_path(L, M, opts);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (path == 3) {
+        const mx::RowsPlan rp = mx::plan_rows(*L, M, 0);
+        if (!rp.ok) return fail(MX_ERR_UNSUPPORTED, "M=%d K=%d: beyond the row path (M <= 4, K <= 4096, one wave)", M, L->K);
+        cudaError_t e = mx::launch_gemm_rows(*L, blob, Aq, s_a, nullptr, MX_F16, 0, M, Y, ldy, rp,
+                                             opts ? opts->debug_partials : nullptr, opts ? opts->status : nullptr, s);
+        if (e != cudaSuccess) return cuda_fail(e, "row decode GEMM launch");
+        return MX_OK;
+    }
     if (path == 1) {
         if (opts && opts->split > 8) return fail(MX_ERR_UNSUPPORTED, "split=%d above the cluster limit 8", opts->split);
-        if (rows_serves(L, M, opts)) {
-            cudaError_t e = mx::launch_gemm_rows(*L, blob, Aq, s_a, nullptr, MX_F16, 0, M, Y, ldy, mx::plan_rows(*L, M, 0),
-                                                 opts ? opts->debug_partials : nullptr,
-                                                 opts ? opts->status : nullptr, s);
-            if (e != cudaSuccess) return cuda_fail(e, "row decode GEMM launch");
-            return MX_OK;
-        }
         mx::DecodePlan plan = mx::plan_decode(*L, M, opts ? opts->split : 0);
         if (!plan.ok)
             return fail(MX_ERR_UNSUPPORTED, "M=%d K=%d: activation slice too large for the decode path", M, L->K);
@@ -255,9 +253,9 @@ size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
 int x_bytes(mx_dtype xdt) { return xdt == MX_F16 ? 2 : 4; }
 
 bool linear_fused(const mx_layout* L, int M, mx_dtype xdt, const mx_gemm_opts* opts) {
-    if (choose_path(L, M, opts) != 1) return false;
-    if (rows_serves(L, M, opts)) return true;
-    if (!mx::decode_can_fuse(*L, M, xdt)) return false;
+    const int path = choose_path(L, M, opts);
+    if (path == 3) return mx::plan_rows(*L, M, 0).ok;
+    if (path != 1 || !mx::decode_can_fuse(*L, M, xdt)) return false;
     const mx::DecodePlan p = mx::plan_decode(*L, M, opts ? opts->split : 0, x_bytes(xdt));
     return p.ok && p.mt <= mx::kMaxFusedTokens;
 }
@@ -298,8 +296,7 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
         if (opts && opts->debug_partials && (st = check_device_ptr(opts->debug_partials, "debug_partials")) != MX_OK)
             return st;
         if (opts && opts->status && (st = check_device_ptr(opts->status, "status")) != MX_OK) return st;
-        if (opts && opts->split > 8) return fail(MX_ERR_UNSUPPORTED, "split=%d above the cluster limit 8", opts->split);
-        if (rows_serves(L, M, opts)) {
+        if (choose_path(L, M, opts) == 3) {
             cudaError_t e = mx::launch_gemm_rows(*L, blob, nullptr, nullptr, X, xdtype, ldx, M, Y, ldy,
                                                  mx::plan_rows(*L, M, x_bytes(xdtype)),
                                                  opts ? opts->debug_partials : nullptr,
@@ -307,6 +304,7 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
             if (e != cudaSuccess) return cuda_fail(e, "row decode GEMM launch");
             return MX_OK;
         }
+        if (opts && opts->split > 8) return fail(MX_ERR_UNSUPPORTED, "split=%d above the cluster limit 8", opts->split);
         mx::DecodePlan plan = mx::plan_decode(*L, M, opts ? opts->split : 0, x_bytes(xdtype));
         cudaError_t e = mx::launch_gemm_decode_fused(*L, blob, X, xdtype, ldx, M, Y, ldy, plan,
                                                      opts ? opts->debug_partials : nullptr,

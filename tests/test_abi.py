@@ -123,13 +123,19 @@ def test_paths_need_no_workspace_and_dispatch_on_m(lib):
     L = mx.mx_layout_init(4096, 4096, 128, 410)
     for M in (1, 16, 17, 2048):
         assert mx.mx_gemm_workspace_size(L, M) == 0
-    assert mx.mx_gemm_select_path(L, 1) == mx.PATH_SPLITK
+    assert mx.mx_gemm_select_path(L, 1) == mx.PATH_ROWS          # short K, M <= 4, one wave
+    assert mx.mx_gemm_select_path(L, 4) == mx.PATH_ROWS
+    assert mx.mx_gemm_select_path(L, 5) == mx.PATH_SPLITK
+    assert mx.mx_gemm_select_path(L, 1, split=2) == mx.PATH_SPLITK   # a split asks for clusters
     assert mx.mx_gemm_select_path(L, 16) == mx.PATH_SPLITK
     assert mx.mx_gemm_select_path(L, 17) == mx.PATH_TENSOR
     assert mx.mx_gemm_select_path(L, 1, path=mx.PATH_TENSOR) == mx.PATH_TENSOR
     # 16 tokens of a 64K-column activation slice cannot be staged per cluster: tensor cores
     Lbig = mx.mx_layout_init(1024, 65536, 128, 102)
     assert mx.mx_gemm_select_path(Lbig, 16) == mx.PATH_TENSOR
+    # the row path needs K <= 4096 and one wave of CTAs
+    assert mx.mx_gemm_select_path(mx.mx_layout_init(4096, 8192, 128, 410), 1) == mx.PATH_SPLITK
+    assert mx.mx_gemm_select_path(mx.mx_layout_init(14336, 4096, 128, 1434), 1) == mx.PATH_SPLITK
 
 
 def test_linear_workspace_follows_the_fused_decode_rule(lib):

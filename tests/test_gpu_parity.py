@@ -297,6 +297,35 @@ def test_gemm_tc_degenerate_fractions(orc, frac):
     run_and_check(orc, X, W, is8, 128, path=mx.PATH_TENSOR)
 
 
+# ------------------------------------------------------------------ row path (3)
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("g", [64, 128])
+def test_rows_path(orc, M, g):
+    lay = inputs.llama_layer(M, 1024, 520, group=g, seed=40 + M + g)
+    run_and_check(orc, lay.X, lay.W, lay.is8, g, path=mx.PATH_ROWS)
+
+
+@pytest.mark.parametrize("N,K,n8", [(256, 512, 0), (256, 512, 256), (130, 384, 3), (4096, 4096, 410),
+                                    (1000, 128, 100)])
+def test_rows_path_shapes(orc, N, K, n8):
+    rng = np.random.default_rng(N + K + n8)
+    W = inputs.weights(rng, N, K, outlier_frac=0.001)
+    is8 = inputs.saliency_mask(np.abs(rng.standard_normal(N)), n8)
+    X = inputs.activations(rng, 2, K, max(1, K // 100))
+    run_and_check(orc, X, W, is8, 128, path=mx.PATH_ROWS)
+
+
+def test_rows_path_refuses_what_it_cannot_serve():
+    rng = np.random.default_rng(5)
+    for N, K, M in ((256, 8192, 1), (256, 512, 5)):
+        L, blob = gpu_pack(inputs.weights(rng, N, K), inputs.saliency_mask(np.abs(rng.standard_normal(N)), 10), 128)
+        Aq, sa = gpu_quant(inputs.activations(rng, M, K, 4))
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev())
+        with pytest.raises(mx.MXError) as e:
+            mx.mx_gemm(L, blob, Aq, sa, Y, path=mx.PATH_ROWS)
+        assert e.value.status == 2
+
+
 def test_paths_agree_bit_exact_partials(orc):
     rng = np.random.default_rng(21)
     M, N, K = 24, 400, 1024
