@@ -3,10 +3,11 @@
 // Two-step dequantization (MixLLM section 3.3) on 5th-generation tensor cores:
 //   step 1: per quantization group, P = A_q . (W_q - z)^T with tcgen05.mma
 //           kind::i8 (int8 x int8 -> int32) into a TMEM accumulator that holds
-//           only that group's sum; the accumulator starts at the fast-I2F bias
-//           integer (section 3.3: the accumulator is initialised with the bias),
-//   step 2: the epilogue warps read bias + P from TMEM, subtract the float bias
-//           (section 3.3, Figure 3) and accumulate acc += float(P) * s_w[row, group]
+//           only that group's sum (the group's first MMA overwrites it),
+//   step 2: the epilogue warps read P from TMEM, convert it with the fast
+//           int-to-float of section 3.3 (Figure 3: add the bias integer, read the
+//           bits as fp32, subtract the float bias) and accumulate
+//           acc += float(P) * s_w[row, group]
 //           in fp32 registers; at the end of the tile Y = fp16(acc * s_a[token])
 //           is scattered to the original output columns (section 3.3, fused
 //           scatter epilogue).
@@ -53,6 +54,9 @@ constexpr int kStages = 3;
 constexpr int kABytes = BM * kKBlock;          // int8 weight operand of one k-block
 constexpr int kBBytes = BN * kKBlock;          // int8 activation operand of one k-block
 constexpr int kRawBytes = BM * kKBlock / 2;    // uint4 codes of one k-block
+// the uint4 codes of a stage land at the top of its weight-operand buffer and are
+// widened in place, k-block after k-block, into the int8 operand below them
+constexpr int kRawBase = kKbPerStage * (kABytes - kRawBytes);
 constexpr int kThreads = 512;
 constexpr int kWidenThreads = 128;
 constexpr int kEpiWarps = 8;
@@ -63,7 +67,7 @@ constexpr int kMmaIssuers = 2;                  // MMA-issuing threads, alternat
 constexpr int kScaleRing = 4;                   // group scales in flight per epilogue thread
 
 struct __align__(1024) Smem {
-    uint8_t A[kStages][kKbPerStage * kABytes];  // raw uint4 codes land at A + kABytes
+    uint8_t A[kStages][kKbPerStage * kABytes];  // raw uint4 codes land at A + kRawBase
     uint8_t B[kStages][kKbPerStage * kBBytes];
     uint64_t full[kStages];       // both copies of the stage landed (2 arrivals + bytes)
     uint64_t wdone[kStages];      // widen -> MMA: weight operand ready
@@ -140,22 +144,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
-    if (warp >= 8) {
-        // every group accumulator starts at the fast-I2F bias, so all MMAs accumulate
-        const uint32_t la = tmem + (uint32_t((warp & 3) * 32) << 16) + ((warp - 8) >> 2) * 64;
-        for (int b = 0; b < kAccBufs; ++b)
-            for (int h = 0; h < 2; ++h) tmem_st_x32_splat(la + b * BN + h * 32, kI2FBiasBits);
-        tmem_wait_st();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
 
     if (warp == 0 || warp == 3) {
         // ------------------------------------------------------------ loaders
         // lane kbi copies k-block kbi of each stage: copies from one thread complete
         // one after another, copies from different lanes overlap
         if (lane < kKbPerStage && !a.stall_test) {
+            constexpr uint32_t kLanes = (1u << kKbPerStage) - 1u;   // the issuing lanes
             const bool weights = warp == 0;
             int it = 0;
             for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
@@ -167,24 +162,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     const uint32_t ph = (it / kStages) & 1;
                     bool ok = true;
                     if (lane == 0) ok = mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, a.status, a.timeout_ns);
-                    if (!__shfl_sync(0x3u, ok, 0)) goto load_done;
+                    if (!__shfl_sync(kLanes, ok, 0)) goto load_done;
                     const int kb0 = sp * kKbPerStage;
                     const int nkb = min(kKbPerStage, g.kblocks - kb0);
                     if (weights) {
                         const uint32_t per = uint32_t(eight ? kABytes : kRawBytes);
                         if (lane == 0) mbar_arrive_expect_tx(&S.full[s], uint32_t(nkb) * per);
-                        __syncwarp(0x3u);
+                        __syncwarp(kLanes);
                         if (lane < nkb) {
                             const uint8_t* src =
                                 eight ? reinterpret_cast<const uint8_t*>(g.codes8) +
                                             (size_t(lt) * g.kblocks + kb0 + lane) * kABytes
                                       : g.codes4 + (size_t(lt) * g.kblocks + kb0 + lane) * kRawBytes;
-                            bulk_g2s((eight ? S.A[s] : S.A[s] + kABytes) + lane * per, src, per, &S.full[s]);
+                            bulk_g2s((eight ? S.A[s] : S.A[s] + kRawBase) + lane * per, src, per, &S.full[s]);
                         }
                     } else {
                         // one box per k-block; a missing last one reads as zeros
                         if (lane == 0) mbar_arrive_expect_tx(&S.full[s], kKbPerStage * kBBytes);
-                        __syncwarp(0x3u);
+                        __syncwarp(kLanes);
                         tma_load_3d(S.B[s] + lane * kBBytes, &amap, 0, tt * BN, kb0 + lane, &S.full[s]);
                     }
                 }
@@ -216,10 +211,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                             if (!mbar_wait_bounded(&S.acc_empty[b], (u & 1) ^ 1, abort, a.status, a.timeout_ns))
                                 goto mma_out;
                             tc_fence_after();
+                            // the group's first k-step overwrites the accumulator, the rest add
                             for (int kk = 0; kk < ksteps; ++kk) {
                                 const uint32_t off = uint32_t(j * g.group + kk * 32);
                                 mma_i8(tmem + b * BN, sw128_kmajor_desc(a0 + off), sw128_kmajor_desc(b0 + off),
-                                       idesc, 1u);
+                                       idesc, kk > 0 ? 1u : 0u);
                             }
                             mma_commit(&S.acc_full[b]);
                         }
@@ -267,14 +263,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 // needs every one of them at the named barrier
                 if (!named_bar_and(kWidenBarrier, kWidenThreads, ok)) return false;
                 if (!eight) {
-                    const uint8_t* raw = S.A[s] + kABytes;
+                    const uint8_t* raw = S.A[s] + kRawBase;
                     for (int kbi = 0; kbi < nkb; ++kbi) {
                         uint4 w[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
                             w[j] = *reinterpret_cast<const uint4*>(raw + kbi * kRawBytes + (wt + kWidenThreads * j) * 16);
-                        // the second k-block overwrites the codes it reads: all reads first
-                        if (kbi == 1) named_bar_and(kWidenBarrier, kWidenThreads, true);
+                        // once the int8 block reaches the codes, every thread reads before any writes
+                        if ((kbi + 1) * kABytes > kRawBase) named_bar_and(kWidenBarrier, kWidenThreads, true);
                         uint8_t* out = S.A[s] + kbi * kABytes;
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
@@ -350,7 +346,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     if (!__all_sync(0xffffffffu, ok)) goto epi_done;
                     tc_fence_after();
                     // drain the group's 64 columns in eight 8-column chunks, loading chunk
-                    // h+1 while chunk h is converted; each chunk is re-armed with the bias
+                    // h+1 while chunk h is converted
                     const uint32_t col0 = lane_addr + b * BN + cb;
                     uint32_t va[8], vb[8];
                     tmem_ld_x8(col0, va);
@@ -360,11 +356,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                         uint32_t (&v)[8] = (h & 1) ? vb : va;
                         uint32_t (&vn)[8] = (h & 1) ? va : vb;
                         if (h < 7) tmem_ld_x8(col0 + (h + 1) * 8, vn);
-                        tmem_st_x8_splat(col0 + h * 8, kI2FBiasBits);
-                        // acc += (float(bias + P) - bias) * s_w, two columns per instruction
+                        // acc += (float(bias + P) - bias) * s_w: the fast int-to-float adds the
+                        // bias as an integer, two columns per float instruction
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
-                            const float2 f = add2(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])),
+                            const float2 f = add2(make_float2(__uint_as_float(v[2 * c] + kI2FBiasBits),
+                                                              __uint_as_float(v[2 * c + 1] + kI2FBiasBits)),
                                                   nbias);
                             acc[h * 4 + c] = fma2(f, s2, acc[h * 4 + c]);
                         }
@@ -373,12 +370,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                             for (int c = 0; c < 8; ++c) {
                                 const int m = tt * BN + cb + h * 8 + c;
                                 if (m < a.M)
-                                    a.debug[(size_t(m) * g.N + orig) * g.G + gi] = int32_t(v[c] - kI2FBiasBits);
+                                    a.debug[(size_t(m) * g.N + orig) * g.G + gi] = int32_t(v[c]);
                             }
                         }
                         if (h < 7) tmem_wait_ld();
                     }
-                    tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.acc_empty[b]);
