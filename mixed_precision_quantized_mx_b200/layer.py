@@ -113,4 +113,6 @@ class GraphedLinear:
             body()
 
     def replay(self) -> None:
-        self.graph.replay()
+        """Launch the captured pass on `self.stream` (a graph replays on the current stream)."""
+        with torch.cuda.stream(self.stream):
+            self.graph.replay()

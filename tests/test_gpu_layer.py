@@ -43,8 +43,12 @@ def test_graphed_host_in_host_out(orc, M):
     for seed in (1, 2):                      # new input in the same pinned buffer each call
         X = inputs.activations(np.random.default_rng(seed), M, 1024, 10)
         x_host.copy_(torch.from_numpy(X))
-        runner.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(runner.stream)
+        runner.replay()                      # runs on runner.stream, whatever stream is current
+        e1.record(runner.stream)
         runner.stream.synchronize()
+        assert e0.elapsed_time(e1) > 0.001   # the copies and the kernel ran between the events
         assert_y_close(runner.y_host.numpy(), oracle_y(orc, X, lay.W, lay.is8, 128))
 
 
