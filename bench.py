@@ -58,7 +58,10 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     p.add_argument("--frac8", type=float, default=0.10)
     p.add_argument("--group", type=int, default=128)
-    p.add_argument("--path", type=int, default=0, help="0 auto, 1 split-K CUDA cores, 2 tensor cores")
+    p.add_argument("--path", type=int, default=0,
+                   help="0 auto, 1 split-K CUDA cores, 2 tensor cores, 3 whole rows per CTA")
+    p.add_argument("--act-group", type=int, default=0,
+                   help="activation scales: 0 one per token; the weight group: one per token and group")
     p.add_argument("--impl", default="mx", choices=["mx", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
@@ -161,7 +164,7 @@ def oracle_step_sample(lay, budget_s: float = 0.5):
     return m, n, f"{budget} random (token, row) outputs of {M}x{N}"
 
 
-def time_oracle(lay, canonical, steps: int, min_seconds: float = 0.0):
+def time_oracle(lay, canonical, steps: int, min_seconds: float = 0.0, act_group: int = 0):
     """Run the oracle's quantize + sampled GEMM; return (seconds per step, sample, fraction)."""
     import oracle
     m, n, desc = oracle_step_sample(lay)
@@ -169,8 +172,8 @@ def time_oracle(lay, canonical, steps: int, min_seconds: float = 0.0):
     X = lay.X.astype(np.float32)
     done, t0 = 0, time.perf_counter()
     while done < steps or time.perf_counter() - t0 < min_seconds:
-        Aq, sa = oracle.quant_act(X)
-        oracle.gemm(Aq, sa, canonical, pairs=(m, n))
+        Aq, sa = oracle.quant_act(X, act_group=act_group)
+        oracle.gemm(Aq, sa, canonical, act_group=act_group, pairs=(m, n))
         done += 1
     return (time.perf_counter() - t0) / done, desc, frac, done
 
@@ -211,8 +214,8 @@ def run_reference(a):
     lay = inputs.llama_layer(M, K, N, a.frac8, a.group, seed=a.seed)
     can = oracle.pack(lay.W, lay.is8, lay.group)
     unit = "GB/s" if M <= HBM_BOUND_MAX_M else "TOPS"
-    time_oracle(lay, can, a.warmup)
-    sec, desc, frac, done = time_oracle(lay, can, a.steps or 5)
+    time_oracle(lay, can, a.warmup, act_group=a.act_group)
+    sec, desc, frac, done = time_oracle(lay, can, a.steps or 5, act_group=a.act_group)
     value = step_units(M, K, N, a.group, lay.n8, unit) * frac / sec
     sample = f"each step: quantize {M}x{K} activations + {desc} (fraction {frac:.3g} of the step)"
     line = {
@@ -221,7 +224,7 @@ def run_reference(a):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": a.workload, "M": M, "K": K, "N": N, "group": a.group,
-                   "frac8": a.frac8, "n8": lay.n8},
+                   "frac8": a.frac8, "n8": lay.n8, "act_group": a.act_group},
         "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -256,6 +259,7 @@ def main():
 
     M, K, N = WORKLOADS[a.workload]
     g = a.group
+    ag = a.act_group
     lay = inputs.llama_layer(M, K, N, a.frac8, g, seed=rank_seed(a.seed, rank))
     n8 = lay.n8
     L = mx.mx_layout_init(N, K, g, n8)
@@ -289,22 +293,22 @@ def main():
     Xs = [Xh.to(dev) for _ in range(R)]
     blobs = [blob0] + [blob0.clone() for _ in range(R - 1)]
     Aqs = [torch.empty((M, K), dtype=torch.int8, device=dev) for _ in range(R)]
-    sas = [torch.empty((M,), dtype=torch.float16, device=dev) for _ in range(R)]
+    sas = [torch.empty((M, K // ag) if ag else (M,), dtype=torch.float16, device=dev) for _ in range(R)]
     Ys = [torch.empty((M, N), dtype=torch.float16, device=dev) for _ in range(R)]
-    ws_bytes = mx.mx_linear_workspace_size(L, M, torch.float16, path=a.path)
+    ws_bytes = mx.mx_linear_workspace_size(L, M, torch.float16, path=a.path, act_group=ag)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
     fused = ws_bytes == 0                      # one kernel quantizes X and multiplies
     path_used = mx.mx_gemm_select_path(L, M, path=a.path)
 
     def step(i):
-        mx.mx_linear(L, blobs[i], Xs[i], Ys[i], workspace=ws, path=a.path)
+        mx.mx_linear(L, blobs[i], Xs[i], Ys[i], workspace=ws, path=a.path, act_group=ag)
 
     def gemm_only(i):
-        mx.mx_gemm(L, blobs[i], Aqs[i], sas[i], Ys[i], path=a.path)
+        mx.mx_gemm(L, blobs[i], Aqs[i], sas[i], Ys[i], path=a.path, act_group=ag)
 
     dominant = step if fused else gemm_only
     for i in range(R):                          # codes the GEMM-only timing reads
-        mx.mx_quant_act(Xs[i], Aqs[i], sas[i])
+        mx.mx_quant_act_grouped(Xs[i], Aqs[i], sas[i], ag)
 
     s = torch.cuda.Stream(dev)
     torch.cuda.synchronize()
@@ -415,7 +419,7 @@ def main():
     layer = MixedPrecisionLinear.from_blob(blob0)
     Xpin = Xh.pin_memory()
     Ypin = torch.empty((M, N), dtype=torch.float16).pin_memory()
-    runner = layer.graphed(Xpin, Ypin, path=a.path)        # H2D, mx_linear, D2H: one graph
+    runner = layer.graphed(Xpin, Ypin, path=a.path, act_group=ag)   # H2D, mx_linear, D2H: one graph
     Ke = max(20, min(K_steps, 5000))
     for _ in range(3):
         runner.replay()
@@ -443,7 +447,7 @@ def main():
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         import oracle
         can = oracle.pack(lay.W, lay.is8, g)
-        sec, desc, frac, done = time_oracle(lay, can, 1, min_seconds=10.0)
+        sec, desc, frac, done = time_oracle(lay, can, 1, min_seconds=10.0, act_group=ag)
         cpu = {"value": units_per_step * frac / sec, "unit": unit, "cores": 1, "kind": "oracle",
                "sample": f"{done} steps, each: quantize {M}x{K} activations + {desc}"}
 
@@ -453,6 +457,7 @@ def main():
         "warmup": a.warmup, "ms_per_step": ms / K_steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": a.workload, "M": M, "K": K, "N": N, "group": g, "frac8": a.frac8,
+                   "act_group": ag,
                    "n8": n8, "path": path_used, "fused_quantizer": fused,
                    "l2": f"inputs rotate over {R} copies ({R * per_step / 1e6:.0f} MB >= 4x the "
                          f"{l2 / 1e6:.0f} MB L2); no flush",

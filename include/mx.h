@@ -39,7 +39,8 @@
 extern "C" {
 #endif
 
-#define MX_ABI_VERSION 1
+#define MX_ABI_VERSION 2
+#define MX_BLOB_VERSION 1          /* packed-blob layout version, in the blob header */
 
 typedef enum mx_status {
     MX_OK = 0,
@@ -66,7 +67,7 @@ typedef enum mx_dtype { MX_F32 = 0, MX_F16 = 1 } mx_dtype;
  *
  * Packed blob (one device buffer, `total_bytes` long, every section 256-byte
  * aligned, offsets from the blob start):
- *   header   [256 B]   magic, version, N, K, group, n8 (see mx_layout_from_header)
+ *   header   [256 B]   magic, MX_BLOB_VERSION, N, K, group, n8 (see mx_layout_from_header)
  *   rowmap   int32 [(t8 + t4) * 128]   packed slot -> original row of W, -1 for
  *                      padding.  Slots 0 .. 128*t8-1 hold the 8-bit rows in
  *                      ascending original index; slots from 128*t8 on hold the
@@ -111,6 +112,11 @@ typedef struct mx_gemm_opts {
                                   and returns */
     int32_t test_stall;        /* testing only: the tensor-core loader issues no
                                   copies, so the waits run out (needs status) */
+    int32_t act_group;         /* activation scales: 0 = one per token, s_a [M];
+                                  g (must equal the weight group) = one per token and
+                                  group of g columns, s_a [M][K/g] (MixLLM section
+                                  3.1.2: group-wise activations), as written by
+                                  mx_quant_act_grouped */
 } mx_gemm_opts;
 
 /* ABI version of the loaded library (MX_ABI_VERSION). */
@@ -169,6 +175,20 @@ mx_status mx_pack_weights(const mx_layout* L, const void* W, mx_dtype wdtype, in
  */
 mx_status mx_quant_act(const void* X, mx_dtype xdtype, int M, int K, int64_t ldx,
                        int8_t* Aq, uint16_t* s_a, void* stream);
+
+/*
+ * mx_quant_act_grouped -- group-wise 8-bit symmetric activation quantization
+ * (MixLLM section 3.1.2: activations quantized group-wise, group 128 as the
+ * weights).  act_group = 0 is mx_quant_act.  Otherwise, with G = K / act_group:
+ *   s_a  device fp16 bits [M][G]: s_a[m,g] = fp16(max |X[m, g*act_group ..
+ *        (g+1)*act_group)| / 127), 0 -> 1
+ *   Aq[m,k] = clamp(round_half_even(X[m,k] / s_a[m, k / act_group]), -127, 127)
+ * act_group must be 0, 64 or 128 and divide K.  Other arguments and errors as
+ * mx_quant_act.  A GEMM reads these scales when its options carry the same
+ * act_group (which must equal the layer's weight group).
+ */
+mx_status mx_quant_act_grouped(const void* X, mx_dtype xdtype, int M, int K, int64_t ldx, int act_group,
+                               int8_t* Aq, uint16_t* s_a, void* stream);
 
 /*
  * mx_gemm_workspace_size -- host only.  Bytes of device workspace mx_gemm

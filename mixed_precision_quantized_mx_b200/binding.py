@@ -26,7 +26,8 @@ PATH_AUTO, PATH_SPLITK, PATH_TENSOR, PATH_ROWS = 0, 1, 2, 3
 
 EXPORTED = ("mx_version", "mx_last_error", "mx_layout_init", "mx_layout_from_header",
             "mx_pack_weights", "mx_quant_act", "mx_gemm_workspace_size", "mx_gemm_select_path",
-            "mx_gemm", "mx_linear_workspace_size", "mx_linear", "mx_linear_noalloc")
+            "mx_gemm", "mx_linear_workspace_size", "mx_linear", "mx_linear_noalloc",
+            "mx_quant_act_grouped")
 
 
 class MXError(RuntimeError):
@@ -48,7 +49,8 @@ class GemmOpts(ctypes.Structure):
     """mirror of mx_gemm_opts"""
     _fields_ = [("path", ctypes.c_int32), ("split", ctypes.c_int32),
                 ("debug_partials", ctypes.c_void_p), ("status", ctypes.c_void_p),
-                ("wait_timeout_us", ctypes.c_int32), ("test_stall", ctypes.c_int32)]
+                ("wait_timeout_us", ctypes.c_int32), ("test_stall", ctypes.c_int32),
+                ("act_group", ctypes.c_int32)]
 
 
 _lib = None
@@ -70,6 +72,7 @@ def lib() -> ctypes.CDLL:
     L.mx_layout_from_header.argtypes = [P, Z, ctypes.POINTER(Layout)]
     L.mx_pack_weights.argtypes = [ctypes.POINTER(Layout), P, I, I64, P, P, P, P]
     L.mx_quant_act.argtypes = [P, I, I, I, I64, P, P, P]
+    L.mx_quant_act_grouped.argtypes = [P, I, I, I, I64, I, P, P, P]
     L.mx_gemm_workspace_size.argtypes = [ctypes.POINTER(Layout), I, ctypes.POINTER(GemmOpts),
                                          ctypes.POINTER(Z)]
     L.mx_gemm_select_path.argtypes = [ctypes.POINTER(Layout), I, ctypes.POINTER(GemmOpts)]
@@ -83,7 +86,7 @@ def lib() -> ctypes.CDLL:
     L.mx_linear_noalloc.argtypes = [ctypes.POINTER(Layout), P, P, I, I, I64, P, I64,
                                     ctypes.POINTER(GemmOpts), P]
     for n in ("mx_layout_init", "mx_layout_from_header", "mx_pack_weights", "mx_quant_act",
-              "mx_gemm_workspace_size", "mx_gemm", "mx_linear_workspace_size", "mx_linear",
+              "mx_quant_act_grouped", "mx_gemm_workspace_size", "mx_gemm", "mx_linear_workspace_size", "mx_linear",
               "mx_linear_noalloc"):
         getattr(L, n).restype = I
     _lib = L
@@ -116,8 +119,8 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _opts(path=0, split=0, debug_partials=None, status=None, wait_timeout_us=0,
-          test_stall=0) -> GemmOpts:
-    return GemmOpts(path, split, _ptr(debug_partials), _ptr(status), wait_timeout_us, test_stall)
+          test_stall=0, act_group=0) -> GemmOpts:
+    return GemmOpts(path, split, _ptr(debug_partials), _ptr(status), wait_timeout_us, test_stall, act_group)
 
 
 # ------------------------------------------------------------------ entry points
@@ -155,6 +158,15 @@ def mx_quant_act(X: torch.Tensor, Aq: torch.Tensor, s_a: torch.Tensor, stream=No
                               _stream(stream)), "mx_quant_act")
 
 
+def mx_quant_act_grouped(X: torch.Tensor, Aq: torch.Tensor, s_a: torch.Tensor, act_group: int,
+                         stream=None) -> None:
+    """s_a: fp16 [M] (act_group 0) or [M, K / act_group]."""
+    assert X.dim() == 2 and X.stride(1) == 1
+    M, K = X.shape
+    _check(lib().mx_quant_act_grouped(_ptr(X), _dtype_code(X), M, K, X.stride(0), act_group, _ptr(Aq),
+                                      _ptr(s_a), _stream(stream)), "mx_quant_act_grouped")
+
+
 def mx_gemm_workspace_size(L: Layout, M: int, path: int = 0, split: int = 0) -> int:
     n = ctypes.c_size_t(0)
     o = _opts(path, split)
@@ -174,17 +186,18 @@ def mx_gemm_select_path(L: Layout, M: int, path: int = 0, split: int = 0) -> int
 def mx_gemm(L: Layout, blob: torch.Tensor, Aq: torch.Tensor, s_a: torch.Tensor, Y: torch.Tensor,
             workspace: torch.Tensor | None = None, path: int = 0, split: int = 0,
             debug_partials: torch.Tensor | None = None, status: torch.Tensor | None = None,
-            wait_timeout_us: int = 0, test_stall: int = 0, stream=None) -> None:
+            wait_timeout_us: int = 0, test_stall: int = 0, act_group: int = 0, stream=None) -> None:
     M = Aq.shape[0]
-    o = _opts(path, split, debug_partials, status, wait_timeout_us, test_stall)
+    o = _opts(path, split, debug_partials, status, wait_timeout_us, test_stall, act_group)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().mx_gemm(ctypes.byref(L), _ptr(blob), _ptr(Aq), _ptr(s_a), M, _ptr(Y), Y.stride(0),
                          _ptr(workspace), ws_bytes, ctypes.byref(o), _stream(stream)), "mx_gemm")
 
 
-def mx_linear_workspace_size(L: Layout, M: int, xdtype=torch.float16, path: int = 0, split: int = 0) -> int:
+def mx_linear_workspace_size(L: Layout, M: int, xdtype=torch.float16, path: int = 0, split: int = 0,
+                             act_group: int = 0) -> int:
     n = ctypes.c_size_t(0)
-    o = _opts(path, split)
+    o = _opts(path, split, act_group=act_group)
     code = MX_F16 if xdtype == torch.float16 else MX_F32
     _check(lib().mx_linear_workspace_size(ctypes.byref(L), M, code, ctypes.byref(o), ctypes.byref(n)),
            "mx_linear_workspace_size")
@@ -194,10 +207,10 @@ def mx_linear_workspace_size(L: Layout, M: int, xdtype=torch.float16, path: int 
 def mx_linear(L: Layout, blob: torch.Tensor, X: torch.Tensor, Y: torch.Tensor,
               workspace: torch.Tensor | None = None, path: int = 0, split: int = 0,
               debug_partials: torch.Tensor | None = None, status: torch.Tensor | None = None,
-              stream=None) -> None:
+              act_group: int = 0, stream=None) -> None:
     assert X.dim() == 2 and X.stride(1) == 1
     M = X.shape[0]
-    o = _opts(path, split, debug_partials, status)
+    o = _opts(path, split, debug_partials, status, act_group=act_group)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().mx_linear(ctypes.byref(L), _ptr(blob), _ptr(X), _dtype_code(X), M, X.stride(0),
                            _ptr(Y), Y.stride(0), _ptr(workspace), ws_bytes, ctypes.byref(o),

@@ -81,8 +81,9 @@ struct DecArgs {
     int kbu;          // k-blocks per CTA
     int kps;          // k-blocks per slot
     int ns;           // ring slots
-    int off_act, off_sa64, off_part, off_raw;   // dynamic shared-memory layout
+    int off_act, off_sa64, off_part, off_raw, off_sag;   // dynamic shared-memory layout
     int xfull;        // in-kernel quantization stages whole X rows (no exchange)
+    int ag;           // 0: one activation scale per token; g: one per token and group
     int32_t* debug;
     int32_t* status;  // MX_ERR_TIMEOUT if a bounded wait ran out (never expected)
 };
@@ -296,6 +297,9 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap codes8_map, const __grid_
     __shared__ float sa_loc[MT];                                  // token scales quantized in-kernel
     bool cluster_waited = false;                                  // (the wait matching the arrive)
     griddep_wait();
+    // group-wise activation scales of this CTA's groups: [MT][kbu * gpk]
+    float* sag = reinterpret_cast<float*>(smem + a.off_sag);
+    const int ngl = a.kbu * gpk;
     if constexpr (std::is_void_v<XT>) {
         // ---- stage Aq[m0 .. m0+MT)[kb0*128 .. kb1*128) (zero rows beyond M)
         const int chunks = nkb * (kKBlock / 16);
@@ -305,6 +309,61 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap codes8_map, const __grid_
             if (m0 + j < a.M)
                 v = __ldg(reinterpret_cast<const uint4*>(a.Aq + int64_t(m0 + j) * g.K + kb0 * kKBlock) + c);
             *reinterpret_cast<uint4*>(act + j * rowb + c * 16) = v;
+        }
+        if (a.ag) {
+            for (int i = tid; i < MT * nkb * gpk; i += kConsumers) {
+                const int j = i / (nkb * gpk), li = i % (nkb * gpk);
+                sag[j * ngl + li] =
+                    m0 + j < a.M ? __half2float(a.s_a[int64_t(m0 + j) * g.G + kb0 * gpk + li]) : 0.0f;
+            }
+        }
+    } else if (a.ag) {
+        // ---- group-wise scales: this CTA's k-blocks hold whole groups, so it stages its
+        // slice, takes each group's absmax over its lane segment and quantizes it; no
+        // exchange between the CTAs of the cluster
+        const XT* X = static_cast<const XT*>(a.X);
+        const int xrow = a.kbu * kKBlock;
+        XT* xs = reinterpret_cast<XT*>(smem + a.off_raw);
+        const int chunks = nkb * kKBlock * int(sizeof(XT)) / 16;
+        for (int i = tid; i < MT * chunks; i += kConsumers) {
+            const int j = i / chunks, c = i % chunks;
+            if (m0 + j < a.M)
+                cp_async16(reinterpret_cast<uint8_t*>(xs + size_t(j) * xrow) + size_t(c) * 16,
+                           reinterpret_cast<const uint8_t*>(X + int64_t(m0 + j) * a.ldx + kb0 * kKBlock) +
+                               size_t(c) * 16);
+        }
+        cp_async_wait_all();
+        consumer_sync();
+        const int cpg = a.ag / 8, n8 = nkb * (kKBlock / 8);
+#pragma unroll
+        for (int j = 0; j < MT; ++j) {
+            const bool row = m0 + j < a.M;
+            for (int c0 = 0; c0 < n8; c0 += kConsumers) {           // same trip count in every lane
+                const int c = c0 + tid;
+                const bool live = row && c < n8;
+                float v[8];
+                if (live) {
+                    smem4(xs + size_t(j) * xrow + c * 8, *reinterpret_cast<float(*)[4]>(v));
+                    smem4(xs + size_t(j) * xrow + c * 8 + 4, *reinterpret_cast<float(*)[4]>(v + 4));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+                }
+                float am = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(v[e]));
+                for (int o = cpg / 2; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+                const float sg = __half2float(act_scale(am)), rg = __frcp_rn(sg);
+                if (c < n8) {
+                    uint2 o = make_uint2(0, 0);
+                    if (live) {
+                        o.x = quant4(v, sg, rg);
+                        o.y = quant4(v + 4, sg, rg);
+                    }
+                    *reinterpret_cast<uint2*>(act + j * rowb + c * 8) = o;
+                    if (c % cpg == 0) sag[j * ngl + c / cpg] = live ? sg : 0.0f;
+                }
+            }
         }
     } else {
         // ---- in-kernel quantization of X.  Short rows (xfull): every CTA stages the
@@ -488,7 +547,11 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap codes8_map, const __grid_
             }
         }
 #pragma unroll
-        for (int j = 0; j < MT; ++j) out[j] = __fmaf_rn(i2f_biased(acc[j]), sw, out[j]);
+        for (int j = 0; j < MT; ++j) {
+            // group-wise activations: the token's scale of this group joins the weight's
+            const float s = a.ag ? __fmul_rn(sw, sag[j * ngl + kl * gpk + gl]) : sw;
+            out[j] = __fmaf_rn(i2f_biased(acc[j]), s, out[j]);
+        }
         if (DEBUG && orig >= 0) {                       // padding rows have no column
             const bool writer = eight ? (g.group == 128 ? sub == 0 : (sub & 1) == 0)
                                       : (g.group == 128 ? sub == 0 : true);
@@ -554,7 +617,8 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap codes8_map, const __grid_
         for (int q = 0; q < a.S; ++q) sum = __fadd_rn(sum, part[(size_t(q) * MT + j) * 128 + rr]);
         const int o = y_col;                      // rr == tid % rows
         float sa;
-        if constexpr (std::is_void_v<XT>) sa = __half2float(a.s_a[m0 + j]);
+        if (a.ag) sa = 1.0f;                  // group-wise scales were applied per group
+        else if constexpr (std::is_void_v<XT>) sa = __half2float(a.s_a[m0 + j]);
         else sa = sa_loc[j];
         if (o >= 0) a.Y[int64_t(m0 + j) * a.ldy + o] = __float2half_rn(__fmul_rn(sum, sa));
     }
@@ -657,6 +721,7 @@ DecArgs base_args(const mx_layout& L, const void* blob, int M, uint16_t* Y, int6
     a.off_part = p.off_part;
     a.off_raw = p.off_raw;
     a.xfull = p.xfull;
+    a.off_sag = p.off_sag;
     a.debug = debug_partials;
     a.status = status;
     return a;
@@ -717,17 +782,19 @@ DecodePlan plan_decode(const mx_layout& L, int M, int split_hint, int x_bytes) {
     p.off_sa64 = int(p.off_act + act);
     p.off_part = int(p.off_sa64 + sa64);
     p.off_raw = int(p.off_part + part);
-    p.smem = size_t(p.off_raw) + raw + 128;        // + room to align the base
+    p.off_sag = int(p.off_raw + raw);
+    p.smem = size_t(p.off_sag) + align16(size_t(p.mt) * p.kbu * 2 * 4) + 128;   // + room to align the base
     p.ok = S >= s_min && size_t(p.kbu) * p.mt * kKBlock <= size_t(kMaxActSmem) && p.smem <= size_t(kMaxSmem);
     return p;
 }
 
 cudaError_t launch_gemm_decode(const mx_layout& L, const void* blob, const int8_t* Aq,
                                const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy,
-                               const DecodePlan& plan, int32_t* debug_partials, int32_t* status,
+                               const DecodePlan& plan, int ag, int32_t* debug_partials, int32_t* status,
                                cudaStream_t s) {
     if (M == 0) return cudaSuccess;
     DecArgs a = base_args(L, blob, M, Y, ldy, plan, debug_partials, status);
+    a.ag = ag;
     a.Aq = Aq;
     a.s_a = reinterpret_cast<const __half*>(s_a);
     CUtensorMap map;
@@ -745,7 +812,7 @@ bool decode_can_fuse(const mx_layout& L, int M, mx_dtype xdt) {
 
 cudaError_t launch_gemm_decode_fused(const mx_layout& L, const void* blob, const void* X, mx_dtype xdt,
                                      int64_t ldx, int M, uint16_t* Y, int64_t ldy, const DecodePlan& plan,
-                                     int32_t* debug_partials, int32_t* status, cudaStream_t s) {
+                                     int ag, int32_t* debug_partials, int32_t* status, cudaStream_t s) {
     if (M == 0) return cudaSuccess;
     if (plan.mt > kMaxFusedTokens || !plan.ok) return cudaErrorInvalidValue;
     // the plan must have room for the raw slice of this input type
@@ -753,6 +820,7 @@ cudaError_t launch_gemm_decode_fused(const mx_layout& L, const void* blob, const
     if (size_t(plan.smem) < size_t(plan.off_raw) + 128 + size_t(plan.mt) * cols * (xdt == MX_F16 ? 2 : 4))
         return cudaErrorInvalidValue;
     DecArgs a = base_args(L, blob, M, Y, ldy, plan, debug_partials, status);
+    a.ag = ag;
     a.X = X;
     a.ldx = ldx;
     CUtensorMap m;

@@ -53,7 +53,8 @@ struct RowsArgs {
     int64_t ldy;
     int M;
     int n8u;                // 8-bit units (t8 * 16); 4-bit units follow
-    int off_sc, off_z, off_act, off_sa64, off_raw, off_red;   // dynamic shared memory
+    int off_sc, off_z, off_act, off_sa64, off_raw, off_red, off_sag;   // dynamic shared memory
+    int ag;                 // 0: one activation scale per token; g: one per token and group
     int32_t* debug;
     int32_t* status;
 };
@@ -160,6 +161,7 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
 
     // ---- activations (these wait for the previous kernel)
     int8_t* act = reinterpret_cast<int8_t*>(smem + a.off_act);    // [MT][K]
+    float* sag = reinterpret_cast<float*>(smem + a.off_sag);        // [MT][G] when a.ag
     griddep_wait();
     if constexpr (std::is_void_v<XT>) {
         const int chunks = K / 16;
@@ -168,7 +170,64 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
             if (m0 + j < a.M) cp_async16(act + size_t(j) * K + c * 16, a.Aq + int64_t(m0 + j) * K + c * 16);
             else *reinterpret_cast<uint4*>(act + size_t(j) * K + c * 16) = make_uint4(0, 0, 0, 0);
         }
+        if (a.ag) {                       // group-wise activation scales s_a[m][g]
+            for (int i = tid; i < MT * g.G; i += kThreads) {
+                const int j = i / g.G, gi = i % g.G;
+                sag[i] = m0 + j < a.M ? __half2float(a.s_a[int64_t(m0 + j) * g.G + gi]) : 0.0f;
+            }
+        }
         cp_async_wait_all();
+        __syncthreads();
+    } else if (a.ag) {
+        // group-wise scales, in one pass: a group's 8-element chunks sit in consecutive
+        // lanes, so its absmax is a shuffle reduction in that lane segment, and every
+        // lane then quantizes the values it holds (the grouped quantizer's operations)
+        const XT* X = static_cast<const XT*>(a.X);
+        const int cpg = a.ag / 8;
+#pragma unroll
+        for (int j = 0; j < MT; ++j) {
+            const bool row = m0 + j < a.M;
+            for (int c0 = 0; c0 < K / 8; c0 += kThreads) {          // same trip count in every lane
+                const int c = c0 + tid;
+                const bool live = row && c < K / 8;
+                float v[8];
+                if (live) {
+                    const XT* xp = X + int64_t(m0 + j) * a.ldx + c * 8;
+                    if constexpr (std::is_same_v<XT, __half>) {
+                        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(xp));
+                        const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __half22float2(h2[e]);
+                            v[2 * e] = f.x;
+                            v[2 * e + 1] = f.y;
+                        }
+                    } else {
+                        const float4 f0 = __ldg(reinterpret_cast<const float4*>(xp));
+                        const float4 f1 = __ldg(reinterpret_cast<const float4*>(xp) + 1);
+                        v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
+                        v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+                }
+                float am = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(v[e]));
+                for (int o = cpg / 2; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+                const float sg = __half2float(act_scale(am)), rg = __frcp_rn(sg);
+                if (c < K / 8) {
+                    uint2 o = make_uint2(0, 0);
+                    if (live) {
+                        o.x = quant4(v, sg, rg);
+                        o.y = quant4(v + 4, sg, rg);
+                    }
+                    *reinterpret_cast<uint2*>(act + size_t(j) * K + c * 8) = o;
+                    if (c % cpg == 0) sag[j * g.G + c / cpg] = live ? sg : 0.0f;
+                }
+            }
+        }
         __syncthreads();
     } else {
         // whole rows: absmax, the fp16 scale, then the codes, with the quantizer's operations
@@ -342,7 +401,11 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
             }
             const float sw = __half2float(SC[gi * R + r]);
 #pragma unroll
-            for (int j = 0; j < MT; ++j) out[j] = __fmaf_rn(i2f_biased(acc[j]), sw, out[j]);
+            for (int j = 0; j < MT; ++j) {
+                // group-wise activations: the token's scale of this group joins the weight's
+                const float s = a.ag ? __fmul_rn(sw, sag[j * g.G + gi]) : sw;
+                out[j] = __fmaf_rn(i2f_biased(acc[j]), s, out[j]);
+            }
             if (DEBUG && orig >= 0) {                                   // padding rows have no column
 #pragma unroll
                 for (int j = 0; j < MT; ++j)
@@ -361,9 +424,11 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
         if (m0 + j < a.M && orig >= 0) {
             float sum = 0.0f;
             for (int q = 0; q < P; ++q) sum = __fadd_rn(sum, red[(q * R + r) * MT + j]);
-            float sa;
-            if constexpr (std::is_void_v<XT>) sa = __half2float(a.s_a[m0 + j]);
-            else sa = sa_loc[j];
+            float sa = 1.0f;                        // group-wise scales were applied per group
+            if (!a.ag) {
+                if constexpr (std::is_void_v<XT>) sa = __half2float(a.s_a[m0 + j]);
+                else sa = sa_loc[j];
+            }
             a.Y[int64_t(m0 + j) * a.ldy + orig] = __float2half_rn(__fmul_rn(sum, sa));
         }
     }
@@ -458,6 +523,8 @@ RowsPlan plan_rows(const mx_layout& L, int M, int x_bytes) {
     off += align16(size_t(p.mt) * L.K * x_bytes);
     p.off_red = int(off);
     off += size_t(kThreads) * p.mt * 4;
+    p.off_sag = int(off);
+    off += align16(size_t(p.mt) * L.G * 4);
     p.smem = off + 1024;                                // + room to align the base
     // one wave with room left for the next launch's CTAs; the shared-memory test
     // assumes fp32 rows whatever x_bytes is, so Aq, fp16 and fp32 inputs of one
@@ -469,7 +536,8 @@ RowsPlan plan_rows(const mx_layout& L, int M, int x_bytes) {
 
 cudaError_t launch_gemm_rows(const mx_layout& L, const void* blob, const int8_t* Aq, const uint16_t* s_a,
                              const void* X, mx_dtype xdt, int64_t ldx, int M, uint16_t* Y, int64_t ldy,
-                             const RowsPlan& p, int32_t* debug_partials, int32_t* status, cudaStream_t s) {
+                             const RowsPlan& p, int ag, int32_t* debug_partials, int32_t* status,
+                             cudaStream_t s) {
     if (M == 0) return cudaSuccess;
     if (!p.ok) return cudaErrorInvalidValue;
     // a raw input needs the plan's room for its rows
@@ -502,6 +570,8 @@ cudaError_t launch_gemm_rows(const mx_layout& L, const void* blob, const int8_t*
     a.off_sa64 = p.off_sa64;
     a.off_raw = p.off_raw;
     a.off_red = p.off_red;
+    a.off_sag = p.off_sag;
+    a.ag = ag;
     a.debug = debug_partials;
     a.status = status;
     if (X == nullptr) return launch_dbg<void>(m4, m8, a, p, s);

@@ -65,6 +65,7 @@ constexpr uint32_t kTmemCols = kAccBufs * BN;   // all 512 columns
 constexpr int kWidenBarrier = 1;                // named barrier of the widening warps
 constexpr int kMmaIssuers = 2;                  // MMA-issuing threads, alternating groups
 constexpr int kScaleRing = 4;                   // group scales in flight per epilogue thread
+constexpr int kSatGroups = 8;                   // group-wise activation scales staged per refill
 
 struct __align__(1024) Smem {
     uint8_t A[kStages][kKbPerStage * kABytes];  // raw uint4 codes land at A + kRawBase
@@ -75,13 +76,16 @@ struct __align__(1024) Smem {
     uint64_t acc_full[kAccBufs];  // MMA -> epilogue: group accumulator complete
     uint64_t acc_empty[kAccBufs]; // epilogue -> MMA: accumulator drained and re-armed
     uint64_t mma_done[kMmaIssuers];
+    // group-wise activation scales: each epilogue warp's 64 tokens for 8 groups
+    __align__(16) __half sat[kEpiWarps][kSatGroups][BN / 2];
     uint32_t tmem_base;
     int abort;
 };
 
 struct TcArgs {
     Geom g;
-    const __half* s_a;
+    const __half* s_a;   // [M], or [M][G] with group-wise activation scales (ag != 0)
+    int ag;
     __half* Y;
     int64_t ldy;
     int M;
@@ -109,7 +113,8 @@ __device__ __forceinline__ void drain_stages(Smem& S, int issued, uint64_t timeo
     }
 }
 
-template <bool DEBUG>
+// AG: group-wise activation scales (s_a [M][G]) instead of one per token
+template <bool DEBUG, bool AG>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -345,6 +350,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     const bool ok = mbar_wait_bounded(&S.acc_full[b], u & 1, abort, a.status, a.timeout_ns);
                     if (!__all_sync(0xffffffffu, ok)) goto epi_done;
                     tc_fence_after();
+                    // group-wise activations: refill this warp's window of token scales
+                    // every kSatGroups groups (warp-private, so only the warp synchronises)
+                    __half (*sat)[BN / 2] = S.sat[warp - 8];
+                    if (AG && gi % kSatGroups == 0) {
+                        __syncwarp();
+                        for (int i = lane; i < kSatGroups * (BN / 2); i += 32) {
+                            const int w = i / (BN / 2), t = i % (BN / 2), m = tt * BN + cb + t;
+                            sat[w][t] = gi + w < g.G && m < a.M ? a.s_a[int64_t(m) * g.G + gi + w]
+                                                                : __float2half_rn(0.0f);
+                        }
+                        __syncwarp();
+                    }
                     // drain the group's 64 columns in eight 8-column chunks, loading chunk
                     // h+1 while chunk h is converted
                     const uint32_t col0 = lane_addr + b * BN + cb;
@@ -358,12 +375,27 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                         if (h < 7) tmem_ld_x8(col0 + (h + 1) * 8, vn);
                         // acc += (float(bias + P) - bias) * s_w: the fast int-to-float adds the
                         // bias as an integer, two columns per float instruction
+                        if constexpr (AG) {
+                            // group-wise activations: column (token) m also takes s_a[m][gi]
+                            const uint4 sv = *reinterpret_cast<const uint4*>(&sat[gi % kSatGroups][h * 8]);
+                            const __half2* sh = reinterpret_cast<const __half2*>(&sv);
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const float2 f = add2(make_float2(__uint_as_float(v[2 * c] + kI2FBiasBits),
-                                                              __uint_as_float(v[2 * c + 1] + kI2FBiasBits)),
-                                                  nbias);
-                            acc[h * 4 + c] = fma2(f, s2, acc[h * 4 + c]);
+                            for (int c = 0; c < 4; ++c) {
+                                const float2 sa2 = __half22float2(sh[c]);
+                                const float2 f = add2(make_float2(__uint_as_float(v[2 * c] + kI2FBiasBits),
+                                                                  __uint_as_float(v[2 * c + 1] + kI2FBiasBits)),
+                                                      nbias);
+                                acc[h * 4 + c] = fma2(f, make_float2(__fmul_rn(sw, sa2.x), __fmul_rn(sw, sa2.y)),
+                                                      acc[h * 4 + c]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const float2 f = add2(make_float2(__uint_as_float(v[2 * c] + kI2FBiasBits),
+                                                                  __uint_as_float(v[2 * c + 1] + kI2FBiasBits)),
+                                                      nbias);
+                                acc[h * 4 + c] = fma2(f, s2, acc[h * 4 + c]);
+                            }
                         }
                         if (DEBUG && orig >= 0) {
 #pragma unroll
@@ -387,9 +419,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int m = tt * BN + cb + 2 * c + e;
-                        if (m < a.M)
-                            a.Y[int64_t(m) * a.ldy + orig] = __float2half_rn(
-                                __fmul_rn(e ? acc[c].y : acc[c].x, __half2float(a.s_a[m])));
+                        if (m < a.M) {
+                            const float v = e ? acc[c].y : acc[c].x;
+                            // group-wise scales were applied per group
+                            a.Y[int64_t(m) * a.ldy + orig] =
+                                __float2half_rn(AG ? v : __fmul_rn(v, __half2float(a.s_a[m])));
+                        }
                     }
                 }
             }
@@ -427,7 +462,7 @@ EncodeTiledFn encode_fn(cudaError_t* err) {
 size_t tc_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* Aq,
-                           const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy,
+                           const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy, int ag,
                            int32_t* debug_partials, int32_t* status, uint64_t timeout_ns,
                            int stall_test, cudaStream_t s) {
     if (M == 0) return cudaSuccess;
@@ -451,12 +486,11 @@ cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* A
     static int sms[64] = {};
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (sms[dev] == 0) {
-        if ((e = cudaFuncSetAttribute(gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(tc_smem_bytes()))) != cudaSuccess)
-            return e;
-        if ((e = cudaFuncSetAttribute(gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(tc_smem_bytes()))) != cudaSuccess)
-            return e;
+        for (auto k : {gemm_tc_kernel<false, false>, gemm_tc_kernel<true, false>, gemm_tc_kernel<false, true>,
+                       gemm_tc_kernel<true, true>})
+            if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(tc_smem_bytes()))) !=
+                cudaSuccess)
+                return e;
         int n = 0;
         if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
         sms[dev] = n;
@@ -464,6 +498,7 @@ cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* A
     TcArgs a{};
     a.g = make_geom(L, blob);
     a.s_a = reinterpret_cast<const __half*>(s_a);
+    a.ag = ag;
     a.Y = reinterpret_cast<__half*>(Y);
     a.ldy = ldy;
     a.M = M;
@@ -474,10 +509,9 @@ cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* A
     a.timeout_ns = timeout_ns;
     a.stall_test = stall_test;
     const int grid = a.n_tiles < sms[dev] ? a.n_tiles : sms[dev];
-    if (debug_partials)
-        gemm_tc_kernel<true><<<grid, kThreads, tc_smem_bytes(), s>>>(map, a);
-    else
-        gemm_tc_kernel<false><<<grid, kThreads, tc_smem_bytes(), s>>>(map, a);
+    auto k = debug_partials ? (ag ? gemm_tc_kernel<true, true> : gemm_tc_kernel<true, false>)
+                            : (ag ? gemm_tc_kernel<false, true> : gemm_tc_kernel<false, false>);
+    k<<<grid, kThreads, tc_smem_bytes(), s>>>(map, a);
     return cudaGetLastError();
 }
 

@@ -57,6 +57,21 @@ mx_status check_layout(const mx_layout* L) {
     return MX_OK;
 }
 
+// act_group: 0 (one activation scale per token) or the layer's weight group
+mx_status check_act_group(const mx_layout* L, const mx_gemm_opts* opts) {
+    const int ag = opts ? opts->act_group : 0;
+    if (ag != 0 && ag != L->group)
+        return fail(MX_ERR_UNSUPPORTED, "act_group=%d: 0 or the weight group %d", ag, L->group);
+    return MX_OK;
+}
+
+int act_group_of(const mx_gemm_opts* opts) { return opts ? opts->act_group : 0; }
+
+// activation scales per token: 1, or one per group
+size_t scales_per_token(const mx_layout* L, const mx_gemm_opts* opts) {
+    return act_group_of(opts) ? size_t(L->G) : 1;
+}
+
 }  // namespace
 
 namespace mx {
@@ -120,7 +135,7 @@ mx_status mx_layout_from_header(const void* host_header, size_t bytes, mx_layout
     uint32_t h[6];
     memcpy(h, host_header, sizeof h);
     if (h[0] != MX_BLOB_MAGIC) return fail(MX_ERR_BAD_BLOB, "bad magic 0x%08x", h[0]);
-    if (h[1] != MX_ABI_VERSION) return fail(MX_ERR_BAD_BLOB, "blob version %u != %d", h[1], MX_ABI_VERSION);
+    if (h[1] != MX_BLOB_VERSION) return fail(MX_ERR_BAD_BLOB, "blob version %u != %d", h[1], MX_BLOB_VERSION);
     mx_status st = mx_layout_init(int(h[2]), int(h[3]), int(h[4]), int(h[5]), out);
     if (st != MX_OK) return fail(MX_ERR_BAD_BLOB, "header geometry invalid: %s", g_err.c_str());
     return MX_OK;
@@ -159,6 +174,28 @@ mx_status mx_quant_act(const void* X, mx_dtype xdtype, int M, int K, int64_t ldx
         return fail(MX_ERR_ALIGNMENT, "X, Aq and every X row must be 16-byte aligned");
     cudaError_t e = mx::launch_quant_act(X, xdtype, M, K, ldx, Aq, s_a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "quant_act launch");
+    return MX_OK;
+}
+
+mx_status mx_quant_act_grouped(const void* X, mx_dtype xdtype, int M, int K, int64_t ldx, int act_group,
+                               int8_t* Aq, uint16_t* s_a, void* stream) {
+    if (act_group == 0) return mx_quant_act(X, xdtype, M, K, ldx, Aq, s_a, stream);
+    if (act_group != 64 && act_group != 128) return fail(MX_ERR_UNSUPPORTED, "act_group=%d (0, 64 or 128)", act_group);
+    if (xdtype != MX_F32 && xdtype != MX_F16) return fail(MX_ERR_INVALID_ARG, "bad xdtype %d", int(xdtype));
+    if (M < 0 || K < 1) return fail(MX_ERR_INVALID_ARG, "M=%d K=%d", M, K);
+    if (K % act_group != 0) return fail(MX_ERR_UNSUPPORTED, "K=%d is not a multiple of act_group=%d", K, act_group);
+    if (ldx < K) return fail(MX_ERR_INVALID_ARG, "ldx=%lld < K=%d", (long long)ldx, K);
+    if (M == 0) return MX_OK;
+    mx_status st;
+    if ((st = check_device_ptr(X, "X")) != MX_OK) return st;
+    if ((st = check_device_ptr(Aq, "Aq")) != MX_OK) return st;
+    if ((st = check_device_ptr(s_a, "s_a")) != MX_OK) return st;
+    const int esz = xdtype == MX_F16 ? 2 : 4;
+    if (!aligned16(X) || (ldx * esz) % 16 != 0 || !aligned16(Aq))
+        return fail(MX_ERR_ALIGNMENT, "X, Aq and every X row must be 16-byte aligned");
+    cudaError_t e = mx::launch_quant_act_grouped(X, xdtype, M, K, ldx, act_group, Aq, s_a,
+                                                 static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "grouped quant_act launch");
     return MX_OK;
 }
 
@@ -201,6 +238,7 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
     if (ldy < L->N) return fail(MX_ERR_INVALID_ARG, "ldy=%lld < N=%d", (long long)ldy, L->N);
     if (M == 0) return MX_OK;
     if (M > 65535) return fail(MX_ERR_UNSUPPORTED, "M=%d above 65535", M);
+    if ((st = check_act_group(L, opts)) != MX_OK) return st;
     if ((st = check_device_ptr(blob, "blob")) != MX_OK) return st;
     if ((st = check_device_ptr(Aq, "Aq")) != MX_OK) return st;
     if ((st = check_device_ptr(s_a, "s_a")) != MX_OK) return st;
@@ -209,12 +247,13 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
     if (opts && opts->debug_partials && (st = check_device_ptr(opts->debug_partials, "debug_partials")) != MX_OK)
         return st;
     if (opts && opts->status && (st = check_device_ptr(opts->status, "status")) != MX_OK) return st;
+    const int ag = act_group_of(opts);
     const int path = choose_path(L, M, opts);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (path == 3) {
         const mx::RowsPlan rp = mx::plan_rows(*L, M, 0);
         if (!rp.ok) return fail(MX_ERR_UNSUPPORTED, "M=%d K=%d: beyond the row path (M <= 4, K <= 4096, one wave)", M, L->K);
-        cudaError_t e = mx::launch_gemm_rows(*L, blob, Aq, s_a, nullptr, MX_F16, 0, M, Y, ldy, rp,
+        cudaError_t e = mx::launch_gemm_rows(*L, blob, Aq, s_a, nullptr, MX_F16, 0, M, Y, ldy, rp, ag,
                                              opts ? opts->debug_partials : nullptr, opts ? opts->status : nullptr, s);
         if (e != cudaSuccess) return cuda_fail(e, "row decode GEMM launch");
         return MX_OK;
@@ -224,7 +263,7 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
         mx::DecodePlan plan = mx::plan_decode(*L, M, opts ? opts->split : 0);
         if (!plan.ok)
             return fail(MX_ERR_UNSUPPORTED, "M=%d K=%d: activation slice too large for the decode path", M, L->K);
-        cudaError_t e = mx::launch_gemm_decode(*L, blob, Aq, s_a, M, Y, ldy, plan,
+        cudaError_t e = mx::launch_gemm_decode(*L, blob, Aq, s_a, M, Y, ldy, plan, ag,
                                                opts ? opts->debug_partials : nullptr,
                                                opts ? opts->status : nullptr, s);
         if (e != cudaSuccess) return cuda_fail(e, "decode GEMM launch");
@@ -236,7 +275,7 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
         if (opts && opts->wait_timeout_us < 0) return fail(MX_ERR_INVALID_ARG, "wait_timeout_us < 0");
         const uint64_t timeout_ns =
             (opts && opts->wait_timeout_us > 0) ? uint64_t(opts->wait_timeout_us) * 1000u : 2000000000ull;
-        cudaError_t e = mx::launch_gemm_tc(*L, blob, Aq, s_a, M, Y, ldy,
+        cudaError_t e = mx::launch_gemm_tc(*L, blob, Aq, s_a, M, Y, ldy, ag,
                                            opts ? opts->debug_partials : nullptr,
                                            opts ? opts->status : nullptr, timeout_ns,
                                            opts ? opts->test_stall : 0, s);
@@ -269,8 +308,9 @@ mx_status mx_linear_workspace_size(const mx_layout* L, int M, mx_dtype xdtype, c
     if (bytes == nullptr) return fail(MX_ERR_INVALID_ARG, "bytes is NULL");
     if (M < 0) return fail(MX_ERR_INVALID_ARG, "M=%d", M);
     if (xdtype != MX_F32 && xdtype != MX_F16) return fail(MX_ERR_INVALID_ARG, "bad xdtype %d", int(xdtype));
+    if ((st = check_act_group(L, opts)) != MX_OK) return st;
     *bytes = (M == 0 || linear_fused(L, M, xdtype, opts)) ? 0
-             : align16(size_t(M) * L->K) + align16(size_t(2) * M);
+             : align16(size_t(M) * L->K) + align16(size_t(2) * M * scales_per_token(L, opts));
     return MX_OK;
 }
 
@@ -286,8 +326,10 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
     if (M == 0) return MX_OK;
     if (M > 65535) return fail(MX_ERR_UNSUPPORTED, "M=%d above 65535", M);
     const int esz = xdtype == MX_F16 ? 2 : 4;
+    if ((st = check_act_group(L, opts)) != MX_OK) return st;
     if ((st = check_device_ptr(X, "X")) != MX_OK) return st;
     if (!aligned16(X) || (ldx * esz) % 16 != 0) return fail(MX_ERR_ALIGNMENT, "X and every X row must be 16-byte aligned");
+    const int ag = act_group_of(opts);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (linear_fused(L, M, xdtype, opts)) {
         if ((st = check_device_ptr(blob, "blob")) != MX_OK) return st;
@@ -298,7 +340,7 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
         if (opts && opts->status && (st = check_device_ptr(opts->status, "status")) != MX_OK) return st;
         if (choose_path(L, M, opts) == 3) {
             cudaError_t e = mx::launch_gemm_rows(*L, blob, nullptr, nullptr, X, xdtype, ldx, M, Y, ldy,
-                                                 mx::plan_rows(*L, M, x_bytes(xdtype)),
+                                                 mx::plan_rows(*L, M, x_bytes(xdtype)), ag,
                                                  opts ? opts->debug_partials : nullptr,
                                                  opts ? opts->status : nullptr, s);
             if (e != cudaSuccess) return cuda_fail(e, "row decode GEMM launch");
@@ -306,20 +348,20 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
         }
         if (opts && opts->split > 8) return fail(MX_ERR_UNSUPPORTED, "split=%d above the cluster limit 8", opts->split);
         mx::DecodePlan plan = mx::plan_decode(*L, M, opts ? opts->split : 0, x_bytes(xdtype));
-        cudaError_t e = mx::launch_gemm_decode_fused(*L, blob, X, xdtype, ldx, M, Y, ldy, plan,
+        cudaError_t e = mx::launch_gemm_decode_fused(*L, blob, X, xdtype, ldx, M, Y, ldy, plan, ag,
                                                      opts ? opts->debug_partials : nullptr,
                                                      opts ? opts->status : nullptr, s);
         if (e != cudaSuccess) return cuda_fail(e, "fused decode GEMM launch");
         return MX_OK;
     }
-    const size_t need = align16(size_t(M) * L->K) + align16(size_t(2) * M);
+    const size_t need = align16(size_t(M) * L->K) + align16(size_t(2) * M * scales_per_token(L, opts));
     if (workspace == nullptr || ws_bytes < need)
         return fail(MX_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace ? ws_bytes : size_t(0));
     if ((st = check_device_ptr(workspace, "workspace")) != MX_OK) return st;
     if (!aligned16(workspace)) return fail(MX_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
     int8_t* Aq = static_cast<int8_t*>(workspace);
     uint16_t* s_a = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + align16(size_t(M) * L->K));
-    if ((st = mx_quant_act(X, xdtype, M, L->K, ldx, Aq, s_a, stream)) != MX_OK) return st;
+    if ((st = mx_quant_act_grouped(X, xdtype, M, L->K, ldx, ag, Aq, s_a, stream)) != MX_OK) return st;
     return mx_gemm(L, blob, Aq, s_a, M, Y, ldy, nullptr, 0, opts, stream);
 }
 

@@ -141,6 +141,8 @@ Geom make_geom(const mx_layout& L, const void* blob);
 cudaError_t launch_pack(const mx_layout& L, const void* W, mx_dtype wdt, int64_t ldw,
                         const uint8_t* is8, void* blob, int32_t* status, cudaStream_t s);
 
+cudaError_t launch_quant_act_grouped(const void* X, mx_dtype xdt, int M, int K, int64_t ldx, int ag,
+                                     int8_t* Aq, uint16_t* s_a, cudaStream_t s);
 cudaError_t launch_quant_act(const void* X, mx_dtype xdt, int M, int K, int64_t ldx,
                              int8_t* Aq, uint16_t* s_a, cudaStream_t s);
 
@@ -161,42 +163,45 @@ struct DecodePlan {
     int ns;             // weight ring slots per CTA
     bool ok;            // the activation slice and the ring fit in shared memory
     size_t smem;        // dynamic shared memory per CTA
-    int off_act, off_sa64, off_part, off_raw;   // its layout
+    int off_act, off_sa64, off_part, off_raw, off_sag;   // its layout
     bool xfull;         // in-kernel quantization stages whole X rows
 };
 
 // x_bytes: 0 when the kernel reads Aq, else 2 / 4 (it stages and quantizes fp16 / fp32 X)
 DecodePlan plan_decode(const mx_layout& L, int M, int split_hint, int x_bytes = 0);
 
+// ag (every launch below): 0 -- s_a holds one scale per token; the weight group g --
+// s_a holds [M][G] scales per token and group (group-wise activations)
 cudaError_t launch_gemm_decode(const mx_layout& L, const void* blob, const int8_t* Aq,
                                const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy,
-                               const DecodePlan& plan, int32_t* debug_partials, int32_t* status,
+                               const DecodePlan& plan, int ag, int32_t* debug_partials, int32_t* status,
                                cudaStream_t s);
 
-// decode GEMM for short K (<= 8192) and M <= 4: every CTA owns whole rows (16 4-bit
-// or 8 8-bit), no split of K.  Reads Aq / s_a, or quantizes X (fp16 / fp32) itself.
+// decode GEMM for short K (<= 4096) and M <= 4: every CTA owns whole rows (32 4-bit
+// or 16 8-bit), no split of K.  Reads Aq / s_a, or quantizes X (fp16 / fp32) itself.
 struct RowsPlan {
     bool ok;            // shape served (K, M, one wave, shared memory)
     int mt, m_tiles;    // tokens per CTA (1, 2, 4); ceil(M / mt)
     int n8u, units;     // 8-bit units; all units
     size_t smem;
-    int off_sc, off_z, off_act, off_sa64, off_raw, off_red;
+    int off_sc, off_z, off_act, off_sa64, off_raw, off_red, off_sag;
 };
 // x_bytes: 0 when the kernel reads Aq, else 2 / 4 (fp16 / fp32 X staged in shared memory)
 RowsPlan plan_rows(const mx_layout& L, int M, int x_bytes);
 cudaError_t launch_gemm_rows(const mx_layout& L, const void* blob, const int8_t* Aq, const uint16_t* s_a,
                              const void* X, mx_dtype xdt, int64_t ldx, int M, uint16_t* Y, int64_t ldy,
-                             const RowsPlan& p, int32_t* debug_partials, int32_t* status, cudaStream_t s);
+                             const RowsPlan& p, int ag, int32_t* debug_partials, int32_t* status,
+                             cudaStream_t s);
 
 // decode GEMM that quantizes X itself (M <= kMaxFusedTokens): one launch per call
 constexpr int kMaxFusedTokens = 4;
 bool decode_can_fuse(const mx_layout& L, int M, mx_dtype xdt);
 cudaError_t launch_gemm_decode_fused(const mx_layout& L, const void* blob, const void* X, mx_dtype xdt,
                                      int64_t ldx, int M, uint16_t* Y, int64_t ldy, const DecodePlan& plan,
-                                     int32_t* debug_partials, int32_t* status, cudaStream_t s);
+                                     int ag, int32_t* debug_partials, int32_t* status, cudaStream_t s);
 
 cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* Aq,
-                           const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy,
+                           const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy, int ag,
                            int32_t* debug_partials, int32_t* status, uint64_t timeout_ns,
                            int stall_test, cudaStream_t s);
 

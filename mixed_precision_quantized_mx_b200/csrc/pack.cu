@@ -33,7 +33,7 @@ pack_rowmap_kernel(const uint8_t* __restrict__ is8, int N, int K, int group, int
         uint32_t v = 0;
         switch (threadIdx.x) {
             case 0: v = MX_BLOB_MAGIC; break;
-            case 1: v = MX_ABI_VERSION; break;
+            case 1: v = MX_BLOB_VERSION; break;
             case 2: v = uint32_t(N); break;
             case 3: v = uint32_t(K); break;
             case 4: v = uint32_t(group); break;

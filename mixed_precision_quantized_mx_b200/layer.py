@@ -52,27 +52,31 @@ class MixedPrecisionLinear:
         if st != 0:
             raise mx.MXError(st, "mx_pack_weights", "device-side error while packing")
 
-    def workspace(self, M: int, xdtype=torch.float16, path: int = 0) -> torch.Tensor | None:
+    def workspace(self, M: int, xdtype=torch.float16, path: int = 0, act_group: int = 0) -> torch.Tensor | None:
         """Device scratch for mx_linear at M tokens (None when it needs none); cached."""
-        key = (M, xdtype, path)
+        key = (M, xdtype, path, act_group)
         if key not in self._ws:
-            n = mx.mx_linear_workspace_size(self.layout, M, xdtype, path=path)
+            n = mx.mx_linear_workspace_size(self.layout, M, xdtype, path=path, act_group=act_group)
             self._ws[key] = torch.empty(n, dtype=torch.uint8, device=self.blob.device) if n else None
         return self._ws[key]
 
-    def forward(self, X: torch.Tensor, out: torch.Tensor | None = None, path: int = 0) -> torch.Tensor:
+    def forward(self, X: torch.Tensor, out: torch.Tensor | None = None, path: int = 0,
+                act_group: int = 0) -> torch.Tensor:
+        """act_group: 0 -- one activation scale per token; the weight group -- group-wise."""
         M, K = X.shape
         if K != self.K:
             raise ValueError(f"X has K={K}, layer expects {self.K}")
         Y = out if out is not None else torch.empty((M, self.N), dtype=torch.float16, device=self.blob.device)
-        mx.mx_linear(self.layout, self.blob, X, Y, workspace=self.workspace(M, X.dtype, path), path=path)
+        mx.mx_linear(self.layout, self.blob, X, Y, workspace=self.workspace(M, X.dtype, path, act_group),
+                     path=path, act_group=act_group)
         return Y
 
     __call__ = forward
 
-    def graphed(self, x_host: torch.Tensor, y_host: torch.Tensor | None = None, path: int = 0) -> "GraphedLinear":
+    def graphed(self, x_host: torch.Tensor, y_host: torch.Tensor | None = None, path: int = 0,
+                act_group: int = 0) -> "GraphedLinear":
         """Capture host-in / host-out calls for this input buffer (see GraphedLinear)."""
-        return GraphedLinear(self, x_host, y_host, path)
+        return GraphedLinear(self, x_host, y_host, path, act_group)
 
 
 class GraphedLinear:
@@ -87,7 +91,7 @@ class GraphedLinear:
     """
 
     def __init__(self, layer: MixedPrecisionLinear, x_host: torch.Tensor, y_host: torch.Tensor | None = None,
-                 path: int = 0):
+                 path: int = 0, act_group: int = 0):
         if not x_host.is_pinned():
             raise ValueError("x_host must be pinned host memory")
         M, K = x_host.shape
@@ -97,12 +101,13 @@ class GraphedLinear:
         self.y_host = y_host if y_host is not None else torch.empty((M, layer.N), dtype=torch.float16).pin_memory()
         self.x_dev = torch.empty((M, K), dtype=x_host.dtype, device=dev)
         self.y_dev = torch.empty((M, layer.N), dtype=torch.float16, device=dev)
-        ws = layer.workspace(M, x_host.dtype, path)
+        ws = layer.workspace(M, x_host.dtype, path, act_group)
         self.stream = torch.cuda.Stream(dev)
 
         def body():
             self.x_dev.copy_(self.x_host, non_blocking=True)
-            mx.mx_linear(layer.layout, layer.blob, self.x_dev, self.y_dev, workspace=ws, path=path)
+            mx.mx_linear(layer.layout, layer.blob, self.x_dev, self.y_dev, workspace=ws, path=path,
+                         act_group=act_group)
             self.y_host.copy_(self.y_dev, non_blocking=True)
 
         with torch.cuda.stream(self.stream):        # configure kernels outside capture

@@ -34,6 +34,17 @@ def gpu_quant(X: np.ndarray):
     return Aq, sa
 
 
+def gpu_quant_grouped(X: np.ndarray, act_group: int):
+    """Group-wise codes and scales: Aq [M, K], s_a [M, K / act_group] (or [M] for 0)."""
+    Xd = to_dev(X)
+    M, K = X.shape
+    Aq = torch.empty((M, K), dtype=torch.int8, device=dev())
+    sa = torch.empty((M, K // act_group) if act_group else (M,), dtype=torch.float16, device=dev())
+    mx.mx_quant_act_grouped(Xd, Aq, sa, act_group)
+    torch.cuda.synchronize()
+    return Aq, sa
+
+
 def gpu_pack(W: np.ndarray, is8: np.ndarray, group: int, n8: int | None = None, status=None):
     N, K = W.shape
     n8 = int(is8.sum()) if n8 is None else n8

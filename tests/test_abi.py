@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version(lib):
-    assert mx.mx_version() == 1
+    assert mx.mx_version() == 2
 
 
 def _expected_total(N, K, g, n8):
@@ -187,3 +187,21 @@ def test_noalloc_scratch_limit_is_checked_before_any_launch(lib):
     assert "fixed array" in lib.mx_last_error().decode()
     assert lib.mx_linear_noalloc(ctypes.byref(L), None, None, 1, 0, 4096, None, 4096,
                                  ctypes.byref(o), None) == 0          # M = 0: no-op
+
+
+def test_group_wise_activation_options_checked_on_the_host(lib):
+    L = mx.mx_layout_init(512, 1024, 128, 51)
+    o = mx.GemmOpts(0, 0, None, None, 0, 0, 64)                      # act_group != weight group
+    assert lib.mx_gemm(ctypes.byref(L), None, None, None, 2, None, 512, None, 0, ctypes.byref(o), None) == 2
+    assert lib.mx_linear(ctypes.byref(L), None, None, 1, 2, 1024, None, 512, None, 0, ctypes.byref(o), None) == 2
+    n = ctypes.c_size_t(0)
+    assert lib.mx_linear_workspace_size(ctypes.byref(L), 8, 1, ctypes.byref(o), ctypes.byref(n)) == 2
+    # the grouped quantizer: act_group 0, 64 or 128, dividing K
+    assert lib.mx_quant_act_grouped(None, 1, 4, 1024, 1024, 32, None, None, None) == 2
+    assert lib.mx_quant_act_grouped(None, 1, 4, 192, 192, 128, None, None, None) == 2
+    assert lib.mx_quant_act_grouped(None, 1, 0, 1024, 1024, 128, None, None, None) == 0   # M = 0
+    # a workspace for grouped scales holds [M][G] of them
+    a16 = lambda v: (v + 15) // 16 * 16
+    assert mx.mx_linear_workspace_size(L, 8, act_group=128) == a16(8 * 1024) + a16(2 * 8 * 8)
+    assert mx.mx_linear_workspace_size(L, 8) == a16(8 * 1024) + a16(2 * 8)
+    assert mx.mx_linear_workspace_size(L, 2, act_group=128) == 0                 # fused

@@ -57,3 +57,13 @@ def test_graphed_rejects_pageable_input():
     layer = MixedPrecisionLinear(torch.from_numpy(lay.W).to(dev()), torch.from_numpy(lay.is8).to(dev()))
     with pytest.raises(ValueError):
         layer.graphed(torch.zeros((1, 256), dtype=torch.float16))
+
+
+@pytest.mark.parametrize("M", [1, 40])
+def test_forward_group_wise_activations(orc, M):
+    lay = inputs.llama_layer(M, 1024, 300, seed=60 + M)
+    layer = MixedPrecisionLinear(torch.from_numpy(lay.W).to(dev()), torch.from_numpy(lay.is8).to(dev()))
+    Y = layer(torch.from_numpy(lay.X).to(dev()), act_group=128)
+    Aq, sa = orc.quant_act(lay.X.astype(np.float32), act_group=128)
+    ref = orc.gemm(Aq, sa, orc.pack(lay.W, lay.is8, 128), act_group=128)[1]
+    assert_y_close(Y.cpu().numpy(), ref)
