@@ -82,10 +82,15 @@ def load_peaks():
             "source": "fallback"}
 
 
-def src_digest() -> str:
+KERNEL_SOURCES = {1: "gemm_decode.cu", 2: "gemm_tc.cu", 3: "gemm_rows.cu"}
+
+
+def src_digest(path: int) -> str:
+    """Digest of one GEMM path's kernel source and the headers every kernel includes:
+    a traffic record stays valid while these are unchanged."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixed_precision_quantized_mx_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in (KERNEL_SOURCES[path], "mx_internal.cuh", "sm100.cuh"):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -344,6 +349,14 @@ def main():
         if grem is not None:
             grem.replay()
 
+    # the first replay of a graph uploads it: do that for every graph of the timed
+    # region before timing (these replays are extra, untimed steps)
+    for gr in (g_rem, g_wrem):
+        if gr is not None:
+            gr.replay()
+    torch.cuda.synchronize()
+
+    lead = torch.empty(int(2 * l2) // 4, dtype=torch.int32, device=dev)
     sampler = ClockSampler(local)
     # sustained run of the same step graph (clock reference even for short timed regions)
     sampler.start()
@@ -359,6 +372,11 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # an L2-sized fill ahead of the start event keeps the device busy while the host
+    # submits the step graphs, so the timed region holds the steps and not the
+    # submission gap; it also leaves L2 holding none of the step's inputs
+    with torch.cuda.stream(s):
+        lead.fill_(1)
     t_time0 = time.perf_counter()
     ev0.record(s)
     with torch.cuda.stream(s):
@@ -402,7 +420,7 @@ def main():
     tfile = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if os.path.exists(tfile):
         rec = json.load(open(tfile)).get(a.workload)
-        if (rec and rec.get("src_digest") == src_digest() and rec.get("path") == path_used
+        if (rec and rec.get("src_digest") == src_digest(path_used) and rec.get("path") == path_used
                 and rec.get("fused", False) == fused):
             traffic = rec["dram_bytes_per_launch"]
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
@@ -436,7 +454,7 @@ def main():
     e2e = {"value": units_per_step * world / (e2e_ms / 1e3), "unit": unit,
            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
            "ms_per_step": e2e_ms,
-           "api": "MixedPrecisionLinear.graphed: pinned X -> device, mx_linear, Y -> pinned, one graph per step"}
+           "api": "MixedPrecisionLinear.graphed: pinned X read in by a copy kernel, mx_linear, Y written to pinned host memory by a copy kernel, one graph per step"}
 
     clocks = sampler.summary(t_time0, t_time1) or sampler.summary(t_load0, t_load1)
     if clocks is not None and "error" not in clocks:

@@ -292,6 +292,28 @@ mx_status mx_linear_noalloc(const mx_layout* L, const void* blob, const void* X,
                             int64_t ldx, uint16_t* Y, int64_t ldy, const mx_gemm_opts* opts,
                             void* stream);
 
+/*
+ * mx_copy_mapped -- copy `bytes` bytes from src to dst with a kernel, where each
+ * of the two may be device memory of the current device or pinned host memory
+ * (page-locked and mapped into the device's address space, as cudaHostAlloc
+ * and torch's pin_memory give).  The method has no counterpart of this call:
+ * it moves a layer's input in and its output out without the copy engines, so
+ * that a graph of [copy in, mx_linear, copy out] holds kernels only, and the
+ * copy-in kernel lets the next kernel start streaming its weights while the
+ * input crosses the bus (programmatic dependent launch).
+ *   dst, src  the two buffers; they must not overlap.  The caller guarantees
+ *             that both ranges lie inside their allocations.
+ *   bytes     0 is a no-op.
+ *   stream    cudaStream_t (NULL: the legacy default stream).
+ * Reads of host memory bypass the caches (ld.global.cv), so a buffer the host
+ * rewrote between two calls is read afresh; writes to host memory are seen by
+ * the host once the stream is synchronised.
+ * Returns MX_ERR_INVALID_ARG for a NULL pointer, pageable (unregistered) host
+ * memory, a host allocation without a device mapping, or another device's
+ * memory; MX_ERR_CUDA when the launch fails.  Asynchronous in `stream`.
+ */
+mx_status mx_copy_mapped(void* dst, const void* src, size_t bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

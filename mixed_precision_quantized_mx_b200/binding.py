@@ -27,7 +27,7 @@ PATH_AUTO, PATH_SPLITK, PATH_TENSOR, PATH_ROWS = 0, 1, 2, 3
 EXPORTED = ("mx_version", "mx_last_error", "mx_layout_init", "mx_layout_from_header",
             "mx_pack_weights", "mx_quant_act", "mx_gemm_workspace_size", "mx_gemm_select_path",
             "mx_gemm", "mx_linear_workspace_size", "mx_linear", "mx_linear_noalloc",
-            "mx_quant_act_grouped")
+            "mx_quant_act_grouped", "mx_copy_mapped")
 
 
 class MXError(RuntimeError):
@@ -85,9 +85,10 @@ def lib() -> ctypes.CDLL:
                             ctypes.POINTER(GemmOpts), P]
     L.mx_linear_noalloc.argtypes = [ctypes.POINTER(Layout), P, P, I, I, I64, P, I64,
                                     ctypes.POINTER(GemmOpts), P]
+    L.mx_copy_mapped.argtypes = [P, P, Z, P]
     for n in ("mx_layout_init", "mx_layout_from_header", "mx_pack_weights", "mx_quant_act",
               "mx_quant_act_grouped", "mx_gemm_workspace_size", "mx_gemm", "mx_linear_workspace_size", "mx_linear",
-              "mx_linear_noalloc"):
+              "mx_linear_noalloc", "mx_copy_mapped"):
         getattr(L, n).restype = I
     _lib = L
     return L
@@ -228,3 +229,15 @@ def mx_linear_noalloc(L: Layout, blob: torch.Tensor, X: torch.Tensor, Y: torch.T
     _check(lib().mx_linear_noalloc(ctypes.byref(L), _ptr(blob), _ptr(X), _dtype_code(X), X.shape[0],
                                    X.stride(0), _ptr(Y), Y.stride(0), ctypes.byref(o), _stream(stream)),
            "mx_linear_noalloc")
+
+
+def mx_copy_mapped(dst: torch.Tensor, src: torch.Tensor, stream=None) -> None:
+    """Copy src into dst with a kernel; either may be pinned host memory (see mx.h)."""
+    if dst.nbytes != src.nbytes:
+        raise ValueError(f"mx_copy_mapped: {dst.nbytes} bytes into {src.nbytes}")
+    if not (dst.is_contiguous() and src.is_contiguous()):
+        raise ValueError("mx_copy_mapped: contiguous tensors only")
+    for t, n in ((dst, "dst"), (src, "src")):
+        if not t.is_cuda and not t.is_pinned():
+            raise ValueError(f"mx_copy_mapped: {n} is pageable host memory (pin it first)")
+    _check(lib().mx_copy_mapped(_ptr(dst), _ptr(src), dst.nbytes, _stream(stream)), "mx_copy_mapped")

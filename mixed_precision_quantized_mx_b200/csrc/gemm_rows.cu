@@ -35,7 +35,11 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 256;
+// threads per CTA: one-token tiles take 512 (more warps to hide the latency of the
+// dot products; two CTAs still fit on an SM), wider tiles 256
+template <int MT>
+constexpr int rows_threads() { return MT == 1 ? 512 : 256; }
+constexpr int kMaxThreads = 512;
 constexpr int kRows4 = 32;                  // 4-bit rows per unit
 constexpr int kRows8 = 16;                  // 8-bit rows per unit
 constexpr int kUnitKbBytes = 2048;          // codes of one unit per k-block
@@ -53,7 +57,7 @@ struct RowsArgs {
     int64_t ldy;
     int M;
     int n8u;                // 8-bit units (t8 * 16); 4-bit units follow
-    int off_sc, off_z, off_act, off_sa64, off_raw, off_red, off_sag;   // dynamic shared memory
+    int off_sc, off_z, off_act, off_sa64, off_red, off_sag;   // dynamic shared memory
     int ag;                 // 0: one activation scale per token; g: one per token and group
     int32_t* debug;
     int32_t* status;
@@ -68,6 +72,16 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
     int d;
     asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
+}
+
+template <typename XT>
+constexpr int x_size() {
+    if constexpr (std::is_void_v<XT>) return 1;   // int8 codes
+    else return int(sizeof(XT));
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 __device__ __forceinline__ void griddep_wait() {
@@ -91,27 +105,59 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
-// four staged activations from shared memory, widened to fp32
-__device__ __forceinline__ void smem4(const __half* p, float (&v)[4]) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(p);
-    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+// eight activations of one row held in registers: fp16 packed, fp32 as two float4
+template <typename XT>
+struct X8;
+template <>
+struct X8<__half> {
+    uint4 v;
+};
+template <>
+struct X8<float> {
+    float4 lo, hi;
+};
+__device__ __forceinline__ void x8_load(X8<__half>& d, const __half* p) { d.v = __ldg(reinterpret_cast<const uint4*>(p)); }
+__device__ __forceinline__ void x8_load(X8<float>& d, const float* p) {
+    d.lo = __ldg(reinterpret_cast<const float4*>(p));
+    d.hi = __ldg(reinterpret_cast<const float4*>(p) + 1);
 }
-__device__ __forceinline__ void smem4(const float* p, float (&v)[4]) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+__device__ __forceinline__ void x8_zero(X8<__half>& d) { d.v = make_uint4(0, 0, 0, 0); }
+__device__ __forceinline__ void x8_zero(X8<float>& d) { d.lo = d.hi = make_float4(0.0f, 0.0f, 0.0f, 0.0f); }
+// |x| maximum, exact in the input type (fp16 stays packed)
+__device__ __forceinline__ float x8_absmax(const X8<__half>& d, float m) {
+    const __half2* h = reinterpret_cast<const __half2*>(&d.v);
+    __half2 a = __hmax2(__habs2(h[0]), __habs2(h[1]));
+    a = __hmax2(a, __hmax2(__habs2(h[2]), __habs2(h[3])));
+    return fmaxf(m, fmaxf(__low2float(a), __high2float(a)));
+}
+__device__ __forceinline__ float x8_absmax(const X8<float>& d, float m) {
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(d.lo.x), fabsf(d.lo.y)), fmaxf(fabsf(d.lo.z), fabsf(d.lo.w))));
+    return fmaxf(m, fmaxf(fmaxf(fabsf(d.hi.x), fabsf(d.hi.y)), fmaxf(fabsf(d.hi.z), fabsf(d.hi.w))));
+}
+__device__ __forceinline__ void x8_float(const X8<__half>& d, float (&v)[8]) {
+    const __half2* h = reinterpret_cast<const __half2*>(&d.v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h[e]);
+        v[2 * e] = f.x;
+        v[2 * e + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void x8_float(const X8<float>& d, float (&v)[8]) {
+    v[0] = d.lo.x; v[1] = d.lo.y; v[2] = d.lo.z; v[3] = d.lo.w;
+    v[4] = d.hi.x; v[5] = d.hi.y; v[6] = d.hi.z; v[7] = d.hi.w;
 }
 
 // XT: void -- read Aq and s_a; __half or float -- quantize X in-kernel.
 template <int MT, bool DEBUG, typename XT>
-__global__ void __launch_bounds__(kThreads, MT <= 2 ? 4 : 2)
+__global__ void __launch_bounds__(rows_threads<MT>(), 2)
 gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant__ CUtensorMap map8,
                  const __grid_constant__ RowsArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // the 64-byte swizzle repeats every 512 bytes: the codes start on a 1 KB boundary
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const Geom& g = a.g;
+    constexpr int NT = rows_threads<MT>();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int u = blockIdx.x;
     const bool eight = u < a.n8u;
@@ -125,7 +171,7 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
 
     __shared__ uint64_t wbar;
     __shared__ float sa_loc[MT];
-    __shared__ float red_w[kThreads / 32][MT];
+    __shared__ float red_w[NT / 32][MT];
     if (tid == 0) {
         mbar_init(&wbar, 1);
         fence_mbar_init();
@@ -145,14 +191,14 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
     {
         const __half* scl = (eight ? g.scales8 : g.scales4) + size_t(tile) * g.G * kTileRows + r0;
         const int chunks = R * 2 / 16;                             // 16-byte chunks per group
-        for (int i = tid; i < g.G * chunks; i += kThreads) {
+        for (int i = tid; i < g.G * chunks; i += NT) {
             const int gi = i / chunks, c = i % chunks;
             cp_async16(SC + gi * R + c * 8, scl + size_t(gi) * kTileRows + c * 8);
         }
         if (!eight) {
             const uint8_t* zr = g.zeros4 + size_t(tile) * g.G * kTileRows + r0;
             const int zch = R / 16;                                  // 16-byte chunks per group
-            for (int i = tid; i < g.G * zch; i += kThreads) {
+            for (int i = tid; i < g.G * zch; i += NT) {
                 const int gi = i / zch, c = i % zch;
                 cp_async16(ZP + gi * R + c * 16, zr + size_t(gi) * kTileRows + c * 16);
             }
@@ -162,16 +208,37 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
     // ---- activations (these wait for the previous kernel)
     int8_t* act = reinterpret_cast<int8_t*>(smem + a.off_act);    // [MT][K]
     float* sag = reinterpret_cast<float*>(smem + a.off_sag);        // [MT][G] when a.ag
+    int32_t* sa64 = reinterpret_cast<int32_t*>(smem + a.off_sa64);  // [MT][K / 64]
+    bool sums_done = false;
+    // this thread's row of the unit, its first k-block, and the row's output column
+    // (weights too: read before the wait)
+    const int P = NT / R;
+    const int r = tid % R, kph = tid / R;
+    const int slot_row = eight ? tile * kTileRows + r0 + r : (g.t8 + tile) * kTileRows + r0 + r;
+    const int orig = g.rowmap[slot_row];
+    // the activation rows of this token tile into L2 while the weights stream: a
+    // prefetch cannot return stale data (L2 is where every write lands), so it may
+    // run before the wait; each CTA takes a share of the 128-byte lines
+    {
+        const uint8_t* xb = std::is_void_v<XT> ? reinterpret_cast<const uint8_t*>(a.Aq)
+                                               : static_cast<const uint8_t*>(a.X);
+        const int64_t pitch = std::is_void_v<XT> ? int64_t(K) : a.ldx * int64_t(x_size<XT>());
+        const int lines = (K * x_size<XT>() + 127) / 128;             // per row
+        for (int i = blockIdx.x + tid * int(gridDim.x); i < MT * lines; i += NT * int(gridDim.x)) {
+            const int j = i / lines, l = i % lines;
+            if (m0 + j < a.M) prefetch_l2(xb + (m0 + j) * pitch + l * 128);
+        }
+    }
     griddep_wait();
     if constexpr (std::is_void_v<XT>) {
         const int chunks = K / 16;
-        for (int i = tid; i < MT * chunks; i += kThreads) {
+        for (int i = tid; i < MT * chunks; i += NT) {
             const int j = i / chunks, c = i % chunks;
             if (m0 + j < a.M) cp_async16(act + size_t(j) * K + c * 16, a.Aq + int64_t(m0 + j) * K + c * 16);
             else *reinterpret_cast<uint4*>(act + size_t(j) * K + c * 16) = make_uint4(0, 0, 0, 0);
         }
         if (a.ag) {                       // group-wise activation scales s_a[m][g]
-            for (int i = tid; i < MT * g.G; i += kThreads) {
+            for (int i = tid; i < MT * g.G; i += NT) {
                 const int j = i / g.G, gi = i % g.G;
                 sag[i] = m0 + j < a.M ? __half2float(a.s_a[int64_t(m0 + j) * g.G + gi]) : 0.0f;
             }
@@ -187,7 +254,7 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
 #pragma unroll
         for (int j = 0; j < MT; ++j) {
             const bool row = m0 + j < a.M;
-            for (int c0 = 0; c0 < K / 8; c0 += kThreads) {          // same trip count in every lane
+            for (int c0 = 0; c0 < K / 8; c0 += NT) {                // same trip count in every lane
                 const int c = c0 + tid;
                 const bool live = row && c < K / 8;
                 float v[8];
@@ -230,68 +297,66 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
         }
         __syncthreads();
     } else {
-        // whole rows: absmax, the fp16 scale, then the codes, with the quantizer's operations
+        // whole rows from registers: every thread holds CPT chunks of eight values of
+        // each row; the absmax (exact in the input type) takes one block reduction, then
+        // the fp16 scale and the codes, with the quantizer's operations.  For 4-bit
+        // units the 64-column code sums come in the same pass: eight consecutive chunks
+        // sit in eight consecutive lanes.
         const XT* X = static_cast<const XT*>(a.X);
-        XT* xs = reinterpret_cast<XT*>(smem + a.off_raw);          // [MT][K]
-        const int chunks = K * int(sizeof(XT)) / 16;
-        for (int i = tid; i < MT * chunks; i += kThreads) {
-            const int j = i / chunks, c = i % chunks;
-            if (m0 + j < a.M)
-                cp_async16(reinterpret_cast<uint8_t*>(xs + size_t(j) * K) + c * 16,
-                           reinterpret_cast<const uint8_t*>(X + int64_t(m0 + j) * a.ldx) + c * 16);
-        }
-        cp_async_wait_all();
-        __syncthreads();
+        constexpr int CPT = (kMaxK / 8 + NT - 1) / NT;            // chunks per thread and row
+        X8<XT> xv[MT][CPT];
+#pragma unroll
+        for (int j = 0; j < MT; ++j)
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) {
+                const int c = tid + i * NT;
+                if (m0 + j < a.M && c < K / 8) x8_load(xv[j][i], X + int64_t(m0 + j) * a.ldx + c * 8);
+                else x8_zero(xv[j][i]);
+            }
 #pragma unroll
         for (int j = 0; j < MT; ++j) {
             float am = 0.0f;
-            if (m0 + j < a.M) {
-#pragma unroll 4
-                for (int c = tid; c < K / 8; c += kThreads) am = absmax8(xs + size_t(j) * K + c * 8, am);
-            }
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) am = x8_absmax(xv[j][i], am);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
             if (lane == 0) red_w[warp][j] = am;
         }
         __syncthreads();
-        float sc[MT], rsc[MT];
 #pragma unroll
         for (int j = 0; j < MT; ++j) {
             float m = red_w[0][j];
 #pragma unroll
-            for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red_w[w][j]);
-            sc[j] = __half2float(act_scale(m));
-            rsc[j] = __frcp_rn(sc[j]);
-            if (tid == j) sa_loc[j] = sc[j];
-        }
-        // four words of codes per thread and pass: independent chains for the schedulers
-#pragma unroll
-        for (int j = 0; j < MT; ++j) {
-            uint32_t* aw = reinterpret_cast<uint32_t*>(act + size_t(j) * K);
-            const XT* xr = xs + size_t(j) * K;
+            for (int w = 1; w < NT / 32; ++w) m = fmaxf(m, red_w[w][j]);
+            const float sc = __half2float(act_scale(m)), rsc = __frcp_rn(sc);
+            if (tid == j) sa_loc[j] = sc;
             const bool live = m0 + j < a.M;
-            for (int c0 = tid; c0 < K / 4; c0 += 4 * kThreads) {
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const int c = c0 + v * kThreads;
-                    if (c < K / 4) {
-                        uint32_t o = 0;
-                        if (live) {
-                            float f[4];
-                            smem4(xr + c * 4, f);
-                            o = quant4(f, sc[j], rsc[j]);
-                        }
-                        aw[c] = o;
-                    }
+            for (int i = 0; i < CPT; ++i) {
+                if (i * NT >= K / 8) break;                          // the same in every lane
+                const int c = tid + i * NT;
+                uint2 o = make_uint2(0, 0);
+                if (live && c < K / 8) {
+                    float v[8];
+                    x8_float(xv[j][i], v);
+                    o.x = quant4(v, sc, rsc);
+                    o.y = quant4(v + 4, sc, rsc);
+                }
+                if (c < K / 8) *reinterpret_cast<uint2*>(act + size_t(j) * K + c * 8) = o;
+                if (!eight) {
+                    int sum = dp4a(o.x, 0x01010101u, dp4a(o.y, 0x01010101u, 0));
+                    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                    sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+                    if ((c & 7) == 0 && c < K / 8) sa64[j * (K / 64) + c / 8] = sum;
                 }
             }
         }
-        __syncthreads();
+        sums_done = true;
     }
     // activation sums of every 64 columns (the zero-point fold of 4-bit rows)
-    int32_t* sa64 = reinterpret_cast<int32_t*>(smem + a.off_sa64);   // [MT][K / 64]
-    if (!eight) {
-        for (int i = tid; i < MT * (K / 64); i += kThreads) {
+    if (!eight && !sums_done) {
+        for (int i = tid; i < MT * (K / 64); i += NT) {
             const int j = i / (K / 64), h = i % (K / 64);
             const uint4* p = reinterpret_cast<const uint4*>(act + size_t(j) * K + h * 64);
             int s = 0;
@@ -307,9 +372,9 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
         }
     }
     cp_async_wait_all();                 // scales and zero points
-    __syncthreads();
 
-    // ---- codes landed (bounded wait; on expiry record it and let the copy drain)
+    // ---- codes landed (bounded wait; on expiry record it and let the copy drain);
+    // the barrier below also publishes the activation codes and sums
     bool ok = true;
     if (tid == 0) {
         const uint64_t t0 = globaltimer_ns();
@@ -327,10 +392,6 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
     if (!__syncthreads_and(ok)) return;
 
     // ---- dot products: thread -> (row r of the unit, k-blocks kph, kph + P, ...)
-    const int P = kThreads / R;
-    const int r = tid % R, kph = tid / R;
-    const int slot_row = eight ? tile * kTileRows + r0 + r : (g.t8 + tile) * kTileRows + r0 + r;
-    const int orig = g.rowmap[slot_row];
     // physical 16-byte chunk = logical chunk ^ swz (8-bit rows: the stored 128-byte
     // swizzle of the tile; 4-bit rows: the copy's 64-byte swizzle)
     const int swz = eight ? (r & 7) : ((r >> 1) & 3);
@@ -346,9 +407,10 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
         for (int gl = 0; gl < 2; ++gl) {
             if (gl >= gpk) break;
             const int gi = kb * gpk + gl;
-            int acc[MT];
+            // two accumulators per token (even and odd chunks): shorter dependent chains
+            int acc[MT], acc2[MT];
 #pragma unroll
-            for (int j = 0; j < MT; ++j) acc[j] = 0;
+            for (int j = 0; j < MT; ++j) acc[j] = acc2[j] = 0;
             if (eight) {
                 // 16 codes per logical chunk; a group is 8 / gpk chunks
 #pragma unroll
@@ -359,19 +421,22 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
 #pragma unroll
                     for (int j = 0; j < MT; ++j) {
                         const uint4 av = *reinterpret_cast<const uint4*>(ak + size_t(j) * K + lc * 16);
-                        acc[j] = dp4a(w.x, av.x, acc[j]);
-                        acc[j] = dp4a(w.y, av.y, acc[j]);
-                        acc[j] = dp4a(w.z, av.z, acc[j]);
-                        acc[j] = dp4a(w.w, av.w, acc[j]);
+                        int& t = (c & 1) ? acc2[j] : acc[j];
+                        t = dp4a(w.x, av.x, t);
+                        t = dp4a(w.y, av.y, t);
+                        t = dp4a(w.z, av.z, t);
+                        t = dp4a(w.w, av.w, t);
                     }
                 }
+#pragma unroll
+                for (int j = 0; j < MT; ++j) acc[j] += acc2[j];
             } else {
                 // 32 codes per logical chunk: word q holds k = 8q .. 8q+7 of the chunk, the
                 // low nibbles k = 8q .. 8q+3, the high nibbles (kept in place: 16 x code as
                 // an unsigned byte) k = 8q+4 .. 8q+7; a group is 4 / gpk chunks
-                int hi16[MT];
+                int hi16[MT], hi16b[MT];
 #pragma unroll
-                for (int j = 0; j < MT; ++j) hi16[j] = 0;
+                for (int j = 0; j < MT; ++j) hi16[j] = hi16b[j] = 0;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     if (c >= 4 / gpk) break;
@@ -381,14 +446,16 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
                     for (int j = 0; j < MT; ++j) {
                         const uint4 a0 = *reinterpret_cast<const uint4*>(ak + size_t(j) * K + lc * 32);
                         const uint4 a1 = *reinterpret_cast<const uint4*>(ak + size_t(j) * K + lc * 32 + 16);
-                        acc[j] = dp4a(w.x & 0x0F0F0F0Fu, a0.x, acc[j]);
-                        hi16[j] = dp4a_us(w.x & 0xF0F0F0F0u, a0.y, hi16[j]);
-                        acc[j] = dp4a(w.y & 0x0F0F0F0Fu, a0.z, acc[j]);
-                        hi16[j] = dp4a_us(w.y & 0xF0F0F0F0u, a0.w, hi16[j]);
-                        acc[j] = dp4a(w.z & 0x0F0F0F0Fu, a1.x, acc[j]);
-                        hi16[j] = dp4a_us(w.z & 0xF0F0F0F0u, a1.y, hi16[j]);
-                        acc[j] = dp4a(w.w & 0x0F0F0F0Fu, a1.z, acc[j]);
-                        hi16[j] = dp4a_us(w.w & 0xF0F0F0F0u, a1.w, hi16[j]);
+                        int& lo = (c & 1) ? acc2[j] : acc[j];
+                        int& hi = (c & 1) ? hi16b[j] : hi16[j];
+                        lo = dp4a(w.x & 0x0F0F0F0Fu, a0.x, lo);
+                        hi = dp4a_us(w.x & 0xF0F0F0F0u, a0.y, hi);
+                        lo = dp4a(w.y & 0x0F0F0F0Fu, a0.z, lo);
+                        hi = dp4a_us(w.y & 0xF0F0F0F0u, a0.w, hi);
+                        lo = dp4a(w.z & 0x0F0F0F0Fu, a1.x, lo);
+                        hi = dp4a_us(w.z & 0xF0F0F0F0u, a1.y, hi);
+                        lo = dp4a(w.w & 0x0F0F0F0Fu, a1.z, lo);
+                        hi = dp4a_us(w.w & 0xF0F0F0F0u, a1.w, hi);
                     }
                 }
                 const int z = ZP[gi * R + r];
@@ -396,7 +463,8 @@ gemm_rows_kernel(const __grid_constant__ CUtensorMap map4, const __grid_constant
                 for (int j = 0; j < MT; ++j) {
                     const int32_t* s64 = sa64 + j * h64 + 2 * kb;
                     const int suma = gpk == 1 ? s64[0] + s64[1] : s64[gl];
-                    acc[j] += (hi16[j] >> 4) - z * suma;      // exact: hi16 is 16 x its sum
+                    // exact: the high-nibble sums are 16 x their value
+                    acc[j] += acc2[j] + ((hi16[j] + hi16b[j]) >> 4) - z * suma;
                 }
             }
             const float sw = __half2float(SC[gi * R + r]);
@@ -452,7 +520,7 @@ cudaError_t launch_t(const CUtensorMap& m4, const CUtensorMap& m8, const RowsArg
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(units, m_tiles);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(rows_threads<MT>());
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -501,14 +569,15 @@ size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
 
 }  // namespace
 
-RowsPlan plan_rows(const mx_layout& L, int M, int x_bytes) {
+RowsPlan plan_rows(const mx_layout& L, int M) {
     RowsPlan p{};
     p.mt = M <= 1 ? 1 : M <= 2 ? 2 : 4;
     p.m_tiles = std::max(1, (M + p.mt - 1) / p.mt);
     p.n8u = L.t8 * (kTileRows / kRows8);
     p.units = p.n8u + L.t4 * (kTileRows / kRows4);
     // shared memory: codes | scales | zero points | activation codes | 64-column sums |
-    // raw X rows (x_bytes per element; 0 when the kernel reads Aq) | partial sums
+    // partial sums | group-wise activation scales.  Raw activation rows are read into
+    // registers, so Aq, fp16 and fp32 inputs of one shape take the same plan.
     size_t off = size_t(L.kblocks) * kUnitKbBytes;
     p.off_sc = int(off);
     off += align16(size_t(L.G) * kRows4 * 2);
@@ -518,19 +587,13 @@ RowsPlan plan_rows(const mx_layout& L, int M, int x_bytes) {
     off += align16(size_t(p.mt) * L.K);
     p.off_sa64 = int(off);
     off += align16(size_t(p.mt) * (L.K / 64) * 4);
-    p.off_raw = int(off);
-    const size_t raw_fp32 = align16(size_t(p.mt) * L.K * 4);
-    off += align16(size_t(p.mt) * L.K * x_bytes);
     p.off_red = int(off);
-    off += size_t(kThreads) * p.mt * 4;
+    off += size_t(kMaxThreads) * p.mt * 4;
     p.off_sag = int(off);
     off += align16(size_t(p.mt) * L.G * 4);
     p.smem = off + 1024;                                // + room to align the base
-    // one wave with room left for the next launch's CTAs; the shared-memory test
-    // assumes fp32 rows whatever x_bytes is, so Aq, fp16 and fp32 inputs of one
-    // shape take the same kernel (and give the same Y)
-    const size_t smem_fp32 = p.smem - align16(size_t(p.mt) * L.K * x_bytes) + raw_fp32;
-    p.ok = M >= 1 && M <= 4 && L.K <= kMaxK && p.units * p.m_tiles <= 2 * 148 && smem_fp32 <= kMaxSmem;
+    // one wave with room left for the next launch's CTAs
+    p.ok = M >= 1 && M <= 4 && L.K <= kMaxK && p.units * p.m_tiles <= 2 * 148 && p.smem <= kMaxSmem;
     return p;
 }
 
@@ -540,9 +603,6 @@ cudaError_t launch_gemm_rows(const mx_layout& L, const void* blob, const int8_t*
                              cudaStream_t s) {
     if (M == 0) return cudaSuccess;
     if (!p.ok) return cudaErrorInvalidValue;
-    // a raw input needs the plan's room for its rows
-    if (X != nullptr && size_t(p.off_red - p.off_raw) < size_t(p.mt) * L.K * (xdt == MX_F16 ? 2 : 4))
-        return cudaErrorInvalidValue;
     cudaError_t e;
     EncodeTiledFn enc = encode_fn(&e);
     if (e != cudaSuccess) return e;
@@ -568,7 +628,6 @@ cudaError_t launch_gemm_rows(const mx_layout& L, const void* blob, const int8_t*
     a.off_z = p.off_z;
     a.off_act = p.off_act;
     a.off_sa64 = p.off_sa64;
-    a.off_raw = p.off_raw;
     a.off_red = p.off_red;
     a.off_sag = p.off_sag;
     a.ag = ag;

@@ -47,6 +47,34 @@ mx_status check_device_ptr(const void* p, const char* name) {
     return MX_OK;
 }
 
+// Device memory of the current device, or pinned host memory with a device
+// mapping: *devp is the address kernels use, *host says which.  Pageable host
+// memory is rejected (a kernel must never dereference it).
+mx_status mapped_ptr(const void* p, const char* name, const void** devp, bool* host) {
+    if (p == nullptr) return fail(MX_ERR_INVALID_ARG, "%s is NULL", name);
+    cudaPointerAttributes at;
+    cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MX_ERR_INVALID_ARG, "%s: not a CUDA pointer (%s)", name, cudaGetErrorString(e));
+    }
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (at.type == cudaMemoryTypeHost) {
+        if (at.devicePointer == nullptr) return fail(MX_ERR_INVALID_ARG, "%s: host memory without a device mapping", name);
+        *devp = at.devicePointer;
+        *host = true;
+        return MX_OK;
+    }
+    if (at.type == cudaMemoryTypeManaged || (at.type == cudaMemoryTypeDevice && at.device == dev)) {
+        *devp = p;
+        *host = false;
+        return MX_OK;
+    }
+    if (at.type == cudaMemoryTypeDevice) return fail(MX_ERR_INVALID_ARG, "%s is another device's memory", name);
+    return fail(MX_ERR_INVALID_ARG, "%s is pageable host memory (pin it first)", name);
+}
+
 mx_status check_layout(const mx_layout* L) {
     if (L == nullptr) return fail(MX_ERR_INVALID_ARG, "layout is NULL");
     mx_layout ref;
@@ -207,7 +235,7 @@ constexpr int kDecodeMaxM = 16;
 // split is asked for.
 static int choose_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
     if (opts && opts->path) return opts->path;
-    if (!(opts && opts->split > 0) && mx::plan_rows(*L, M, 0).ok) return 3;
+    if (!(opts && opts->split > 0) && mx::plan_rows(*L, M).ok) return 3;
     if (M <= kDecodeMaxM && mx::plan_decode(*L, M, 0).ok) return 1;
     return 2;
 }
@@ -251,7 +279,7 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
     const int path = choose_path(L, M, opts);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (path == 3) {
-        const mx::RowsPlan rp = mx::plan_rows(*L, M, 0);
+        const mx::RowsPlan rp = mx::plan_rows(*L, M);
         if (!rp.ok) return fail(MX_ERR_UNSUPPORTED, "M=%d K=%d: beyond the row path (M <= 4, K <= 4096, one wave)", M, L->K);
         cudaError_t e = mx::launch_gemm_rows(*L, blob, Aq, s_a, nullptr, MX_F16, 0, M, Y, ldy, rp, ag,
                                              opts ? opts->debug_partials : nullptr, opts ? opts->status : nullptr, s);
@@ -293,13 +321,25 @@ int x_bytes(mx_dtype xdt) { return xdt == MX_F16 ? 2 : 4; }
 
 bool linear_fused(const mx_layout* L, int M, mx_dtype xdt, const mx_gemm_opts* opts) {
     const int path = choose_path(L, M, opts);
-    if (path == 3) return mx::plan_rows(*L, M, 0).ok;
+    if (path == 3) return mx::plan_rows(*L, M).ok;
     if (path != 1 || !mx::decode_can_fuse(*L, M, xdt)) return false;
     const mx::DecodePlan p = mx::plan_decode(*L, M, opts ? opts->split : 0, x_bytes(xdt));
     return p.ok && p.mt <= mx::kMaxFusedTokens;
 }
 
 }  // namespace
+
+mx_status mx_copy_mapped(void* dst, const void* src, size_t bytes, void* stream) {
+    const void *d = nullptr, *s = nullptr;
+    bool dh = false, sh = false;
+    mx_status st = mapped_ptr(dst, "dst", &d, &dh);
+    if (st != MX_OK) return st;
+    if ((st = mapped_ptr(src, "src", &s, &sh)) != MX_OK) return st;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(d), b0 = reinterpret_cast<uintptr_t>(s);
+    if (bytes && a0 < b0 + bytes && b0 < a0 + bytes) return fail(MX_ERR_INVALID_ARG, "dst and src overlap");
+    cudaError_t e = mx::launch_copy_mapped(const_cast<void*>(d), s, bytes, sh, dh, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MX_OK : cuda_fail(e, "copy_mapped launch");
+}
 
 mx_status mx_linear_workspace_size(const mx_layout* L, int M, mx_dtype xdtype, const mx_gemm_opts* opts,
                                    size_t* bytes) {
@@ -340,7 +380,7 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
         if (opts && opts->status && (st = check_device_ptr(opts->status, "status")) != MX_OK) return st;
         if (choose_path(L, M, opts) == 3) {
             cudaError_t e = mx::launch_gemm_rows(*L, blob, nullptr, nullptr, X, xdtype, ldx, M, Y, ldy,
-                                                 mx::plan_rows(*L, M, x_bytes(xdtype)), ag,
+                                                 mx::plan_rows(*L, M), ag,
                                                  opts ? opts->debug_partials : nullptr,
                                                  opts ? opts->status : nullptr, s);
             if (e != cudaSuccess) return cuda_fail(e, "row decode GEMM launch");

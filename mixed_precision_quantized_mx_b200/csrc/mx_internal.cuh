@@ -141,6 +141,9 @@ Geom make_geom(const mx_layout& L, const void* blob);
 cudaError_t launch_pack(const mx_layout& L, const void* W, mx_dtype wdt, int64_t ldw,
                         const uint8_t* is8, void* blob, int32_t* status, cudaStream_t s);
 
+cudaError_t launch_copy_mapped(void* dst, const void* src, size_t bytes, bool src_host, bool dst_host,
+                               cudaStream_t s);
+
 cudaError_t launch_quant_act_grouped(const void* X, mx_dtype xdt, int M, int K, int64_t ldx, int ag,
                                      int8_t* Aq, uint16_t* s_a, cudaStream_t s);
 cudaError_t launch_quant_act(const void* X, mx_dtype xdt, int M, int K, int64_t ldx,
@@ -184,10 +187,10 @@ struct RowsPlan {
     int mt, m_tiles;    // tokens per CTA (1, 2, 4); ceil(M / mt)
     int n8u, units;     // 8-bit units; all units
     size_t smem;
-    int off_sc, off_z, off_act, off_sa64, off_raw, off_red, off_sag;
+    int off_sc, off_z, off_act, off_sa64, off_red, off_sag;
 };
-// x_bytes: 0 when the kernel reads Aq, else 2 / 4 (fp16 / fp32 X staged in shared memory)
-RowsPlan plan_rows(const mx_layout& L, int M, int x_bytes);
+// the same plan serves Aq, fp16 and fp32 inputs (raw rows are read into registers)
+RowsPlan plan_rows(const mx_layout& L, int M);
 cudaError_t launch_gemm_rows(const mx_layout& L, const void* blob, const int8_t* Aq, const uint16_t* s_a,
                              const void* X, mx_dtype xdt, int64_t ldx, int M, uint16_t* Y, int64_t ldy,
                              const RowsPlan& p, int ag, int32_t* debug_partials, int32_t* status,

@@ -86,6 +86,9 @@ class GraphedLinear:
     (quantize + GEMM, one kernel for decode-sized M) and copies Y back into the
     pinned host output, so one `replay()` per
     step is the whole host-to-host pass with a single launch from the host.
+    The copies are kernels that read and write the mapped host buffers
+    (mx_copy_mapped), so the graph holds kernels only and mx_linear's weight
+    stream starts while the input crosses the bus.
     The caller rewrites `x_host` between replays and reads `y_host` after the
     stream is synchronised (or after an event recorded after `replay()`).
     """
@@ -94,6 +97,8 @@ class GraphedLinear:
                  path: int = 0, act_group: int = 0):
         if not x_host.is_pinned():
             raise ValueError("x_host must be pinned host memory")
+        if y_host is not None and not y_host.is_pinned():
+            raise ValueError("y_host must be pinned host memory")
         M, K = x_host.shape
         dev = layer.blob.device
         self.layer = layer
@@ -105,10 +110,10 @@ class GraphedLinear:
         self.stream = torch.cuda.Stream(dev)
 
         def body():
-            self.x_dev.copy_(self.x_host, non_blocking=True)
+            mx.mx_copy_mapped(self.x_dev, self.x_host)
             mx.mx_linear(layer.layout, layer.blob, self.x_dev, self.y_dev, workspace=ws, path=path,
                          act_group=act_group)
-            self.y_host.copy_(self.y_dev, non_blocking=True)
+            mx.mx_copy_mapped(self.y_host, self.y_dev)
 
         with torch.cuda.stream(self.stream):        # configure kernels outside capture
             body()
