@@ -59,7 +59,8 @@ def parse():
     p.add_argument("--frac8", type=float, default=0.10)
     p.add_argument("--group", type=int, default=128)
     p.add_argument("--path", type=int, default=0,
-                   help="0 auto, 1 split-K CUDA cores, 2 tensor cores, 3 whole rows per CTA")
+                   help="0 auto, 1 split-K CUDA cores, 2 tensor cores, 3 whole rows per CTA, "
+                        "4 tensor cores on CTA pairs")
     p.add_argument("--act-group", type=int, default=0,
                    help="activation scales: 0 one per token; the weight group: one per token and group")
     p.add_argument("--impl", default="mx", choices=["mx", "reference"])
@@ -82,7 +83,7 @@ def load_peaks():
             "source": "fallback"}
 
 
-KERNEL_SOURCES = {1: "gemm_decode.cu", 2: "gemm_tc.cu", 3: "gemm_rows.cu"}
+KERNEL_SOURCES = {1: "gemm_decode.cu", 2: "gemm_tc.cu", 3: "gemm_rows.cu", 4: "gemm_tc2.cu"}
 
 
 def src_digest(path: int) -> str:
@@ -427,7 +428,8 @@ def main():
                 "frac": achieved / peak, "traffic": traffic,
                 "kernel": {1: "gemm_decode_kernel (cluster split-K, CUDA cores)",
                            2: "gemm_tc_kernel (tcgen05)",
-                           3: "gemm_rows_kernel (whole rows per CTA, CUDA cores)"}[path_used]
+                           3: "gemm_rows_kernel (whole rows per CTA, CUDA cores)",
+                           4: "gemm_tc2_kernel (tcgen05 on CTA pairs)"}[path_used]
                           + (", activation quantizer fused" if fused else ""),
                 "algorithmic_per_launch": algo, "launch_ms": gemm_ms,
                 "peak_source": (f"{peaks['source']} HBM copy" if bound == "hbm" else

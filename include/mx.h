@@ -99,7 +99,8 @@ typedef struct mx_layout {
 /* Options of mx_gemm; pass NULL for the defaults (all fields zero). */
 typedef struct mx_gemm_opts {
     int32_t path;              /* 0 auto; 1 split-K CUDA-core path; 2 tensor-core path;
-                                  3 row CUDA-core path (whole rows per CTA) */
+                                  3 row CUDA-core path (whole rows per CTA); 4 tensor-core
+                                  path on CTA pairs (cta_group::2, 256 rows x 192 tokens) */
     int32_t split;             /* path 1: CTAs (a thread-block cluster, 1..8) that split
                                   the K range of each row unit (0 = auto); a split
                                   asked for under auto selects path 1 */

@@ -297,17 +297,16 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
         if (e != cudaSuccess) return cuda_fail(e, "decode GEMM launch");
         return MX_OK;
     }
-    if (path == 2) {
+    if (path == 2 || path == 4) {
         if (opts && opts->test_stall && !opts->status)
             return fail(MX_ERR_INVALID_ARG, "test_stall needs a status word");
         if (opts && opts->wait_timeout_us < 0) return fail(MX_ERR_INVALID_ARG, "wait_timeout_us < 0");
         const uint64_t timeout_ns =
             (opts && opts->wait_timeout_us > 0) ? uint64_t(opts->wait_timeout_us) * 1000u : 2000000000ull;
-        cudaError_t e = mx::launch_gemm_tc(*L, blob, Aq, s_a, M, Y, ldy, ag,
-                                           opts ? opts->debug_partials : nullptr,
-                                           opts ? opts->status : nullptr, timeout_ns,
-                                           opts ? opts->test_stall : 0, s);
-        if (e != cudaSuccess) return cuda_fail(e, "tensor-core GEMM launch");
+        auto launch = path == 2 ? mx::launch_gemm_tc : mx::launch_gemm_tc2;
+        cudaError_t e = launch(*L, blob, Aq, s_a, M, Y, ldy, ag, opts ? opts->debug_partials : nullptr,
+                               opts ? opts->status : nullptr, timeout_ns, opts ? opts->test_stall : 0, s);
+        if (e != cudaSuccess) return cuda_fail(e, path == 2 ? "tensor-core GEMM launch" : "pair tensor-core GEMM launch");
         return MX_OK;
     }
     return fail(MX_ERR_INVALID_ARG, "unknown GEMM path %d", path);

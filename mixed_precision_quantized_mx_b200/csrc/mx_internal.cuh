@@ -208,4 +208,10 @@ cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* A
                            int32_t* debug_partials, int32_t* status, uint64_t timeout_ns,
                            int stall_test, cudaStream_t s);
 
+// the same GEMM on CTA pairs (cta_group::2): 256 weight rows x 192 tokens per tile
+cudaError_t launch_gemm_tc2(const mx_layout& L, const void* blob, const int8_t* Aq,
+                            const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy, int ag,
+                            int32_t* debug_partials, int32_t* status, uint64_t timeout_ns,
+                            int stall_test, cudaStream_t s);
+
 }  // namespace mx
