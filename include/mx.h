@@ -208,8 +208,11 @@ mx_status mx_gemm_workspace_size(const mx_layout* L, int M, const mx_gemm_opts* 
  *       4-bit (or 16 8-bit) rows over the whole K, no reduction between CTAs;
  *   1 = split-K path: M <= 16; the K split of each row unit is one thread-block
  *       cluster reduced through distributed shared memory;
- *   2 = tensor-core path (larger M).
- * Auto selection tries them in that order.  Negative mx_status on bad arguments.
+ *   4 = tensor cores on CTA pairs (larger M): tcgen05.mma.cta_group::2 over 256
+ *       weight rows x 128 tokens per pair of CTAs.
+ * Auto selection tries them in that order.  2 = the one-CTA tensor-core kernel
+ * (128 x 128 tiles) is taken only when opts->path asks for it.  Negative
+ * mx_status on bad arguments.
  */
 int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts);
 

@@ -228,16 +228,18 @@ mx_status mx_quant_act_grouped(const void* X, mx_dtype xdtype, int M, int K, int
 }
 
 // Decode-sized M is bound by HBM: the split-K CUDA-core path streams the
-// weights with enough CTAs; from 17 tokens on, the tensor-core path.
+// weights with enough CTAs; from 17 tokens on, the tensor cores.
 constexpr int kDecodeMaxM = 16;
 
 // Short K and M <= 4 take the row kernel (whole rows per CTA) unless a cluster
-// split is asked for.
+// split is asked for; larger M the tensor cores on CTA pairs, which measured at
+// least as fast as the one-CTA tensor-core kernel from 32 tokens up on the
+// Llama shapes (path 2 stays available when asked for).
 static int choose_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
     if (opts && opts->path) return opts->path;
     if (!(opts && opts->split > 0) && mx::plan_rows(*L, M).ok) return 3;
     if (M <= kDecodeMaxM && mx::plan_decode(*L, M, 0).ok) return 1;
-    return 2;
+    return 4;
 }
 
 int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {

@@ -128,11 +128,12 @@ def test_paths_need_no_workspace_and_dispatch_on_m(lib):
     assert mx.mx_gemm_select_path(L, 5) == mx.PATH_SPLITK
     assert mx.mx_gemm_select_path(L, 1, split=2) == mx.PATH_SPLITK   # a split asks for clusters
     assert mx.mx_gemm_select_path(L, 16) == mx.PATH_SPLITK
-    assert mx.mx_gemm_select_path(L, 17) == mx.PATH_TENSOR
-    assert mx.mx_gemm_select_path(L, 1, path=mx.PATH_TENSOR) == mx.PATH_TENSOR
+    assert mx.mx_gemm_select_path(L, 17) == mx.PATH_PAIR           # tensor cores on CTA pairs
+    assert mx.mx_gemm_select_path(L, 2048) == mx.PATH_PAIR
+    assert mx.mx_gemm_select_path(L, 1, path=mx.PATH_TENSOR) == mx.PATH_TENSOR   # asked for
     # 16 tokens of a 64K-column activation slice cannot be staged per cluster: tensor cores
     Lbig = mx.mx_layout_init(1024, 65536, 128, 102)
-    assert mx.mx_gemm_select_path(Lbig, 16) == mx.PATH_TENSOR
+    assert mx.mx_gemm_select_path(Lbig, 16) == mx.PATH_PAIR
     # the row path needs K <= 4096 and one wave of CTAs
     assert mx.mx_gemm_select_path(mx.mx_layout_init(4096, 8192, 128, 410), 1) == mx.PATH_SPLITK
     assert mx.mx_gemm_select_path(mx.mx_layout_init(14336, 4096, 128, 1434), 1) == mx.PATH_SPLITK
