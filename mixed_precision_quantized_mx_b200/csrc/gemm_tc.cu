@@ -332,17 +332,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             // group scales live in a ring of kScaleRing registers, each loaded kScaleRing
             // groups before its use; the group loop is unrolled by kScaleRing so every
             // ring slot is a fixed register and no instruction waits on a young load
-            float swr[kScaleRing];
+            // (the ring holds the raw fp16 values: converting at the load would wait for it)
+            __half swr[kScaleRing];
 #pragma unroll
             for (int j = 0; j < kScaleRing; ++j)
-                swr[j] = j < g.G ? __half2float(sc[size_t(j) * kTileRows]) : 0.0f;
+                swr[j] = j < g.G ? sc[size_t(j) * kTileRows] : __float2half_rn(0.0f);
             for (int gi0 = 0; gi0 < g.G; gi0 += kScaleRing) {
 #pragma unroll
                 for (int j = 0; j < kScaleRing; ++j) {
                     const int gi = gi0 + j;
                     if (gi >= g.G) break;
-                    const float sw = swr[j];
-                    if (gi + kScaleRing < g.G) swr[j] = __half2float(sc[size_t(gi + kScaleRing) * kTileRows]);
+                    const float sw = __half2float(swr[j]);
+                    if (gi + kScaleRing < g.G) swr[j] = sc[size_t(gi + kScaleRing) * kTileRows];
                     const float2 s2 = make_float2(sw, sw);
                     const uint32_t b = gc % kAccBufs, u = gc / kAccBufs;
                     // every lane waits; the warp leaves together if any lane gave up, because

@@ -341,17 +341,18 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
             // groups before its use; the group loop is unrolled by kScaleRing so every
             // ring slot is a fixed register and no instruction waits on a young load
             // (a tile without rows multiplies by zero)
-            float swr[kScaleRing];
+            // (the ring holds the raw fp16 values: converting at the load would wait for it)
+            __half swr[kScaleRing];
 #pragma unroll
             for (int j = 0; j < kScaleRing; ++j)
-                swr[j] = un.rows && j < g.G ? __half2float(sc[size_t(j) * kTileRows]) : 0.0f;
+                swr[j] = un.rows && j < g.G ? sc[size_t(j) * kTileRows] : __float2half_rn(0.0f);
             for (int gi0 = 0; gi0 < g.G; gi0 += kScaleRing) {
 #pragma unroll
                 for (int j = 0; j < kScaleRing; ++j) {
                     const int gi = gi0 + j;
                     if (gi >= g.G) break;
-                    const float sw = swr[j];
-                    if (un.rows && gi + kScaleRing < g.G) swr[j] = __half2float(sc[size_t(gi + kScaleRing) * kTileRows]);
+                    const float sw = __half2float(swr[j]);
+                    if (un.rows && gi + kScaleRing < g.G) swr[j] = sc[size_t(gi + kScaleRing) * kTileRows];
                     const uint32_t b = gc % kAccBufs;
                     // every lane waits; the warp leaves together if any lane gave up (the
                     // TMEM accesses below are warp-collective)
