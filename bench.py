@@ -66,6 +66,9 @@ def parse():
     p.add_argument("--impl", default="mx", choices=["mx", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--sweep", action="store_true",
+                   help="the K = N = 8192 sweep over 8-bit row fraction, M and group size: one JSON "
+                        "line per (fraction, group, M, path) and the GEMV / tensor-core crossover")
     a = p.parse_args()
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -237,11 +240,117 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ sweep
+SWEEP_FRACS = (0.0, 0.05, 0.10, 0.25, 0.50)
+SWEEP_M = (1, 8, 64, 512, 8192)
+SWEEP_GROUPS = (64, 128)
+
+
+def run_sweep(a):
+    """K = N = 8192: 8-bit row fraction x M x group size.  Every step is one mx_linear call
+    (quantizer + GEMM) replayed from a CUDA graph over rotated copies (>= 4x L2), timed with
+    events on its stream after warm-up replays.  Each (fraction, group, M) is timed on the
+    decode path (split-K, 1) where it serves and on the tensor cores (4, on CTA pairs); the
+    crossover is the smallest M at which the tensor cores win."""
+    import torch
+    from mixed_precision_quantized_mx_b200 import binding as mx
+    from mixed_precision_quantized_mx_b200 import build as mxbuild
+    from mixed_precision_quantized_mx_b200 import inputs, model
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    mxbuild.build()
+    peaks = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    K = N = 8192
+    s = torch.cuda.Stream(dev)
+    rows = []
+    for g in SWEEP_GROUPS:
+        for frac in SWEEP_FRACS:
+            base = inputs.llama_layer(1, K, N, frac, g, seed=a.seed)
+            n8 = base.n8
+            L = mx.mx_layout_init(N, K, g, n8)
+            blob0 = torch.empty(L.total_bytes, dtype=torch.uint8, device=dev)
+            mx.mx_pack_weights(L, torch.from_numpy(base.W).to(dev), torch.from_numpy(base.is8).to(dev), blob0)
+            rng = np.random.default_rng(a.seed + 17)
+            for M in SWEEP_M:
+                X = torch.from_numpy(inputs.activations(rng, M, K, int(round(0.01 * K)), dtype=np.float16)).to(dev)
+                per_step = L.total_bytes + X.nbytes + 2 * M * N
+                R = int(min(16, max(2, math.ceil(4 * l2 / per_step))))
+                blobs = [blob0] + [blob0.clone() for _ in range(R - 1)]
+                Xs = [X] + [X.clone() for _ in range(R - 1)] if M <= 64 else [X] * R
+                Ys = [torch.empty((M, N), dtype=torch.float16, device=dev) for _ in range(min(R, 2))]
+                auto = mx.mx_gemm_select_path(L, M)
+                for path in (1, 4):
+                    if path == 1 and M > 64:
+                        continue                       # decode-sized M only
+                    try:
+                        ws_n = mx.mx_linear_workspace_size(L, M, torch.float16, path=path)
+                    except mx.MXError:
+                        continue
+                    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
+
+                    def step(i):
+                        mx.mx_linear(L, blobs[i], Xs[i], Ys[i % len(Ys)], workspace=ws, path=path)
+                    try:
+                        with torch.cuda.stream(s):
+                            for i in range(R):
+                                step(i)
+                        torch.cuda.synchronize()
+                    except mx.MXError:
+                        continue                       # the path does not serve this shape
+                    gr = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(gr, stream=s):
+                        for i in range(R):
+                            step(i)
+                    for _ in range(3):                 # uploads the graph and warms up
+                        gr.replay()
+                    torch.cuda.synchronize()
+                    t0 = time.perf_counter()
+                    gr.replay()
+                    torch.cuda.synchronize()
+                    reps = int(min(200, max(3, 0.15 / max(time.perf_counter() - t0, 1e-6))))
+                    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    ev0.record(s)
+                    with torch.cuda.stream(s):
+                        for _ in range(reps):
+                            gr.replay()
+                    ev1.record(s)
+                    torch.cuda.synchronize()
+                    us = ev0.elapsed_time(ev1) * 1e3 / (reps * R)
+                    ops = model.gemm_ops(M, N, K)
+                    byts = model.linear_bytes(M, N, K, g, n8, 2)
+                    row = {"sweep": "K=N=8192", "frac8": frac, "group": g, "n8": n8, "M": M, "path": path,
+                           "auto_path": auto, "us_per_step": round(us, 3),
+                           "tops": round(ops / us / 1e6, 2), "gbs": round(byts / us / 1e3, 1),
+                           "frac_hbm": round(byts / us / 1e3 / peaks["hbm_gbs"], 4),
+                           "frac_int8": round(ops / us / 1e6 / (2 * peaks["bf16_tflops"]), 4)}
+                    rows.append(row)
+                    print(json.dumps(row), flush=True)
+                    del gr
+                del blobs, Xs, Ys
+                torch.cuda.empty_cache()
+    # the crossover: smallest M at which the tensor cores beat the decode path
+    summary = []
+    for g in SWEEP_GROUPS:
+        for frac in SWEEP_FRACS:
+            cross = None
+            for M in SWEEP_M:
+                t = {r["path"]: r["us_per_step"] for r in rows if r["group"] == g and r["frac8"] == frac and r["M"] == M}
+                if 4 in t and (1 not in t or t[4] < t[1]):
+                    cross = M
+                    break
+            summary.append({"frac8": frac, "group": g, "tensor_cores_from_M": cross})
+    print(json.dumps({"sweep_crossover": summary}), flush=True)
+
+
 # ------------------------------------------------------------------ main arm
 def main():
     a = parse()
     if a.impl == "reference":
         return run_reference(a)
+    if a.sweep:
+        return run_sweep(a)
 
     import torch
     import torch.distributed as dist
