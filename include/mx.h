@@ -100,10 +100,13 @@ typedef struct mx_layout {
 typedef struct mx_gemm_opts {
     int32_t path;              /* 0 auto; 1 split-K CUDA-core path; 2 tensor-core path;
                                   3 row CUDA-core path (whole rows per CTA); 4 tensor-core
-                                  path on CTA pairs (cta_group::2, 256 rows x 192 tokens) */
+                                  path on CTA pairs (cta_group::2, 256 rows x 128 tokens) */
     int32_t split;             /* path 1: CTAs (a thread-block cluster, 1..8) that split
                                   the K range of each row unit (0 = auto); a split
-                                  asked for under auto selects path 1 */
+                                  asked for under auto selects path 1 for M <= 16.
+                                  path 4: K splits (1..8; 0 = auto: more than one only
+                                  when the unsplit grid leaves CTA pairs idle and the
+                                  workspace holds the split sums) */
     int32_t* debug_partials;   /* device int32 [M][N][G] or NULL: every per-group
                                   int32 partial P[m][n][g] (original row order) */
     int32_t* status;           /* device int32 or NULL: kernel-side error code */
@@ -193,9 +196,9 @@ mx_status mx_quant_act_grouped(const void* X, mx_dtype xdtype, int M, int K, int
 
 /*
  * mx_gemm_workspace_size -- host only.  Bytes of device workspace mx_gemm
- * needs for this layer at M tokens with these options.  Both GEMM paths of this
- * version run without scratch memory, so it reports 0; callers that size and
- * pass a workspace stay correct if a later version needs one.
+ * uses for this layer at M tokens with these options: S * M * N * 4 (rounded up
+ * to 256) when path 4 splits K S > 1 ways, else 0.  A negative split is
+ * MX_ERR_INVALID_ARG.
  */
 mx_status mx_gemm_workspace_size(const mx_layout* L, int M, const mx_gemm_opts* opts,
                                  size_t* bytes);
@@ -222,9 +225,12 @@ int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts);
  *   blob    device, produced by mx_pack_weights for the same layout
  *   Aq      device int8 [M][K] row-major (dense); s_a device fp16 bits [M]
  *   Y       device fp16 [M][ldy], ldy >= N; column n is original row n of W
- *   workspace / ws_bytes: device scratch of at least
- *           mx_gemm_workspace_size(L, M, opts) bytes (may be NULL if 0; unused
- *           by this version)
+ *   workspace / ws_bytes: device scratch, 16-byte aligned, of
+ *           mx_gemm_workspace_size(L, M, opts) bytes (NULL if 0).  Path 4 splits
+ *           K S > 1 ways only into such a workspace: each split writes fp32 sums
+ *           [S][M][N] and a second kernel adds them in split order.  Without it
+ *           an automatic split runs unsplit; an asked-for split returns
+ *           MX_ERR_WORKSPACE.
  * Per group g: P = sum_{k in g} Aq[m,k] (W_q[n,k] - z[n,g]) exactly in int32
  * (|P| <= 127*127*128 < 2^22), acc[m,n] = sum_g float(P) * s_w[n,g] in fp32,
  * then Y[m,n] = fp16_rn(acc * s_a[m]).  The fp32 summation order depends on the
@@ -239,7 +245,9 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
  * mx_linear_workspace_size -- host only.  Bytes of device scratch mx_linear
  * needs at M tokens of activations of type xdtype: 0 when the call is served by
  * the decode kernel that quantizes X itself, else room for Aq (M*K bytes) and
- * s_a (2*M bytes), each rounded up to 16 bytes.
+ * s_a (2*M bytes, or 2*M*G with group-wise scales), each rounded up to 16
+ * bytes, followed (from the next 256-byte boundary) by mx_gemm's workspace when
+ * it needs one.  Less than that but at least Aq and s_a runs unsplit.
  */
 mx_status mx_linear_workspace_size(const mx_layout* L, int M, mx_dtype xdtype,
                                    const mx_gemm_opts* opts, size_t* bytes);
@@ -284,9 +292,12 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
  * Nothing in the array has to start at zero: the quantizer writes every byte
  * of it that the GEMM then reads.  The call never allocates or frees device
  * or host memory.
- * Returns MX_ERR_WORKSPACE, before anything is launched, when the scratch
- * needed exceeds MX_NOALLOC_SCRATCH_BYTES; MX_ERR_CUDA when the address
- * lookup fails; otherwise what mx_linear returns.
+ * A K split of the tensor-core GEMM (see mx_gemm) uses the rest of the array
+ * when its sums fit there, else the GEMM runs unsplit: the result is that of
+ * mx_linear given a workspace of MX_NOALLOC_SCRATCH_BYTES bytes.
+ * Returns MX_ERR_WORKSPACE, before anything is launched, when Aq and s_a
+ * exceed MX_NOALLOC_SCRATCH_BYTES; MX_ERR_CUDA when the address lookup fails;
+ * otherwise what mx_linear returns.
  * All calls on one device share the one array, so two calls whose kernels can
  * run at the same time (streams with no order between them, or several host
  * threads) race on it; calls in one stream are ordered and safe.  Make the

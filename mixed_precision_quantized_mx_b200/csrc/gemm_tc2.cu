@@ -93,7 +93,10 @@ struct Tc2Args {
     int64_t ldy;
     int M;
     int n_tt;            // token tiles of BN
-    int n_units;         // pairs of row tiles x token tiles
+    int n_units;         // pairs of row tiles x K splits x token tiles
+    int S;               // K splits (1: each unit covers the whole K)
+    int ss_per;          // stages per split
+    float* part;         // S > 1: fp32 partial sums [S][M][N] (original column order)
     int32_t* debug;
     int32_t* status;
     uint64_t timeout_ns;
@@ -107,21 +110,27 @@ __device__ __forceinline__ uint32_t widen_hi(uint32_t w, uint32_t zc) {
     return (((w >> 4) & 0x0F0F0F0Fu) + zc) ^ 0x80808080u;
 }
 
-// Unit u of the persistent walk: a pair of consecutive row tiles and a token
-// tile.  Consecutive units share the row-tile pair, so the pairs working at one
-// time read each weight block from HBM about once.
+// Unit u of the persistent walk: a pair of consecutive row tiles, a range of K
+// (a split) and a token tile.  Consecutive units share the row-tile pair and the
+// split, so the pairs working at one time read each weight block from HBM about once.
 struct Unit {
     int rt;       // this CTA's row tile (may be past the last: then it has no rows)
     int tt;       // token tile
+    int ks;       // K split
+    int sp0, sp1; // its stages [sp0, sp1)
     bool rows;    // this CTA has weight rows in this unit
     bool eight;
     int lt;       // index among the tiles of its kind
 };
 
-__device__ __forceinline__ Unit unit_of(const Tc2Args& a, int u, uint32_t rank) {
+__device__ __forceinline__ Unit unit_of(const Tc2Args& a, int u, uint32_t rank, int n_ss) {
     Unit r;
-    r.rt = 2 * (u / a.n_tt) + int(rank);
+    const int pk = u / a.n_tt;                    // (pair, split)
+    r.rt = 2 * (pk / a.S) + int(rank);
+    r.ks = pk % a.S;
     r.tt = u % a.n_tt;
+    r.sp0 = r.ks * a.ss_per;
+    r.sp1 = min(n_ss, r.sp0 + a.ss_per);
     r.rows = r.rt < a.g.t8 + a.g.t4;
     r.eight = r.rt < a.g.t8;
     r.lt = r.eight ? r.rt : r.rt - a.g.t8;
@@ -190,8 +199,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
         int it = 0;
         if (!a.stall_test) {
             for (int u = cid; u < a.n_units; u += ncl) {
-                const Unit un = unit_of(a, u, rank);
-                for (int sp = 0; sp < n_ss; ++sp, ++it) {
+                const Unit un = unit_of(a, u, rank, n_ss);
+                for (int sp = un.sp0; sp < un.sp1; ++sp, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
                     bool ok = true;
@@ -230,7 +239,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
             int it = 0;
             uint32_t gc = 0;
             for (int u = cid; u < a.n_units; u += ncl) {
-                for (int sp = 0; sp < n_ss; ++sp, ++it) {
+                const Unit un = unit_of(a, u, rank, n_ss);
+                for (int sp = un.sp0; sp < un.sp1; ++sp, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
                     if (!mbar_wait_bounded(&S.ready[s], ph, abort, a.status, a.timeout_ns)) goto mma_out;
@@ -266,9 +276,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
         const int wt = threadIdx.x - 64;
         int it = 0;
         for (int u = cid; u < a.n_units; u += ncl) {
-            const Unit un = unit_of(a, u, rank);
+            const Unit un = unit_of(a, u, rank, n_ss);
             const bool widen = un.rows && !un.eight;
-            for (int sp = 0; sp < n_ss; ++sp, ++it) {
+            for (int sp = un.sp0; sp < un.sp1; ++sp, ++it) {
                 const int s = it % kStages;
                 const uint32_t ph = (it / kStages) & 1;
                 const bool ok = mbar_wait_bounded(&S.full[s], ph, abort, a.status, a.timeout_ns);
@@ -330,8 +340,10 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
             for (int b = 0; b < kAccBufs; ++b) mbar_arrive_cluster(acc_empty_c + 8u * uint32_t(b));
         uint32_t gc = 0;
         for (int u = cid; u < a.n_units; u += ncl) {
-            const Unit un = unit_of(a, u, rank);
-            const __half* sc = (un.eight ? g.scales8 : g.scales4) + size_t(un.lt) * g.G * kTileRows + row;
+            const Unit un = unit_of(a, u, rank, n_ss);
+            // this unit's groups [g0, g1)
+            const int g0 = un.sp0 * KPS * gpk, g1 = min(g.G, un.sp1 * KPS * gpk);
+            const __half* sc = (un.eight ? g.scales8 : g.scales4) + (size_t(un.lt) * g.G + g0) * kTileRows + row;
             const int orig = un.rows ? g.rowmap[un.rt * kTileRows + row] : -1;
             const int m0 = un.tt * BN + cb;          // this warp's first token
             float2 acc[kEpiTokens / 2];
@@ -345,14 +357,14 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
             __half swr[kScaleRing];
 #pragma unroll
             for (int j = 0; j < kScaleRing; ++j)
-                swr[j] = un.rows && j < g.G ? sc[size_t(j) * kTileRows] : __float2half_rn(0.0f);
-            for (int gi0 = 0; gi0 < g.G; gi0 += kScaleRing) {
+                swr[j] = un.rows && g0 + j < g1 ? sc[size_t(j) * kTileRows] : __float2half_rn(0.0f);
+            for (int gi0 = g0; gi0 < g1; gi0 += kScaleRing) {
 #pragma unroll
                 for (int j = 0; j < kScaleRing; ++j) {
                     const int gi = gi0 + j;
-                    if (gi >= g.G) break;
+                    if (gi >= g1) break;
                     const float sw = __half2float(swr[j]);
-                    if (un.rows && gi + kScaleRing < g.G) swr[j] = sc[size_t(gi + kScaleRing) * kTileRows];
+                    if (un.rows && gi + kScaleRing < g1) swr[j] = sc[size_t(gi - g0 + kScaleRing) * kTileRows];
                     const uint32_t b = gc % kAccBufs;
                     // every lane waits; the warp leaves together if any lane gave up (the
                     // TMEM accesses below are warp-collective)
@@ -361,7 +373,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
                     if (!__all_sync(0xffffffffu, ok)) goto epi_done;
                     tc_fence_after();
                     __half (*sat)[kEpiTokens] = S.sat[e];
-                    if (AG && gi % kSatGroups == 0) {
+                    if (AG && (gi - g0) % kSatGroups == 0) {
                         // group-wise activations: this warp's token scales for the next groups
                         __syncwarp();
                         for (int i = lane; i < kSatGroups * kEpiTokens; i += 32) {
@@ -380,7 +392,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
                         for (int hh = 0; hh < 2; ++hh) {
                             const int h = 2 * quarter + hh;                 // 8-column chunk
                             if constexpr (AG) {
-                                const uint4 sv = *reinterpret_cast<const uint4*>(&sat[gi % kSatGroups][h * 8]);
+                                const uint4 sv = *reinterpret_cast<const uint4*>(&sat[(gi - g0) % kSatGroups][h * 8]);
                                 const __half2* sh = reinterpret_cast<const __half2*>(&sv);
 #pragma unroll
                                 for (int c = 0; c < 4; ++c) {
@@ -430,6 +442,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
                 }
             }
             if (orig >= 0) {
+                // one split: Y; several: this split's fp32 sums, added in split order and
+                // scaled by the reduction kernel
+                float* part = a.S > 1 ? a.part + size_t(un.ks) * a.M * g.N : nullptr;
 #pragma unroll
                 for (int c = 0; c < kEpiTokens / 2; ++c) {
 #pragma unroll
@@ -437,8 +452,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
                         const int m = m0 + 2 * c + x;
                         if (m < a.M) {
                             const float v = x ? acc[c].y : acc[c].x;
-                            a.Y[int64_t(m) * a.ldy + orig] =
-                                __float2half_rn(AG ? v : __fmul_rn(v, __half2float(a.s_a[m])));
+                            if (part) part[int64_t(m) * g.N + orig] = v;
+                            else a.Y[int64_t(m) * a.ldy + orig] =
+                                     __float2half_rn(AG ? v : __fmul_rn(v, __half2float(a.s_a[m])));
                         }
                     }
                 }
@@ -456,15 +472,55 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
     }
 }
 
+// Y[m][n] = fp16(the splits' fp32 sums of (m, n), added in split order, x s_a[m]);
+// group-wise activation scales were applied per group.  Elementwise over M x N.
+__global__ void __launch_bounds__(256) split_reduce_kernel(const float* __restrict__ part, int S, int M, int N,
+                                                           const __half* __restrict__ s_a, int ag, __half* Y,
+                                                           int64_t ldy) {
+    const int64_t total = int64_t(M) * N;
+    for (int64_t i = int64_t(blockIdx.x) * 256 + threadIdx.x; i < total; i += int64_t(gridDim.x) * 256) {
+        const int m = int(i / N), n = int(i % N);
+        float v = part[i];
+        for (int k = 1; k < S; ++k) v = __fadd_rn(v, part[int64_t(k) * total + i]);
+        Y[int64_t(m) * ldy + n] = __float2half_rn(ag ? v : __fmul_rn(v, __half2float(s_a[m])));
+    }
+}
+
 }  // namespace
 
 size_t tc2_smem_bytes() { return sizeof(Smem) + 1024; }
 
+int tc2_stages(const mx_layout& L) { return (L.kblocks + KPS - 1) / KPS; }
+
+int tc2_auto_split(const mx_layout& L, int M, int clusters) {
+    const int units1 = ((L.t8 + L.t4 + 1) / 2) * ((M + BN - 1) / BN);
+    const int n_ss = tc2_stages(L);
+    if (M <= 0 || clusters <= 0 || units1 >= clusters || n_ss < 2) return 1;
+    // waves x stages per unit, smallest first; the split adds partial sums to write
+    // and read back, so a tie keeps fewer splits
+    int best = 1;
+    long best_t = long(n_ss);
+    for (int S = 2; S <= kTc2MaxSplit && S <= n_ss; ++S) {
+        const int per = (n_ss + S - 1) / S;
+        if ((n_ss + per - 1) / per != S) continue;            // no empty split
+        const long t = (long(units1) * S + clusters - 1) / clusters * per;
+        if (t < best_t) {
+            best_t = t;
+            best = S;
+        }
+    }
+    return best;
+}
+
+size_t tc2_split_bytes(const mx_layout& L, int M, int S) {
+    return S > 1 ? (size_t(S) * size_t(M) * size_t(L.N) * 4 + 255) & ~size_t(255) : 0;
+}
+
 // Served by the pair kernel: any M >= 1 (token tiles of 128; rows past M are
 // zero-filled by the copies and never stored).
 cudaError_t launch_gemm_tc2(const mx_layout& L, const void* blob, const int8_t* Aq, const uint16_t* s_a, int M,
-                            uint16_t* Y, int64_t ldy, int ag, int32_t* debug_partials, int32_t* status,
-                            uint64_t timeout_ns, int stall_test, cudaStream_t s) {
+                            uint16_t* Y, int64_t ldy, int ag, int S, float* part, int32_t* debug_partials,
+                            int32_t* status, uint64_t timeout_ns, int stall_test, cudaStream_t s) {
     if (M == 0) return cudaSuccess;
     cudaError_t e;
     EncodeTiledFn enc = encode_fn(&e);
@@ -502,7 +558,14 @@ cudaError_t launch_gemm_tc2(const mx_layout& L, const void* blob, const int8_t* 
     a.ldy = ldy;
     a.M = M;
     a.n_tt = (M + BN - 1) / BN;
-    a.n_units = ((L.t8 + L.t4 + 1) / 2) * a.n_tt;
+    // S splits of the stages (the last split may be shorter, none is empty)
+    const int n_ss = tc2_stages(L);
+    if (S < 1 || S > kTc2MaxSplit || (S > 1 && part == nullptr)) return cudaErrorInvalidValue;
+    S = std::min(S, n_ss);
+    a.ss_per = (n_ss + S - 1) / S;
+    a.S = (n_ss + a.ss_per - 1) / a.ss_per;
+    a.part = a.S > 1 ? part : nullptr;
+    a.n_units = ((L.t8 + L.t4 + 1) / 2) * a.S * a.n_tt;
     a.debug = debug_partials;
     a.status = status;
     a.timeout_ns = timeout_ns;
@@ -511,6 +574,10 @@ cudaError_t launch_gemm_tc2(const mx_layout& L, const void* blob, const int8_t* 
     auto k = debug_partials ? (ag ? gemm_tc2_kernel<true, true> : gemm_tc2_kernel<true, false>)
                             : (ag ? gemm_tc2_kernel<false, true> : gemm_tc2_kernel<false, false>);
     k<<<2 * pairs, kThreads, tc2_smem_bytes(), s>>>(map, a);
+    if ((e = cudaGetLastError()) != cudaSuccess || a.S == 1) return e;
+    const int64_t total = int64_t(M) * L.N;
+    const int blocks = int(std::min<int64_t>((total + 255) / 256, int64_t(sms[dev]) * 8));
+    split_reduce_kernel<<<blocks, 256, 0, s>>>(a.part, a.S, M, L.N, a.s_a, ag, a.Y, ldy);
     return cudaGetLastError();
 }
 

@@ -242,6 +242,36 @@ static int choose_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
     return 4;
 }
 
+// CTA pairs the device holds (148 SMs on a B200; that figure when no device answers)
+static int pair_count() {
+    static int pairs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return 74;
+    }
+    if (pairs[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 2) {
+            cudaGetLastError();
+            return 74;
+        }
+        pairs[dev] = n / 2;
+    }
+    return pairs[dev];
+}
+
+// K splits path 4 takes: the caller's, or the automatic choice (1 when the grid is full)
+static int pair_split(const mx_layout* L, int M, const mx_gemm_opts* opts) {
+    return opts && opts->split > 0 ? opts->split : mx::tc2_auto_split(*L, M, pair_count());
+}
+
+// scratch mx_gemm uses at M tokens: the fp32 split sums of path 4, else nothing
+static size_t gemm_ws_bytes(const mx_layout* L, int M, const mx_gemm_opts* opts) {
+    if (M <= 0 || choose_path(L, M, opts) != 4) return 0;
+    return mx::tc2_split_bytes(*L, M, pair_split(L, M, opts));
+}
+
 int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
     mx_status st = check_layout(L);
     if (st != MX_OK) return -int(st);
@@ -254,8 +284,8 @@ mx_status mx_gemm_workspace_size(const mx_layout* L, int M, const mx_gemm_opts* 
     if (st != MX_OK) return st;
     if (bytes == nullptr) return fail(MX_ERR_INVALID_ARG, "bytes is NULL");
     if (M < 0) return fail(MX_ERR_INVALID_ARG, "M=%d", M);
-    *bytes = 0;   // both paths run without scratch memory
-    (void)opts;
+    if (opts && opts->split < 0) return fail(MX_ERR_INVALID_ARG, "split=%d", opts->split);
+    *bytes = gemm_ws_bytes(L, M, opts);   // only split tensor-core runs use scratch
     return MX_OK;
 }
 
@@ -305,10 +335,34 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
         if (opts && opts->wait_timeout_us < 0) return fail(MX_ERR_INVALID_ARG, "wait_timeout_us < 0");
         const uint64_t timeout_ns =
             (opts && opts->wait_timeout_us > 0) ? uint64_t(opts->wait_timeout_us) * 1000u : 2000000000ull;
-        auto launch = path == 2 ? mx::launch_gemm_tc : mx::launch_gemm_tc2;
-        cudaError_t e = launch(*L, blob, Aq, s_a, M, Y, ldy, ag, opts ? opts->debug_partials : nullptr,
-                               opts ? opts->status : nullptr, timeout_ns, opts ? opts->test_stall : 0, s);
-        if (e != cudaSuccess) return cuda_fail(e, path == 2 ? "tensor-core GEMM launch" : "pair tensor-core GEMM launch");
+        cudaError_t e;
+        if (path == 2) {
+            e = mx::launch_gemm_tc(*L, blob, Aq, s_a, M, Y, ldy, ag, opts ? opts->debug_partials : nullptr,
+                                   opts ? opts->status : nullptr, timeout_ns, opts ? opts->test_stall : 0, s);
+            if (e != cudaSuccess) return cuda_fail(e, "tensor-core GEMM launch");
+            return MX_OK;
+        }
+        // K splits: the caller's (needs the workspace) or automatic (taken only when the
+        // workspace holds the split sums)
+        const bool asked = opts && opts->split > 0;
+        if (opts && (opts->split < 0 || opts->split > mx::kTc2MaxSplit))
+            return fail(MX_ERR_UNSUPPORTED, "split=%d: 1..%d on path 4", opts->split, mx::kTc2MaxSplit);
+        int S = pair_split(L, M, opts);
+        const size_t need = mx::tc2_split_bytes(*L, M, S);
+        if (S > 1 && (workspace == nullptr || ws_bytes < need)) {
+            if (asked)
+                return fail(MX_ERR_WORKSPACE, "split %d needs a workspace of %zu bytes, %zu given", S, need,
+                            workspace ? ws_bytes : size_t(0));
+            S = 1;
+        }
+        if (S > 1) {
+            if ((st = check_device_ptr(workspace, "workspace")) != MX_OK) return st;
+            if (!aligned16(workspace)) return fail(MX_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+        }
+        e = mx::launch_gemm_tc2(*L, blob, Aq, s_a, M, Y, ldy, ag, S, S > 1 ? static_cast<float*>(workspace) : nullptr,
+                                opts ? opts->debug_partials : nullptr, opts ? opts->status : nullptr, timeout_ns,
+                                opts ? opts->test_stall : 0, s);
+        if (e != cudaSuccess) return cuda_fail(e, "pair tensor-core GEMM launch");
         return MX_OK;
     }
     return fail(MX_ERR_INVALID_ARG, "unknown GEMM path %d", path);
@@ -319,6 +373,20 @@ namespace {
 size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
 
 int x_bytes(mx_dtype xdt) { return xdt == MX_F16 ? 2 : 4; }
+
+bool linear_fused(const mx_layout* L, int M, mx_dtype xdt, const mx_gemm_opts* opts);
+
+// mx_linear's scratch: Aq | s_a | (256-byte aligned) the GEMM's own scratch when
+// with_gemm; 0 when one kernel does the whole step
+size_t linear_aq_sa_bytes(const mx_layout* L, int M, const mx_gemm_opts* opts) {
+    return align16(size_t(M) * L->K) + align16(size_t(2) * M * scales_per_token(L, opts));
+}
+size_t linear_ws_bytes(const mx_layout* L, int M, mx_dtype xdt, const mx_gemm_opts* opts, bool with_gemm) {
+    if (M == 0 || linear_fused(L, M, xdt, opts)) return 0;
+    const size_t base = linear_aq_sa_bytes(L, M, opts);
+    const size_t g = with_gemm ? gemm_ws_bytes(L, M, opts) : 0;
+    return g ? ((base + 255) & ~size_t(255)) + g : base;
+}
 
 bool linear_fused(const mx_layout* L, int M, mx_dtype xdt, const mx_gemm_opts* opts) {
     const int path = choose_path(L, M, opts);
@@ -350,8 +418,7 @@ mx_status mx_linear_workspace_size(const mx_layout* L, int M, mx_dtype xdtype, c
     if (M < 0) return fail(MX_ERR_INVALID_ARG, "M=%d", M);
     if (xdtype != MX_F32 && xdtype != MX_F16) return fail(MX_ERR_INVALID_ARG, "bad xdtype %d", int(xdtype));
     if ((st = check_act_group(L, opts)) != MX_OK) return st;
-    *bytes = (M == 0 || linear_fused(L, M, xdtype, opts)) ? 0
-             : align16(size_t(M) * L->K) + align16(size_t(2) * M * scales_per_token(L, opts));
+    *bytes = linear_ws_bytes(L, M, xdtype, opts, true);
     return MX_OK;
 }
 
@@ -395,7 +462,7 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
         if (e != cudaSuccess) return cuda_fail(e, "fused decode GEMM launch");
         return MX_OK;
     }
-    const size_t need = align16(size_t(M) * L->K) + align16(size_t(2) * M * scales_per_token(L, opts));
+    const size_t need = linear_aq_sa_bytes(L, M, opts);
     if (workspace == nullptr || ws_bytes < need)
         return fail(MX_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace ? ws_bytes : size_t(0));
     if ((st = check_device_ptr(workspace, "workspace")) != MX_OK) return st;
@@ -403,7 +470,10 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
     int8_t* Aq = static_cast<int8_t*>(workspace);
     uint16_t* s_a = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + align16(size_t(M) * L->K));
     if ((st = mx_quant_act_grouped(X, xdtype, M, L->K, ldx, ag, Aq, s_a, stream)) != MX_OK) return st;
-    return mx_gemm(L, blob, Aq, s_a, M, Y, ldy, nullptr, 0, opts, stream);
+    // the rest of the workspace (from a 256-byte boundary) is the GEMM's scratch
+    const size_t off = (need + 255) & ~size_t(255);
+    void* gws = ws_bytes > off ? static_cast<uint8_t*>(workspace) + off : nullptr;
+    return mx_gemm(L, blob, Aq, s_a, M, Y, ldy, gws, gws ? ws_bytes - off : 0, opts, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -451,6 +521,9 @@ mx_status mx_linear_noalloc(const mx_layout* L, const void* blob, const void* X,
     size_t need = 0;
     mx_status st = mx_linear_workspace_size(L, M, xdtype, opts, &need);
     if (st != MX_OK) return st;
+    // the limit holds for Aq and s_a; split sums of the tensor-core path use the rest of
+    // the array when they fit, else the GEMM runs unsplit
+    need = linear_ws_bytes(L, M, xdtype, opts, false);
     if (need > MX_NOALLOC_SCRATCH_BYTES)
         return fail(MX_ERR_WORKSPACE, "%zu bytes of scratch needed, the fixed array holds %u", need,
                     MX_NOALLOC_SCRATCH_BYTES);

@@ -208,10 +208,16 @@ cudaError_t launch_gemm_tc(const mx_layout& L, const void* blob, const int8_t* A
                            int32_t* debug_partials, int32_t* status, uint64_t timeout_ns,
                            int stall_test, cudaStream_t s);
 
-// the same GEMM on CTA pairs (cta_group::2): 256 weight rows x 192 tokens per tile
+// the same GEMM on CTA pairs (cta_group::2): 256 weight rows x 128 tokens per tile.
+// With S > 1 the stages are split S ways over more units; each split writes fp32
+// sums to part [S][M][N] and a second kernel adds them in split order into Y.
+constexpr int kTc2MaxSplit = 8;
+int tc2_stages(const mx_layout& L);                            // stages of two k-blocks
+int tc2_auto_split(const mx_layout& L, int M, int clusters);   // 1 when the grid is full
+size_t tc2_split_bytes(const mx_layout& L, int M, int S);      // part's bytes (0 for S = 1)
 cudaError_t launch_gemm_tc2(const mx_layout& L, const void* blob, const int8_t* Aq,
-                            const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy, int ag,
-                            int32_t* debug_partials, int32_t* status, uint64_t timeout_ns,
-                            int stall_test, cudaStream_t s);
+                            const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy, int ag, int S,
+                            float* part, int32_t* debug_partials, int32_t* status,
+                            uint64_t timeout_ns, int stall_test, cudaStream_t s);
 
 }  // namespace mx

@@ -119,10 +119,18 @@ def test_host_argument_checks_before_any_launch(lib):
     assert n.value == 0
 
 
-def test_paths_need_no_workspace_and_dispatch_on_m(lib):
+def test_gemm_workspace_and_dispatch_on_m(lib):
     L = mx.mx_layout_init(4096, 4096, 128, 410)
-    for M in (1, 16, 17, 2048):
+    for M in (1, 16, 2048):
         assert mx.mx_gemm_workspace_size(L, M) == 0
+    # 33 row tiles = 17 CTA pairs: one token tile leaves pairs idle, so path 4 splits K
+    # and sums the splits in a workspace; 16 token tiles fill the grid unsplit
+    n17 = mx.mx_gemm_workspace_size(L, 17)
+    assert n17 > 0 and n17 % (17 * 4096 * 4) == 0 and n17 // (17 * 4096 * 4) in range(2, 9)
+    a256 = lambda v: (v + 255) // 256 * 256
+    assert mx.mx_gemm_workspace_size(L, 17, split=3) == a256(3 * 17 * 4096 * 4)
+    assert mx.mx_gemm_workspace_size(L, 17, path=mx.PATH_TENSOR) == 0     # the one-CTA kernel
+    assert mx.mx_gemm_workspace_size(L, 17, split=1) == 0
     assert mx.mx_gemm_select_path(L, 1) == mx.PATH_ROWS          # short K, M <= 4, one wave
     assert mx.mx_gemm_select_path(L, 4) == mx.PATH_ROWS
     assert mx.mx_gemm_select_path(L, 5) == mx.PATH_SPLITK
@@ -147,10 +155,14 @@ def test_linear_workspace_follows_the_fused_decode_rule(lib):
         assert mx.mx_linear_workspace_size(L, M, torch.float16) == 0
         assert mx.mx_linear_workspace_size(L, M, torch.float32) == 0
     assert mx.mx_linear_workspace_size(L, 0, torch.float16) == 0
-    # more tokens, the tensor-core path, or a forced path: Aq + s_a, 16-byte rounded
+    # more tokens, the tensor-core path, or a forced path: Aq + s_a, 16-byte rounded, then
+    # (from a 256-byte boundary) the GEMM's own workspace when it splits K
     a16 = lambda v: (v + 15) // 16 * 16
+    a256 = lambda v: (v + 255) // 256 * 256
     for M in (5, 16, 17, 2048):
-        assert mx.mx_linear_workspace_size(L, M, torch.float16) == a16(M * 4096) + a16(2 * M)
+        g = mx.mx_gemm_workspace_size(L, M)
+        base = a16(M * 4096) + a16(2 * M)
+        assert mx.mx_linear_workspace_size(L, M, torch.float16) == (a256(base) + g if g else base)
     assert mx.mx_linear_workspace_size(L, 1, torch.float16, path=mx.PATH_TENSOR) == 4096 + 16
     # 4 fp32 rows of 8192 columns exceed the 64 KB the fused kernel stages
     Lw = mx.mx_layout_init(1024, 8192, 128, 102)

@@ -57,7 +57,9 @@ def run_grouped(orc, M, K, N, g, path=0, split=0, seed=0):
     Aq, sa, Aq_o, sa_o = check_quant_grouped(orc, lay.X, g)
     Y = torch.full((M, N), float("nan"), dtype=torch.float16, device=dev())
     P = torch.zeros((M, N, L.G), dtype=torch.int32, device=dev())
-    mx.mx_gemm(L, blob, Aq, sa, Y, path=path, split=split, debug_partials=P, act_group=g)
+    ws = torch.empty(max(16, mx.mx_gemm_workspace_size(L, M, path=path, split=split)), dtype=torch.uint8,
+                     device=dev())
+    mx.mx_gemm(L, blob, Aq, sa, Y, workspace=ws, path=path, split=split, debug_partials=P, act_group=g)
     torch.cuda.synchronize()
     c = orc.pack(lay.W, lay.is8, g)
     P_o, _ = orc.partials(Aq_o, c)
@@ -103,7 +105,9 @@ def test_linear_grouped_matches_two_calls(orc, M, split, xdtype):
     assert_y_close(Y.cpu().numpy(), orc.gemm(Aq_o, sa_o, c, act_group=128)[1])
     Aq, sa = gpu_quant_grouped(Xo.astype(np.float16) if xdtype == torch.float16 else Xo, 128)
     Y2 = torch.empty_like(Y)
-    mx.mx_gemm(L, blob, Aq, sa, Y2, split=split, act_group=128)
+    # the GEMM's own workspace, as mx_linear gives it (a K split of the tensor cores)
+    gws = torch.empty(max(16, mx.mx_gemm_workspace_size(L, M, split=split)), dtype=torch.uint8, device=dev())
+    mx.mx_gemm(L, blob, Aq, sa, Y2, workspace=gws, split=split, act_group=128)
     torch.cuda.synchronize()
     assert torch.equal(Y, Y2)
 

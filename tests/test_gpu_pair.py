@@ -1,13 +1,14 @@
 """Parity of the tensor-core path on CTA pairs (path 4: cta_group::2, 256 weight
-rows x 192 tokens per tile) against the oracle.
+rows x 128 tokens per tile) against the oracle.
 
 Partials P[m, n, g] are compared bit for bit, Y within the tolerance of the
-other paths.  The pair kernel does the same arithmetic in the same order as the
-one-CTA tensor-core kernel, so their Y must be identical too.  Shapes cover an
-odd number of row tiles (the last pair has a CTA without rows), token counts on
-both sides of the 96-token halves and the 192-token tiles, both group sizes,
-all-4-bit and all-8-bit layers, group-wise activation scales, and the bounded
-waits.
+other paths.  Unsplit, the pair kernel does the same arithmetic in the same order
+as the one-CTA tensor-core kernel, so their Y must be identical too.  Shapes cover
+an odd number of row tiles (the last pair has a CTA without rows), token counts on
+both sides of the 64-token halves and the 128-token tiles, both group sizes,
+all-4-bit and all-8-bit layers, group-wise activation scales, splits of K (even and
+uneven, through mx_gemm and mx_linear, and the workspace they need), and the
+bounded waits.
 """
 import numpy as np
 import pytest
@@ -30,7 +31,7 @@ def _layer(rng, M, N, K, n8, outliers=4):
     return X, W, is8
 
 
-@pytest.mark.parametrize("M", [1, 95, 96, 97, 191, 192, 193, 400])
+@pytest.mark.parametrize("M", [1, 63, 64, 65, 127, 128, 129, 400])
 @pytest.mark.parametrize("g", [64, 128])
 def test_pair_token_counts(orc, M, g):
     # N = 430 with 37 8-bit rows: one 8-bit and four 4-bit row tiles, so the last
@@ -64,7 +65,7 @@ def test_pair_equals_one_cta_kernel(orc):
     Aq, sa = gpu_quant(X)
     L, blob = gpu_pack(W, is8, 128)
     Y2, P2, _ = gpu_gemm(L, blob, Aq, sa, path=mx.PATH_TENSOR, debug=True)
-    Y4, P4, _ = gpu_gemm(L, blob, Aq, sa, path=mx.PATH_PAIR, debug=True)
+    Y4, P4, _ = gpu_gemm(L, blob, Aq, sa, path=mx.PATH_PAIR, split=1, debug=True)   # unsplit
     assert torch.equal(P2, P4)
     assert torch.equal(Y2.view(torch.int16), Y4.view(torch.int16))
 
@@ -114,3 +115,62 @@ def test_pair_wait_timeout_sets_status_and_context_survives(orc):
     mx.mx_gemm(L, blob, Aq, sa, Y, path=mx.PATH_PAIR, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
+
+
+# ------------------------------------------------------------------ K split over CTA pairs
+@pytest.mark.parametrize("M", [1, 100, 300])
+@pytest.mark.parametrize("split", [2, 3, 5])
+def test_pair_split_matches_oracle(orc, M, split):
+    # K = 1152: nine k-blocks in five stages, so the splits are uneven
+    rng = np.random.default_rng(M + 31 * split)
+    X, W, is8 = _layer(rng, M, 430, 1152, 37)
+    Y = run_and_check(orc, X, W, is8, 128, path=mx.PATH_PAIR, split=split)
+    # the splits are added in a fixed order: the same Y every time
+    Aq, sa = gpu_quant(X)
+    L, blob = gpu_pack(W, is8, 128)
+    Y2, _, _ = gpu_gemm(L, blob, Aq, sa, path=mx.PATH_PAIR, split=split)
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+
+
+def test_pair_split_group_wise_and_g64(orc):
+    run_grouped(orc, 40, 1024, 430, 64, path=mx.PATH_PAIR, split=3, seed=5)
+
+
+def test_pair_split_workspace_rules(orc):
+    rng = np.random.default_rng(4)
+    M, N, K = 64, 430, 1024
+    X, W, is8 = _layer(rng, M, N, K, 37)
+    Aq, sa = gpu_quant(X)
+    L, blob = gpu_pack(W, is8, 128)
+    Y = torch.zeros((M, N), dtype=torch.float16, device=dev())
+    with pytest.raises(mx.MXError) as e:            # an asked-for split needs its workspace
+        mx.mx_gemm(L, blob, Aq, sa, Y, path=mx.PATH_PAIR, split=2)
+    assert e.value.status == 7
+    # an automatic split without a workspace runs unsplit: bit-identical to split=1
+    assert mx.mx_gemm_workspace_size(L, M) > 0
+    mx.mx_gemm(L, blob, Aq, sa, Y)
+    Y1, _, _ = gpu_gemm(L, blob, Aq, sa, path=mx.PATH_PAIR, split=1)
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), Y1.view(torch.int16))
+    # with it, the automatic split agrees with the oracle
+    Ya, _, _ = gpu_gemm(L, blob, Aq, sa)
+    Aq_o, sa_o = orc.quant_act(X.astype(np.float32))
+    assert_y_close(Ya.cpu().numpy(), orc.gemm(Aq_o, sa_o, orc.pack(W, is8, 128))[1])
+
+
+def test_pair_split_through_mx_linear(orc):
+    # the layer call sizes its workspace with the split sums and gives the two-call result
+    rng = np.random.default_rng(8)
+    M, N, K = 48, 430, 2048
+    X, W, is8 = _layer(rng, M, N, K, 37)
+    L, blob = gpu_pack(W, is8, 128)
+    Xd = torch.from_numpy(X).to(dev())
+    n = mx.mx_linear_workspace_size(L, M, Xd.dtype)
+    assert n > mx.mx_linear_workspace_size(L, M, Xd.dtype, split=1)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev())
+    Y = torch.empty((M, N), dtype=torch.float16, device=dev())
+    mx.mx_linear(L, blob, Xd, Y, workspace=ws)
+    Aq, sa = gpu_quant(X)
+    Y2, _, _ = gpu_gemm(L, blob, Aq, sa)
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))

@@ -22,9 +22,11 @@ def _built():
 
 
 def with_workspace(L, blob, Xd):
+    # a caller workspace of the fixed array's size: mx_linear then takes the same
+    # decisions (a K split of the tensor cores only when its sums fit) as the array
     Y = torch.empty((Xd.shape[0], L.N), dtype=torch.float16, device=dev())
     n = mx.mx_linear_workspace_size(L, Xd.shape[0], Xd.dtype)
-    ws = torch.empty(n, dtype=torch.uint8, device=dev()) if n else None
+    ws = torch.empty(mx.NOALLOC_SCRATCH_BYTES, dtype=torch.uint8, device=dev()) if n else None
     mx.mx_linear(L, blob, Xd, Y, workspace=ws)
     return Y
 
@@ -71,7 +73,8 @@ def test_largest_fit_and_first_refusal():
     lay = inputs.llama_layer(1, K, 256, seed=104)
     L, blob = gpu_pack(lay.W, lay.is8, 128)
     cap = mx.NOALLOC_SCRATCH_BYTES
-    M_fit = max(m for m in range(cap // K - 2, cap // K + 1) if mx.mx_linear_workspace_size(L, m) <= cap)
+    # the limit is on Aq and s_a (the unsplit scratch)
+    M_fit = max(m for m in range(cap // K - 2, cap // K + 1) if mx.mx_linear_workspace_size(L, m, split=1) <= cap)
     rng = np.random.default_rng(105)
     Xd = to_dev(inputs.activations(rng, M_fit + 1, K, 41))
     Y = nan_out(L, M_fit)
