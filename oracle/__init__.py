@@ -61,6 +61,8 @@ def _load():
     lib.mxo_partials.restype = ctypes.c_int64
     lib.mxo_gemm.argtypes = [P, P, I, I, I, I, I, P, I, P, P, P, P, P, P, P, ctypes.c_long, P, P]
     lib.mxo_gemm.restype = I
+    lib.mxo_saliency.argtypes = [P, I, P, I, I, I, I, P]
+    lib.mxo_saliency.restype = I
     _lib = lib
     return lib
 
@@ -232,3 +234,28 @@ def dequant_weights(c: Canonical) -> np.ndarray:
             w = c.codes4[r].astype(np.float64) - np.repeat(c.zeros4[r].astype(np.float64), g)
             W[n] = w * np.repeat(s4[r], g)
     return W
+
+
+def saliency(W, G, group: int) -> np.ndarray:
+    """Channel saliency of the global precision search (MixLLM section 3.2, Eq. 4
+    with one gradient batch, Algorithm 1 lines 3-6): per output row,
+    S = |S1 + S1^2/2| with S1 = sum_k G * (dequant(quantize4(W)) - W), in fp64."""
+    W = np.ascontiguousarray(_f32(W))
+    G = np.ascontiguousarray(_f32(G))
+    N, K = W.shape
+    assert G.shape == (N, K)
+    S = np.zeros(N, np.float64)
+    if _load().mxo_saliency(_p(W), K, _p(G), K, N, K, group, _p(S)) != 0:
+        raise ValueError("bad saliency arguments")
+    return S
+
+
+def select_top(scores, n_top: int) -> np.ndarray:
+    """Algorithm 1 lines 9-10 over the scores of all layers concatenated: the
+    n_top largest are the 8-bit channels (reading P8: ties go to the lower global
+    index, i.e. the earlier layer, then the lower row).  Returns a uint8 mask."""
+    scores = np.asarray(scores)
+    order = np.lexsort((np.arange(scores.size), -scores.astype(np.float64)))
+    mask = np.zeros(scores.size, np.uint8)
+    mask[order[:max(0, min(n_top, scores.size))]] = 1
+    return mask

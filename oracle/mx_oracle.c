@@ -323,3 +323,39 @@ int mxo_gemm(const int8_t *Aq, const uint16_t *s_a, int act_group, int M, int K,
     free(inv);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Channel saliency of the global precision search (MixLLM section 3.2,     */
+/* Eq. 4 with the gradient of one calibration batch, as Algorithm 1 uses    */
+/* it): per output row n of one layer,                                     */
+/*   dW = dequant(quantize(W)) - W   (quantize: the 4-bit asymmetric group  */
+/*        quantizer above, the precision a row falls to when it is not      */
+/*        selected; reading R13),                                           */
+/*   S1 = sum_k G[n,k] * dW[n,k],  S[n] = | S1 + S1^2 / 2 |.                */
+/* W, G: [N][ld] fp32.  S: [N] fp64.  All arithmetic after the codes is     */
+/* fp64.  Returns 0, or -1 on bad arguments.                                */
+/* ------------------------------------------------------------------------ */
+int mxo_saliency(const float *W, int ldw, const float *G, int ldg, int N, int K, int group, double *S)
+{
+    if (N < 0 || K <= 0 || group <= 0 || K % group != 0 || ldw < K || ldg < K) return -1;
+    uint8_t *q = (uint8_t *)malloc((size_t)group);
+    if (!q) return -1;
+    for (int n = 0; n < N; ++n) {
+        double s1 = 0.0;
+        for (int g0 = 0; g0 < K; g0 += group) {
+            const float *w = W + (size_t)n * ldw + g0;
+            const float *gr = G + (size_t)n * ldg + g0;
+            uint8_t z;
+            uint16_t sb;
+            mxo_quant_asym4(w, group, q, &z, &sb);
+            const double s = mxo_fp16_value(sb);
+            for (int k = 0; k < group; ++k) {
+                const double dq = ((double)q[k] - (double)z) * s;   /* dequantized weight */
+                s1 += (double)gr[k] * (dq - (double)w[k]);
+            }
+        }
+        S[n] = fabs(s1 + 0.5 * s1 * s1);
+    }
+    free(q);
+    return 0;
+}

@@ -367,3 +367,87 @@ def test_gemm_group_activations(orc):
     err_group = np.linalg.norm(Xd - X)
     err_token = np.linalg.norm(Xt - X)
     assert err_group < err_token
+
+
+# --------------------------------------------------------------- global saliency (NEXT-2)
+def _asym4_grid_rows(rng, N, K, g):
+    """W whose every group is exactly on its 4-bit asymmetric grid (codes 0 and 15 present)."""
+    W = np.zeros((N, K))
+    for n in range(N):
+        for gi in range(K // g):
+            s = float(np.float16(10.0 ** rng.uniform(-3, -1)))
+            z = int(rng.integers(0, 16))
+            q = rng.integers(0, 16, g)
+            q[:2] = (0, 15)
+            rng.shuffle(q)
+            W[n, gi * g:(gi + 1) * g] = (q - z) * s
+    return W.astype(np.float32)
+
+
+def test_saliency_vanishes_on_the_4bit_grid(orc):
+    # quantize() is the 4-bit asymmetric quantizer: on its grid dW = 0, whatever G is.
+    # An 8-bit (or any other) quantizer would not reproduce these values exactly.
+    rng = np.random.default_rng(40)
+    W = _asym4_grid_rows(rng, 12, 512, 128)
+    G = rng.standard_normal(W.shape).astype(np.float32) * 100.0
+    assert np.array_equal(orc.saliency(W, G, 128), np.zeros(12))
+    W8 = (rng.integers(-127, 128, (12, 512)) * 0.01).astype(np.float32)   # on an 8-bit grid only
+    assert (orc.saliency(W8, G, 128) > 0).any()
+
+
+def test_saliency_unit_gradient_is_one_element_error(orc):
+    # G = e_k in row n: S1 is that element's quantization error d, S = |d + d^2/2|
+    rng = np.random.default_rng(41)
+    W = (rng.standard_normal((3, 256)) * 0.05).astype(np.float32)
+    for n, k in ((0, 5), (1, 200), (2, 129)):
+        G = np.zeros_like(W)
+        G[n, k] = 1.0
+        g0 = (k // 128) * 128
+        q, z, sb = orc.quant_asym4(W[n, g0:g0 + 128])
+        d = (float(q[k - g0]) - z) * orc.fp16_value(sb) - float(W[n, k])
+        S = orc.saliency(W, G, 128)
+        assert S[n] == pytest.approx(abs(d + 0.5 * d * d), rel=1e-15, abs=0)
+        assert np.array_equal(np.delete(S, n), np.zeros(2))
+
+
+def test_saliency_first_and_second_order_terms(orc):
+    # flipping G flips S1: S(G) = |S1 + S1^2/2|, S(-G) = |-S1 + S1^2/2|.  For 0 < |S1| < 2
+    # both are S1-linear plus or minus the same square: their half-sum is |S1| and their
+    # difference is S1^2 (a dropped or mis-scaled second-order term fails this)
+    rng = np.random.default_rng(42)
+    W = (rng.standard_normal((8, 384)) * 0.02).astype(np.float32)
+    G = (rng.standard_normal(W.shape) * 10.0).astype(np.float32)
+    Sp, Sm = orc.saliency(W, G, 128), orc.saliency(W, -G, 128)
+    s1 = 0.5 * (Sp + Sm)
+    assert (s1 > 1e-3).all() and (s1 < 2).all()
+    assert np.allclose(np.abs(Sp - Sm), s1 * s1, rtol=1e-9, atol=0)
+    # and S1 is linear in G: doubling G doubles |S1|
+    S2p, S2m = orc.saliency(W, 2 * G, 128), orc.saliency(W, -2 * G, 128)
+    assert np.allclose(0.5 * (S2p + S2m), 2 * s1, rtol=1e-9, atol=0)
+
+
+def test_saliency_group_sizes_and_zero_gradient(orc):
+    rng = np.random.default_rng(43)
+    W = (rng.standard_normal((5, 256)) * 0.02).astype(np.float32)
+    assert np.array_equal(orc.saliency(W, np.zeros_like(W), 64), np.zeros(5))
+    with pytest.raises(ValueError):
+        orc.saliency(W[:, :200], np.zeros((5, 200), np.float32), 128)   # K not a multiple of g
+
+
+def test_select_top_brute_force(orc):
+    # the n_top largest scores, ties to the lower index: against an exhaustive check of
+    # every index subset on tiny inputs
+    import itertools
+    rng = np.random.default_rng(44)
+    for _ in range(200):
+        n = int(rng.integers(1, 8))
+        s = rng.integers(0, 4, n).astype(np.float64)        # many ties
+        k = int(rng.integers(0, n + 1))
+        best = None
+        for sub in itertools.combinations(range(n), k):      # lexicographically first optimum
+            key = (sum(s[list(sub)]), [-i for i in sub])
+            if best is None or key > best[0]:
+                best = (key, sub)
+        want = np.zeros(n, np.uint8)
+        want[list(best[1])] = 1
+        assert np.array_equal(orc.select_top(s, k), want), (s, k)
