@@ -69,6 +69,9 @@ def parse():
     p.add_argument("--sweep", action="store_true",
                    help="the K = N = 8192 sweep over 8-bit row fraction, M and group size: one JSON "
                         "line per (fraction, group, M, path) and the GEMV / tensor-core crossover")
+    p.add_argument("--search", action="store_true",
+                   help="the global precision search: channel saliency of one Llama-3-8B decoder "
+                        "layer's seven linears, then the top-10%% choice over all 32 layers' rows")
     a = p.parse_args()
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -344,6 +347,97 @@ def run_sweep(a):
     print(json.dumps({"sweep_crossover": summary}), flush=True)
 
 
+# ------------------------------------------------------------------ precision search
+SEARCH_LINEARS = {"q": (4096, 4096), "k": (4096, 1024), "v": (4096, 1024), "o": (4096, 4096),
+                  "gate": (4096, 14336), "up": (4096, 14336), "down": (14336, 4096)}   # (K, N)
+SEARCH_LAYERS = 32
+
+
+def run_search(a):
+    """Times the two steps of the precision search on Llama-3-8B shapes.  Saliency: one
+    decoder layer's seven linears, W and G fp16 on the device (W ~ N(0, 0.02), G ~ N(0, 1e-3)
+    times a log-normal row scale, from a seeded device generator), 872 MB per pass, so
+    larger than L2; HBM-bound: its algorithmic bytes are N K (2 + 2) + 4 N per linear.
+    Selection: the 10% largest of all 32 layers' 1,376,256 row scores (fp32).  The oracle's
+    saliency is timed beside it on a bounded sample of rows of the gate projection."""
+    import torch
+    from mixed_precision_quantized_mx_b200 import binding as mx
+    from mixed_precision_quantized_mx_b200 import build as mxbuild
+    from mixed_precision_quantized_mx_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    mxbuild.build()
+    peaks = load_peaks()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(a.seed)
+    s = torch.cuda.Stream(dev)
+    lin = []
+    for name, (K, N) in SEARCH_LINEARS.items():
+        W = (torch.randn((N, K), generator=gen, device=dev) * 0.02).half()
+        rs = torch.exp(torch.randn((N, 1), generator=gen, device=dev))
+        G = (torch.randn((N, K), generator=gen, device=dev) * 1e-3 * rs).half()
+        lin.append((name, W, G, torch.empty(N, dtype=torch.float32, device=dev)))
+    nbytes = sum(W.numel() * 2 + G.numel() * 2 + 4 * S.numel() for _, W, G, S in lin)
+
+    def sal_pass():
+        for _, W, G, S in lin:
+            mx.mx_saliency(W, G, a.group, S, stream=s)
+
+    with torch.cuda.stream(s):
+        for _ in range(a.warmup):
+            sal_pass()
+    torch.cuda.synchronize()
+    steps = a.steps or 20
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(s)
+    for _ in range(steps):
+        sal_pass()
+    ev[1].record(s)
+    torch.cuda.synchronize()
+    us_sal = ev[0].elapsed_time(ev[1]) * 1e3 / steps
+    gbs = nbytes / us_sal / 1e3
+    # the global choice over all layers' scores (the layer's own scores, perturbed per layer)
+    S_one = torch.cat([S for *_, S in lin])
+    S_all = torch.cat([S_one * (1 + 1e-3 * torch.rand(S_one.shape, generator=gen, device=dev))
+                       for _ in range(SEARCH_LAYERS)])
+    n = S_all.numel()
+    n_top = inputs.n8_for(n, 0.10)
+    is8 = torch.empty(n, dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(s):
+        for _ in range(a.warmup):
+            mx.mx_select_top(S_all, n_top, is8, stream=s)
+    torch.cuda.synchronize()
+    ev[0].record(s)
+    for _ in range(steps):
+        mx.mx_select_top(S_all, n_top, is8, stream=s)
+    ev[1].record(s)
+    torch.cuda.synchronize()
+    us_sel = ev[0].elapsed_time(ev[1]) * 1e3 / steps
+    assert int(is8.sum().item()) == n_top
+    line = {"metric": "saliency_bandwidth", "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1,
+            "steps": steps, "warmup": a.warmup, "us_per_layer_saliency": round(us_sal, 2),
+            "select_rows": n, "select_top": n_top, "us_select": round(us_sel, 2),
+            "dtype": "f16 in, f64 sums", "data": "synthetic",
+            "config": {"workload": "llama3-8b decoder layer, 7 linears, group %d" % a.group,
+                       "bytes_per_pass": nbytes, "l2": "inputs 872 MB > L2"},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None}}
+    if not a.no_cpu_baseline:
+        import oracle
+        rng = np.random.default_rng(a.seed)
+        rows = 256
+        Wc = inputs.weights(rng, rows, 4096)
+        Gc = inputs.gradients(rng, rows, 4096)
+        t0 = time.perf_counter()
+        oracle.saliency(Wc, Gc, a.group)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": round(rows * 4096 * 4 / dt / 1e9, 3), "unit": "GB/s", "cores": 1,
+                                "kind": "oracle", "sample": "%d rows of the gate projection (K=4096), bytes counted "
+                                                           "as fp16 W and G like the GPU line" % rows}
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ main arm
 def main():
     a = parse()
@@ -351,6 +445,8 @@ def main():
         return run_reference(a)
     if a.sweep:
         return run_sweep(a)
+    if a.search:
+        return run_search(a)
 
     import torch
     import torch.distributed as dist

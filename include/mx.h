@@ -308,6 +308,44 @@ mx_status mx_linear_noalloc(const mx_layout* L, const void* blob, const void* X,
                             void* stream);
 
 /*
+ * mx_saliency -- channel saliency of the global precision search (MixLLM
+ * section 3.2: Eq. 4 with the gradient of one calibration batch, as Algorithm 1
+ * scores a layer) for every output row of one layer:
+ *   dW = dequant(quantize(W)) - W, with the 4-bit asymmetric group quantizer of
+ *        mx_pack_weights (the precision a row drops to when it is not chosen),
+ *   S1 = sum_k G[n,k] * dW[n,k]  (summed in fp64),
+ *   S[n] = |S1 + S1^2 / 2|, rounded to fp32 once.
+ *   W, G   device [N][ld] row-major, fp32 or fp16 each (wdtype, gdtype);
+ *          G is the loss gradient with respect to W
+ *   N, K   rows and columns; group 64 or 128 dividing K
+ *   S      device fp32 [N], written
+ * The method has no other use for G; the scores feed mx_select_top.  Returns
+ * MX_ERR_INVALID_ARG / MX_ERR_UNSUPPORTED on bad arguments before any launch.
+ * Asynchronous in `stream`.
+ */
+mx_status mx_saliency(const void* W, mx_dtype wdtype, int64_t ldw, const void* G, mx_dtype gdtype, int64_t ldg,
+                      int N, int K, int group, float* S, void* stream);
+
+/* Bytes of device workspace mx_select_top needs (a fixed few hundred bytes). */
+mx_status mx_select_top_workspace_size(int64_t n, size_t* bytes);
+
+/*
+ * mx_select_top -- the global choice of Algorithm 1: over the
+ * scores S of all layers' rows, concatenated in layer order (n rows in all),
+ * is8[i] = 1 for the n_top largest scores and 0 for the rest; ties go to the
+ * lower index (the earlier layer, then the lower row).  Exact: a radix select
+ * over (score bits, complemented index) keys, deterministic.  The slice of is8
+ * of each layer is that layer's mask for mx_pack_weights.
+ *   S          device fp32 [n], finite and >= 0 (as mx_saliency writes them)
+ *   n, n_top   0 <= n_top <= n < 2^32
+ *   is8        device uint8 [n], written
+ *   workspace  device, 16-byte aligned, mx_select_top_workspace_size bytes
+ * Asynchronous in `stream`.
+ */
+mx_status mx_select_top(const float* S, int64_t n, int64_t n_top, uint8_t* is8, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/*
  * mx_copy_mapped -- copy `bytes` bytes from src to dst with a kernel, where each
  * of the two may be device memory of the current device or pinned host memory
  * (page-locked and mapped into the device's address space, as cudaHostAlloc

@@ -27,7 +27,8 @@ PATH_AUTO, PATH_SPLITK, PATH_TENSOR, PATH_ROWS, PATH_PAIR = 0, 1, 2, 3, 4
 EXPORTED = ("mx_version", "mx_last_error", "mx_layout_init", "mx_layout_from_header",
             "mx_pack_weights", "mx_quant_act", "mx_gemm_workspace_size", "mx_gemm_select_path",
             "mx_gemm", "mx_linear_workspace_size", "mx_linear", "mx_linear_noalloc",
-            "mx_quant_act_grouped", "mx_copy_mapped")
+            "mx_quant_act_grouped", "mx_copy_mapped", "mx_saliency", "mx_select_top_workspace_size",
+            "mx_select_top")
 
 
 class MXError(RuntimeError):
@@ -86,9 +87,13 @@ def lib() -> ctypes.CDLL:
     L.mx_linear_noalloc.argtypes = [ctypes.POINTER(Layout), P, P, I, I, I64, P, I64,
                                     ctypes.POINTER(GemmOpts), P]
     L.mx_copy_mapped.argtypes = [P, P, Z, P]
+    L.mx_saliency.argtypes = [P, I, I64, P, I, I64, I, I, I, P, P]
+    L.mx_select_top_workspace_size.argtypes = [I64, ctypes.POINTER(Z)]
+    L.mx_select_top.argtypes = [P, I64, I64, P, P, Z, P]
     for n in ("mx_layout_init", "mx_layout_from_header", "mx_pack_weights", "mx_quant_act",
               "mx_quant_act_grouped", "mx_gemm_workspace_size", "mx_gemm", "mx_linear_workspace_size", "mx_linear",
-              "mx_linear_noalloc", "mx_copy_mapped"):
+              "mx_linear_noalloc", "mx_copy_mapped", "mx_saliency", "mx_select_top_workspace_size",
+              "mx_select_top"):
         getattr(L, n).restype = I
     _lib = L
     return L
@@ -241,3 +246,30 @@ def mx_copy_mapped(dst: torch.Tensor, src: torch.Tensor, stream=None) -> None:
         if not t.is_cuda and not t.is_pinned():
             raise ValueError(f"mx_copy_mapped: {n} is pageable host memory (pin it first)")
     _check(lib().mx_copy_mapped(_ptr(dst), _ptr(src), dst.nbytes, _stream(stream)), "mx_copy_mapped")
+
+
+def mx_saliency(W: torch.Tensor, G: torch.Tensor, group: int, S: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """Per-row channel saliency of one layer (see mx.h); returns S (device fp32 [N])."""
+    assert W.dim() == 2 and W.stride(1) == 1 and G.shape == W.shape and G.stride(1) == 1
+    N, K = W.shape
+    if S is None:
+        S = torch.empty(N, dtype=torch.float32, device=W.device)
+    _check(lib().mx_saliency(_ptr(W), _dtype_code(W), W.stride(0), _ptr(G), _dtype_code(G), G.stride(0), N, K,
+                             group, _ptr(S), _stream(stream)), "mx_saliency")
+    return S
+
+
+def mx_select_top(S: torch.Tensor, n_top: int, is8: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The n_top largest of the concatenated scores, ties to the lower index (see mx.h);
+    returns the uint8 mask."""
+    assert S.dim() == 1 and S.dtype == torch.float32 and S.is_contiguous()
+    n = S.numel()
+    if is8 is None:
+        is8 = torch.empty(n, dtype=torch.uint8, device=S.device)
+    nb = ctypes.c_size_t(0)
+    _check(lib().mx_select_top_workspace_size(n, ctypes.byref(nb)), "mx_select_top_workspace_size")
+    ws = torch.empty(max(nb.value, 16), dtype=torch.uint8, device=S.device)
+    _check(lib().mx_select_top(_ptr(S), n, n_top, _ptr(is8), _ptr(ws), ws.numel(), _stream(stream)),
+           "mx_select_top")
+    return is8

@@ -104,6 +104,13 @@ size_t scales_per_token(const mx_layout* L, const mx_gemm_opts* opts) {
 
 namespace mx {
 
+// the precision search (saliency.cu)
+cudaError_t launch_saliency(const void* W, mx_dtype wdt, int64_t ldw, const void* G, mx_dtype gdt, int64_t ldg,
+                            int N, int K, int group, float* S, cudaStream_t s);
+size_t select_workspace_bytes();
+cudaError_t launch_select_top(const float* S, int64_t n, int64_t n_top, uint8_t* is8, void* workspace,
+                              cudaStream_t s);
+
 Geom make_geom(const mx_layout& L, const void* blob) {
     const uint8_t* b = static_cast<const uint8_t*>(blob);
     Geom g;
@@ -397,6 +404,47 @@ bool linear_fused(const mx_layout* L, int M, mx_dtype xdt, const mx_gemm_opts* o
 }
 
 }  // namespace
+
+mx_status mx_saliency(const void* W, mx_dtype wdtype, int64_t ldw, const void* G, mx_dtype gdtype, int64_t ldg,
+                      int N, int K, int group, float* S, void* stream) {
+    if (N < 0 || K <= 0) return fail(MX_ERR_INVALID_ARG, "N=%d K=%d", N, K);
+    if (group != 64 && group != 128) return fail(MX_ERR_UNSUPPORTED, "group=%d: 64 or 128", group);
+    if (K % group != 0) return fail(MX_ERR_INVALID_ARG, "K=%d is not a multiple of the group %d", K, group);
+    if (ldw < K || ldg < K) return fail(MX_ERR_INVALID_ARG, "ldw=%lld ldg=%lld < K=%d", (long long)ldw,
+                                        (long long)ldg, K);
+    for (mx_dtype t : {wdtype, gdtype})
+        if (t != MX_F32 && t != MX_F16) return fail(MX_ERR_INVALID_ARG, "bad dtype %d", int(t));
+    if (N == 0) return MX_OK;
+    mx_status st;
+    if ((st = check_device_ptr(W, "W")) != MX_OK) return st;
+    if ((st = check_device_ptr(G, "G")) != MX_OK) return st;
+    if ((st = check_device_ptr(S, "S")) != MX_OK) return st;
+    cudaError_t e = mx::launch_saliency(W, wdtype, ldw, G, gdtype, ldg, N, K, group, S, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MX_OK : cuda_fail(e, "saliency launch");
+}
+
+mx_status mx_select_top_workspace_size(int64_t n, size_t* bytes) {
+    if (bytes == nullptr) return fail(MX_ERR_INVALID_ARG, "bytes is NULL");
+    if (n < 0 || n > int64_t(0xFFFFFFFFu)) return fail(MX_ERR_INVALID_ARG, "n=%lld", (long long)n);
+    *bytes = mx::select_workspace_bytes();
+    return MX_OK;
+}
+
+mx_status mx_select_top(const float* S, int64_t n, int64_t n_top, uint8_t* is8, void* workspace, size_t ws_bytes,
+                        void* stream) {
+    if (n < 0 || n > int64_t(0xFFFFFFFFu)) return fail(MX_ERR_INVALID_ARG, "n=%lld", (long long)n);
+    if (n_top < 0 || n_top > n) return fail(MX_ERR_INVALID_ARG, "n_top=%lld of %lld", (long long)n_top, (long long)n);
+    if (n == 0) return MX_OK;
+    mx_status st;
+    if ((st = check_device_ptr(S, "S")) != MX_OK) return st;
+    if ((st = check_device_ptr(is8, "is8")) != MX_OK) return st;
+    if (workspace == nullptr || ws_bytes < mx::select_workspace_bytes())
+        return fail(MX_ERR_WORKSPACE, "workspace of %zu bytes needed", mx::select_workspace_bytes());
+    if ((st = check_device_ptr(workspace, "workspace")) != MX_OK) return st;
+    if (!aligned16(workspace)) return fail(MX_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+    cudaError_t e = mx::launch_select_top(S, n, n_top, is8, workspace, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MX_OK : cuda_fail(e, "select_top launch");
+}
 
 mx_status mx_copy_mapped(void* dst, const void* src, size_t bytes, void* stream) {
     const void *d = nullptr, *s = nullptr;

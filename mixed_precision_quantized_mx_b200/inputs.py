@@ -82,6 +82,16 @@ def weights(rng: np.random.Generator, N: int, K: int, std: float = 0.02,
     return W
 
 
+def gradients(rng: np.random.Generator, N: int, K: int, std: float = 1e-3, row_sigma: float = 1.0,
+              dtype=np.float32) -> np.ndarray:
+    """Stand-in for the loss gradient of a weight matrix on a calibration batch:
+    G ~ N(0, std) times a log-normal scale per output row (sigma row_sigma), so that
+    a few rows carry most of the gradient."""
+    G = rng.standard_normal((N, K), dtype=np.float32)
+    G *= (np.float32(std) * np.exp(rng.standard_normal(N) * row_sigma).astype(np.float32))[:, None]
+    return G.astype(dtype)
+
+
 def tiny_layer(seed: int = 0) -> Layer:
     """Tiny linear layer: M=16, K=N=512, g=128, 51 of 512 rows at 8 bits, fp32 X."""
     rng = np.random.default_rng(seed)

@@ -238,7 +238,7 @@ def dequant_weights(c: Canonical) -> np.ndarray:
 
 def saliency(W, G, group: int) -> np.ndarray:
     """Channel saliency of the global precision search (MixLLM section 3.2, Eq. 4
-    with one gradient batch, Algorithm 1 lines 3-6): per output row,
+    with one gradient batch, as Algorithm 1 scores a layer): per output row,
     S = |S1 + S1^2/2| with S1 = sum_k G * (dequant(quantize4(W)) - W), in fp64."""
     W = np.ascontiguousarray(_f32(W))
     G = np.ascontiguousarray(_f32(G))
@@ -251,8 +251,8 @@ def saliency(W, G, group: int) -> np.ndarray:
 
 
 def select_top(scores, n_top: int) -> np.ndarray:
-    """Algorithm 1 lines 9-10 over the scores of all layers concatenated: the
-    n_top largest are the 8-bit channels (reading P8: ties go to the lower global
+    """The global choice of Algorithm 1 over the scores of all layers concatenated: the
+    n_top largest are the 8-bit channels (the paper leaves ties open: they go to the lower global
     index, i.e. the earlier layer, then the lower row).  Returns a uint8 mask."""
     scores = np.asarray(scores)
     order = np.lexsort((np.arange(scores.size), -scores.astype(np.float64)))

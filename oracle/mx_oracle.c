@@ -101,7 +101,9 @@ double mxo_fp16_value(uint16_t h)
     return s ? -v : v;
 }
 
-/* R5/R7: the fp16 scale actually used by the quantizers */
+/* The fp16 scale the quantizers use: the fp32 scale rounded to fp16,      */
+/* saturated at 65504; zero (or an fp16 underflow) becomes 1.  The paper   */
+/* fixes only the fp16 type of the scales (MixLLM section 3.3).           */
 static float scale_to_fp16(float s32, uint16_t *bits)
 {
     double s16 = mxo_fp16_round((double)s32);
@@ -118,7 +120,8 @@ static float clampf_(float v, float lo, float hi)
 
 /* ------------------------------------------------------------------------ */
 /* Symmetric 8-bit quantizer (section 2.1 "quantization scheme", range      */
-/* +-127 by R1): s = fp16(absmax/127), q = clamp(round(x/s), -127, 127).    */
+/* +-127; the range is left open there): s = fp16(absmax/127),            */
+/* q = clamp(round(x/s), -127, 127).                                        */
 /* ------------------------------------------------------------------------ */
 void mxo_quant_sym8(const float *x, int n, int8_t *q, uint16_t *s_bits)
 {
@@ -136,7 +139,7 @@ void mxo_quant_sym8(const float *x, int n, int8_t *q, uint16_t *s_bits)
 
 /* ------------------------------------------------------------------------ */
 /* Asymmetric 4-bit quantizer (section 2.1 affine form; z is uint4 per      */
-/* section 3.3, so the range includes 0 by R3):                              */
+/* section 3.3, so the range includes 0):                                   */
 /*   lo = min(0, min x), hi = max(0, max x), s = fp16((hi - lo)/15),         */
 /*   z = clamp(round(-lo/s), 0, 15), q = clamp(round(x/s) + z, 0, 15).       */
 /* ------------------------------------------------------------------------ */
@@ -159,7 +162,8 @@ void mxo_quant_asym4(const float *x, int n, uint8_t *q, uint8_t *z, uint16_t *s_
 
 /* ------------------------------------------------------------------------ */
 /* Activation quantization: 8-bit symmetric per token (act_group == 0) or   */
-/* per group of act_group columns (section 3.1.2 reading, see R2).          */
+/* per group of act_group columns (section 3.1.2 names group-wise scales;  */
+/* the measured configuration uses one scale per token).                    */
 /* X: [M][ldx] fp32.  Aq: [M][K] int8.  s_a: [M] (per token) or [M][K/ag].  */
 /* Returns 0, or -1 on bad arguments.                                       */
 /* ------------------------------------------------------------------------ */
@@ -330,7 +334,7 @@ int mxo_gemm(const int8_t *Aq, const uint16_t *s_a, int act_group, int M, int K,
 /* it): per output row n of one layer,                                     */
 /*   dW = dequant(quantize(W)) - W   (quantize: the 4-bit asymmetric group  */
 /*        quantizer above, the precision a row falls to when it is not      */
-/*        selected; reading R13),                                           */
+/*        selected; no other quantizer is named for this step),            */
 /*   S1 = sum_k G[n,k] * dW[n,k],  S[n] = | S1 + S1^2 / 2 |.                */
 /* W, G: [N][ld] fp32.  S: [N] fp64.  All arithmetic after the codes is     */
 /* fp64.  Returns 0, or -1 on bad arguments.                                */
