@@ -26,10 +26,6 @@ namespace {
 constexpr int kSalWarps = 8;
 constexpr int kSelThreads = 256;
 
-template <typename T> __device__ __forceinline__ float ldv(const T* p);
-template <> __device__ __forceinline__ float ldv<float>(const float* p) { return __ldg(p); }
-template <> __device__ __forceinline__ float ldv<__half>(const __half* p) { return __half2float(__ldg(p)); }
-
 // fp16 scale of an fp32 value: saturate at 65504, zero -> 1 (the packer's rule)
 __device__ __forceinline__ float scale16(float s32) {
     __half h = __float2half_rn(fminf(s32, 65504.0f));
@@ -37,41 +33,112 @@ __device__ __forceinline__ float scale16(float s32) {
     return __half2float(h);
 }
 
-template <typename TW, typename TG>
+// E consecutive elements as fp32: one vector load (streaming, read once) when kVec,
+// else E scalar loads
+template <typename T, int E, bool kVec> struct Vec;
+template <int E> struct Vec<float, E, false> {
+    static __device__ __forceinline__ void load(const float* p, float (&v)[E]) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[e] = __ldg(p + e);
+    }
+};
+template <int E> struct Vec<__half, E, false> {
+    static __device__ __forceinline__ void load(const __half* p, float (&v)[E]) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[e] = __half2float(__ldg(p + e));
+    }
+};
+template <> struct Vec<float, 4, true> {
+    static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
+        const float4 x = __ldcs(reinterpret_cast<const float4*>(p));
+        v[0] = x.x, v[1] = x.y, v[2] = x.z, v[3] = x.w;
+    }
+};
+template <> struct Vec<float, 2, true> {
+    static __device__ __forceinline__ void load(const float* p, float (&v)[2]) {
+        const float2 x = __ldcs(reinterpret_cast<const float2*>(p));
+        v[0] = x.x, v[1] = x.y;
+    }
+};
+template <> struct Vec<__half, 4, true> {
+    static __device__ __forceinline__ void load(const __half* p, float (&v)[4]) {
+        const uint2 x = __ldcs(reinterpret_cast<const uint2*>(p));
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&x.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&x.y));
+        v[0] = a.x, v[1] = a.y, v[2] = b.x, v[3] = b.y;
+    }
+};
+template <> struct Vec<__half, 2, true> {
+    static __device__ __forceinline__ void load(const __half* p, float (&v)[2]) {
+        const unsigned x = __ldcs(reinterpret_cast<const unsigned*>(p));
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&x));
+        v[0] = a.x, v[1] = a.y;
+    }
+};
+
+// One row is scored by `split` warps (1, 2, 4 or 8), each over a contiguous range of
+// groups; a group of 32 E columns is one load of E elements per lane, and U groups
+// are loaded before any is used, so each lane has U (E of W + E of G) in flight.  The
+// warps' fp64 partial sums are added in warp order (deterministic for a shape).
+template <typename TW, typename TG, int E, int U, bool kVec>
 __global__ void __launch_bounds__(kSalWarps * 32)
 saliency_kernel(const TW* __restrict__ W, int64_t ldw, const TG* __restrict__ G, int64_t ldg, int N, int K,
-                int group, float* __restrict__ S) {
-    const int lane = threadIdx.x & 31;
-    const int n = blockIdx.x * kSalWarps + (threadIdx.x >> 5);
-    if (n >= N) return;
-    const TW* w = W + int64_t(n) * ldw;
-    const TG* gr = G + int64_t(n) * ldg;
+                int split, float* __restrict__ S) {
+    constexpr int kGroup = 32 * E;
+    __shared__ double part_sum[kSalWarps];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int slot = warp / split, part = warp % split;
+    const int n = blockIdx.x * (kSalWarps / split) + slot;
+    const int n_groups = K / kGroup;
+    const int per = (n_groups + split - 1) / split;
+    const int g_begin = min(n_groups, part * per), g_end = min(n_groups, g_begin + per);
     double s1 = 0.0;
-    for (int k0 = 0; k0 < K; k0 += group) {
-        // the group's range, then its fp16 scale and zero point
-        float lo = 0.0f, hi = 0.0f;
-        for (int k = lane; k < group; k += 32) {
-            const float v = ldv(w + k0 + k);
-            lo = fminf(lo, v);
-            hi = fmaxf(hi, v);
-        }
+    if (n < N) {                                   // warp-uniform
+        const TW* w_row = W + int64_t(n) * ldw + lane * E;
+        const TG* g_row = G + int64_t(n) * ldg + lane * E;
+        for (int gi = g_begin; gi < g_end; gi += U) {
+            float w[U][E], gv[U][E];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-        }
-        const float s = scale16(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
-        const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.0f), 15.0f);
-        for (int k = lane; k < group; k += 32) {
-            const float v = ldv(w + k0 + k);
-            const float q = fminf(fmaxf(rintf(__fdiv_rn(v, s)) + zf, 0.0f), 15.0f);
-            const double d = double(__fmul_rn(q - zf, s)) - double(v);   // (q - z) s is exact in fp32
-            s1 = fma(double(ldv(gr + k0 + k)), d, s1);
+            for (int u = 0; u < U; ++u) {
+                if (gi + u < g_end) {              // warp-uniform
+                    Vec<TW, E, kVec>::load(w_row + int64_t(gi + u) * kGroup, w[u]);
+                    Vec<TG, E, kVec>::load(g_row + int64_t(gi + u) * kGroup, gv[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (gi + u < g_end) {
+                    // the group's range (0 included), then its fp16 scale and zero point
+                    float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) lo = fminf(lo, w[u][e]), hi = fmaxf(hi, w[u][e]);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+                        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+                    }
+                    const float sc = scale16(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
+                    const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, sc)), 0.0f), 15.0f);
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        const float q = fminf(fmaxf(rintf(__fdiv_rn(w[u][e], sc)) + zf, 0.0f), 15.0f);
+                        // (q - z) s is exact in fp32; the difference with w is taken in fp64
+                        const double d = double(__fmul_rn(q - zf, sc)) - double(w[u][e]);
+                        s1 = fma(double(gv[u][e]), d, s1);
+                    }
+                }
+            }
         }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-    if (lane == 0) S[n] = float(fabs(s1 + 0.5 * s1 * s1));
+    if (lane == 0) part_sum[warp] = s1;
+    __syncthreads();
+    if (part == 0 && lane == 0 && n < N) {
+        double t = 0.0;
+        for (int p = 0; p < split; ++p) t += part_sum[slot * split + p];
+        S[n] = float(fabs(t + 0.5 * t * t));
+    }
 }
 
 // 64-bit key of row i: score bits, then the complemented index (ties: lower first)
@@ -127,25 +194,42 @@ select_mark_kernel(const float* __restrict__ S, int64_t n, int64_t n_top, const 
         is8[i] = n_top >= n ? 1 : (n_top == 0 ? 0 : (sel_key(S, i) >= T ? 1 : 0));
 }
 
+template <typename TW, typename TG, int E, int U>
+cudaError_t launch_saliency_t(const void* W, int64_t ldw, const void* G, int64_t ldg, int N, int K, int split,
+                              float* S, cudaStream_t s) {
+    const TW* w = static_cast<const TW*>(W);
+    const TG* g = static_cast<const TG*>(G);
+    // vector loads when every row's E-element runs are aligned to the vector size
+    const bool vec = reinterpret_cast<uintptr_t>(W) % (E * sizeof(TW)) == 0 && ldw % E == 0 &&
+                     reinterpret_cast<uintptr_t>(G) % (E * sizeof(TG)) == 0 && ldg % E == 0;
+    const dim3 grid((N + kSalWarps / split - 1) / (kSalWarps / split)), block(kSalWarps * 32);
+    if (vec)
+        saliency_kernel<TW, TG, E, U, true><<<grid, block, 0, s>>>(w, ldw, g, ldg, N, K, split, S);
+    else
+        saliency_kernel<TW, TG, E, U, false><<<grid, block, 0, s>>>(w, ldw, g, ldg, N, K, split, S);
+    return cudaGetLastError();
+}
+
+template <typename TW, typename TG>
+cudaError_t launch_saliency_g(const void* W, int64_t ldw, const void* G, int64_t ldg, int N, int K, int group,
+                              float* S, cudaStream_t s) {
+    // warps per row: enough rows' warps to fill every SM about 32 warps deep, at most
+    // one warp per group
+    int split = 1;
+    while (split < kSalWarps && int64_t(N) * split < 148 * 32 && 2 * split <= K / group) split *= 2;
+    return group == 128 ? launch_saliency_t<TW, TG, 4, 4>(W, ldw, G, ldg, N, K, split, S, s)
+                        : launch_saliency_t<TW, TG, 2, 8>(W, ldw, G, ldg, N, K, split, S, s);
+}
+
 }  // namespace
 
 cudaError_t launch_saliency(const void* W, mx_dtype wdt, int64_t ldw, const void* G, mx_dtype gdt, int64_t ldg,
                             int N, int K, int group, float* S, cudaStream_t s) {
     if (N == 0) return cudaSuccess;
-    const dim3 grid((N + kSalWarps - 1) / kSalWarps), block(kSalWarps * 32);
-    if (wdt == MX_F16 && gdt == MX_F16)
-        saliency_kernel<__half, __half><<<grid, block, 0, s>>>(static_cast<const __half*>(W), ldw,
-                                                              static_cast<const __half*>(G), ldg, N, K, group, S);
-    else if (wdt == MX_F16)
-        saliency_kernel<__half, float><<<grid, block, 0, s>>>(static_cast<const __half*>(W), ldw,
-                                                             static_cast<const float*>(G), ldg, N, K, group, S);
-    else if (gdt == MX_F16)
-        saliency_kernel<float, __half><<<grid, block, 0, s>>>(static_cast<const float*>(W), ldw,
-                                                             static_cast<const __half*>(G), ldg, N, K, group, S);
-    else
-        saliency_kernel<float, float><<<grid, block, 0, s>>>(static_cast<const float*>(W), ldw,
-                                                            static_cast<const float*>(G), ldg, N, K, group, S);
-    return cudaGetLastError();
+    if (wdt == MX_F16 && gdt == MX_F16) return launch_saliency_g<__half, __half>(W, ldw, G, ldg, N, K, group, S, s);
+    if (wdt == MX_F16) return launch_saliency_g<__half, float>(W, ldw, G, ldg, N, K, group, S, s);
+    if (gdt == MX_F16) return launch_saliency_g<float, __half>(W, ldw, G, ldg, N, K, group, S, s);
+    return launch_saliency_g<float, float>(W, ldw, G, ldg, N, K, group, S, s);
 }
 
 size_t select_workspace_bytes() { return (sizeof(SelState) + 255) & ~size_t(255); }
