@@ -92,6 +92,14 @@ def gradients(rng: np.random.Generator, N: int, K: int, std: float = 1e-3, row_s
     return G.astype(dtype)
 
 
+def block_codes(rng: np.random.Generator, N: int, K: int, probs=(0.25, 0.25, 0.25, 0.25),
+                block_rows: int = 64, block_cols: int = 128) -> np.ndarray:
+    """2-bit code (0..3) of every block of block_rows output rows x block_cols input
+    columns, drawn with the given probabilities: [ceil(N / block_rows), K / block_cols]."""
+    shape = ((N + block_rows - 1) // block_rows, K // block_cols)
+    return rng.choice(4, size=shape, p=np.asarray(probs, np.float64)).astype(np.uint8)
+
+
 def tiny_layer(seed: int = 0) -> Layer:
     """Tiny linear layer: M=16, K=N=512, g=128, 51 of 512 rows at 8 bits, fp32 X."""
     rng = np.random.default_rng(seed)

@@ -63,6 +63,12 @@ def _load():
     lib.mxo_gemm.restype = I
     lib.mxo_saliency.argtypes = [P, I, P, I, I, I, I, P]
     lib.mxo_saliency.restype = I
+    lib.mxo_quant_asym.argtypes = [P, I, I, P, P, P]
+    lib.mxo_quant_asym.restype = I
+    lib.mxo_pack_blockwise.argtypes = [P, I, I, I, P, P, P, P, P]
+    lib.mxo_pack_blockwise.restype = I
+    lib.mxo_gemm_blockwise.argtypes = [P, P, I, I, I, P, P, P, P, P, ctypes.c_long, P, P, P]
+    lib.mxo_gemm_blockwise.restype = ctypes.c_int64
     _lib = lib
     return lib
 
@@ -259,3 +265,107 @@ def select_top(scores, n_top: int) -> np.ndarray:
     mask = np.zeros(scores.size, np.uint8)
     mask[order[:max(0, min(n_top, scores.size))]] = 1
     return mask
+
+
+# ----------------------------------------------------------------- block-wise bit widths
+BLOCK_ROWS, BLOCK_COLS = 64, 128
+
+
+def quant_asym(x, bits: int) -> tuple[np.ndarray, int, int]:
+    """Asymmetric b-bit quantizer of one group, 1 <= b <= 7 (the 4-bit quantizer of
+    MixLLM section 2.1 with 2^b - 1 levels; b = 4 is quant_asym4)."""
+    x = _f32(x).ravel()
+    q = np.zeros(x.size, np.uint8)
+    z = np.zeros(1, np.uint8)
+    s = np.zeros(1, np.uint16)
+    if _load().mxo_quant_asym(_p(x), x.size, int(bits), _p(q), _p(z), _p(s)) != 0:
+        raise ValueError("quant_asym: bad arguments")
+    return q, int(z[0]), int(s[0])
+
+
+def pack_block_codes(codes: np.ndarray) -> np.ndarray:
+    """2-bit block codes [NB, KB] (values 0..3) packed four to a byte, block i (row-major)
+    in bits 2 (i mod 4) of byte i / 4 (the ScaleBITS blog page's 2-bit metadata, section 3.2)."""
+    flat = np.asarray(codes, dtype=np.uint8).ravel()
+    assert flat.size == 0 or int(flat.max()) <= 3
+    out = np.zeros((flat.size + 3) // 4, np.uint8)
+    for i, c in enumerate(flat):
+        out[i >> 2] |= np.uint8(int(c) << (2 * (i & 3)))
+    return out
+
+
+@dataclass
+class Blockwise:
+    """A layer with one bit width per 64 x 128 block, in original row order."""
+    N: int
+    K: int
+    table: np.ndarray     # [4] uint8: the widths the 2-bit codes select
+    codes: np.ndarray     # [NB, KB] uint8: each block's 2-bit code
+    meta: np.ndarray      # packed codes (pack_block_codes)
+    q: np.ndarray         # [N, K] int16: -127..127 in 8-bit blocks, else 0..2^b - 1
+    zeros: np.ndarray     # [N, KB] uint8 (0 in 8-bit blocks)
+    scales: np.ndarray    # [N, KB] uint16 fp16 bits
+
+    @property
+    def KB(self) -> int:
+        return self.K // BLOCK_COLS
+
+    def widths(self) -> np.ndarray:
+        """[NB, KB] bit width of every block."""
+        return self.table[self.codes]
+
+
+def pack_blockwise(W, codes, table) -> Blockwise:
+    """Quantize W block by block (ScaleBITS blog page, sections 1.2.2 and 3.2): each row's
+    128 weights inside a block are one group, 8-bit blocks symmetric, narrower blocks
+    asymmetric with 2^b levels."""
+    W = _f32(W)
+    N, K = W.shape
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    table = np.ascontiguousarray(table, dtype=np.uint8)
+    assert table.shape == (4,)
+    assert codes.shape == ((N + BLOCK_ROWS - 1) // BLOCK_ROWS, K // BLOCK_COLS)
+    meta = pack_block_codes(codes)
+    KB = K // BLOCK_COLS
+    q = np.zeros((N, K), np.int16)
+    zeros = np.zeros((N, KB), np.uint8)
+    scales = np.zeros((N, KB), np.uint16)
+    if _load().mxo_pack_blockwise(_p(W), N, K, K, _p(table), _p(meta), _p(q), _p(zeros), _p(scales)) != 0:
+        raise ValueError("mxo_pack_blockwise: bad arguments")
+    return Blockwise(N, K, table, codes, meta, q, zeros, scales)
+
+
+def gemm_blockwise(Aq: np.ndarray, s_a: np.ndarray, b: Blockwise,
+                   pairs: tuple[np.ndarray, np.ndarray] | None = None):
+    """fp64 Y two ways (plain definition; two-step form of MixLLM section 3.3 over each
+    block's groups) and the int64 partials P [.., KB].  Returns (Y_def, Y_two, P, max |P|)."""
+    Aq = np.ascontiguousarray(Aq, dtype=np.int8)
+    s_a = np.ascontiguousarray(s_a, dtype=np.uint16)
+    M = Aq.shape[0]
+    assert Aq.shape[1] == b.K and s_a.shape == (M,)
+    if pairs is None:
+        pm = pn = None
+        cnt = M * b.N
+        shape = (M, b.N)
+    else:
+        pm = np.ascontiguousarray(pairs[0], dtype=np.int32)
+        pn = np.ascontiguousarray(pairs[1], dtype=np.int32)
+        cnt = pm.size
+        shape = (cnt,)
+    yd = np.zeros(cnt, np.float64)
+    yt = np.zeros(cnt, np.float64)
+    P = np.zeros((cnt, b.KB), np.int64)
+    pmax = _load().mxo_gemm_blockwise(_p(Aq), _p(s_a), M, b.K, b.N, _p(b.q), _p(b.zeros), _p(b.scales),
+                                      None if pm is None else _p(pm), None if pn is None else _p(pn),
+                                      cnt, _p(yd), _p(yt), _p(P))
+    if pmax < 0:
+        raise ValueError("mxo_gemm_blockwise: bad arguments")
+    return yd.reshape(shape), yt.reshape(shape), P.reshape(shape + (b.KB,)), int(pmax)
+
+
+def bits_per_weight(b: Blockwise) -> float:
+    """Average stored bits per weight: each block's codes plus its 2-bit metadata (the
+    per-row fp16 scales and zeros are counted separately by the layout)."""
+    rows = np.minimum(BLOCK_ROWS, b.N - np.arange(b.codes.shape[0]) * BLOCK_ROWS)
+    code_bits = float((b.widths().astype(np.int64) * rows[:, None] * BLOCK_COLS).sum())
+    return (code_bits + 2.0 * b.codes.size) / (b.N * b.K)

@@ -363,3 +363,135 @@ int mxo_saliency(const float *W, int ldw, const float *G, int ldg, int N, int K,
     free(q);
     return 0;
 }
+
+/* ======================================================================== */
+/* Block-wise bit widths (ScaleBITS blog page: section 1.2.2, the hardware- */
+/* aligned block partition with one bit width per 64 x 128 block; section   */
+/* 3.2, the block-wise layout with 2-bit metadata recording each block's    */
+/* width; section 4.2, the width search space {1, 2, 3, 4, 6, 8}).          */
+/*                                                                          */
+/* Readings (the page gives no quantizer and no layout beyond that):        */
+/*  - a block is 64 output rows x 128 input columns; the last row block may */
+/*    be short; K is a multiple of 128;                                     */
+/*  - the 2-bit code of a block indexes a four-entry width table of the     */
+/*    layer; the codes are stored four to a byte, block i in bits           */
+/*    2(i mod 4) of byte i / 4, blocks in row-major (row block, column      */
+/*    block) order;                                                         */
+/*  - inside a block each row's 128 weights are one group with its own fp16 */
+/*    scale (and zero), as MixLLM's group-wise weights;                     */
+/*  - b = 8: the symmetric 8-bit quantizer above (z = 0); b < 8: the        */
+/*    asymmetric b-bit form of the 4-bit quantizer above, levels            */
+/*    0 .. 2^b - 1.  So q - z always fits int8 and the same two-step int8   */
+/*    dequantization applies to every block.                                */
+/* ======================================================================== */
+
+/* Asymmetric b-bit quantizer, 1 <= b <= 7 (b = 4 is mxo_quant_asym4):       */
+/*   qmax = 2^b - 1, lo = min(0, min x), hi = max(0, max x),                */
+/*   s = fp16((hi - lo)/qmax), z = clamp(round(-lo/s), 0, qmax),            */
+/*   q = clamp(round(x/s) + z, 0, qmax).                                    */
+int mxo_quant_asym(const float *x, int n, int bits, uint8_t *q, uint8_t *z, uint16_t *s_bits)
+{
+    if (n <= 0 || bits < 1 || bits > 7) return -1;
+    const float qmax = (float)((1 << bits) - 1);
+    float lo = 0.0f, hi = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        if (x[i] < lo) lo = x[i];
+        if (x[i] > hi) hi = x[i];
+    }
+    float range = hi - lo;
+    float s = scale_to_fp16(range / qmax, s_bits);
+    float zf = clampf_(rintf(-lo / s), 0.0f, qmax);
+    *z = (uint8_t)zf;
+    for (int i = 0; i < n; ++i) {
+        float r = rintf(x[i] / s) + zf;
+        q[i] = (uint8_t)clampf_(r, 0.0f, qmax);
+    }
+    return 0;
+}
+
+#define MXO_BLK_ROWS 64
+#define MXO_BLK_COLS 128
+
+/* the width of block (rb, kb) from the packed 2-bit codes and the table */
+static int block_bits(const uint8_t *meta, const uint8_t *table, int KB, int rb, int kb)
+{
+    long i = (long)rb * KB + kb;
+    return table[(meta[i >> 2] >> (2 * (i & 3))) & 3];
+}
+
+/* Quantize W [N][ldw] fp32 block by block.  table: four widths, each in    */
+/* 1..8.  meta: ceil(NB * KB / 4) bytes of 2-bit codes, NB = ceil(N / 64),  */
+/* KB = K / 128.  Out, in original row order: q [N][K] int16 (the code:     */
+/* -127..127 for 8-bit blocks, 0..2^b - 1 otherwise), zeros [N][KB] uint8   */
+/* (0 for 8-bit blocks), scales [N][KB] fp16 bits.  Returns 0, or -1.       */
+int mxo_pack_blockwise(const float *W, int N, int K, int ldw, const uint8_t *table, const uint8_t *meta,
+                       int16_t *q, uint8_t *zeros, uint16_t *scales)
+{
+    if (N < 0 || K <= 0 || K % MXO_BLK_COLS || ldw < K) return -1;
+    for (int c = 0; c < 4; ++c)
+        if (table[c] < 1 || table[c] > 8) return -1;
+    const int KB = K / MXO_BLK_COLS;
+    int8_t c8[MXO_BLK_COLS];
+    uint8_t ca[MXO_BLK_COLS];
+    for (int n = 0; n < N; ++n)
+        for (int kb = 0; kb < KB; ++kb) {
+            const float *w = W + (size_t)n * ldw + (size_t)kb * MXO_BLK_COLS;
+            const int b = block_bits(meta, table, KB, n / MXO_BLK_ROWS, kb);
+            int16_t *qo = q + (size_t)n * K + (size_t)kb * MXO_BLK_COLS;
+            uint16_t sb;
+            if (b == 8) {
+                mxo_quant_sym8(w, MXO_BLK_COLS, c8, &sb);
+                for (int k = 0; k < MXO_BLK_COLS; ++k) qo[k] = c8[k];
+                zeros[(size_t)n * KB + kb] = 0;
+            } else {
+                uint8_t z;
+                mxo_quant_asym(w, MXO_BLK_COLS, b, ca, &z, &sb);
+                for (int k = 0; k < MXO_BLK_COLS; ++k) qo[k] = ca[k];
+                zeros[(size_t)n * KB + kb] = z;
+            }
+            scales[(size_t)n * KB + kb] = sb;
+        }
+    return 0;
+}
+
+/* The two-step GEMM over a block-wise layer (MixLLM section 3.3 applied to  */
+/* each 128-column group), fp64, at the listed (m, n) pairs (pairs == NULL: */
+/* every (m, n), row-major [M][N]), two ways that must agree:               */
+/*   Y_def = sum_k (Aq s_a)[m][k] * ((q - z) s_w)[n][k]                     */
+/*   Y_two = sum_kb s_a[m] s_w[n][kb] P[m][n][kb],                          */
+/*           P[m][n][kb] = sum_{k in kb} Aq[m][k] (q[n][k] - z[n][kb])       */
+/* P (optional, [n_pairs][KB] int64) receives the partials.  s_a: one fp16   */
+/* scale per token.  Returns the largest |P|, or -1 on bad arguments.       */
+int64_t mxo_gemm_blockwise(const int8_t *Aq, const uint16_t *s_a, int M, int K, int N, const int16_t *q,
+                           const uint8_t *zeros, const uint16_t *scales, const int32_t *pair_m,
+                           const int32_t *pair_n, long n_pairs, double *Y_def, double *Y_two, int64_t *P)
+{
+    if (M < 0 || N < 0 || K <= 0 || K % MXO_BLK_COLS) return -1;
+    const int KB = K / MXO_BLK_COLS;
+    const long total = pair_m ? n_pairs : (long)M * N;
+    int64_t pmax = 0;
+    for (long t = 0; t < total; ++t) {
+        const int m = pair_m ? pair_m[t] : (int)(t / (N > 0 ? N : 1));
+        const int n = pair_m ? pair_n[t] : (int)(t % (N > 0 ? N : 1));
+        if (m < 0 || m >= M || n < 0 || n >= N) return -1;
+        const double sa = mxo_fp16_value(s_a[m]);
+        double ydef = 0.0, ytwo = 0.0;
+        for (int kb = 0; kb < KB; ++kb) {
+            const double sw = mxo_fp16_value(scales[(size_t)n * KB + kb]);
+            const int z = zeros[(size_t)n * KB + kb];
+            int64_t p = 0;
+            for (int k = kb * MXO_BLK_COLS; k < (kb + 1) * MXO_BLK_COLS; ++k) {
+                const int a = Aq[(size_t)m * K + k];
+                const int w = q[(size_t)n * K + k] - z;
+                ydef += ((double)a * sa) * ((double)w * sw);
+                p += (int64_t)a * (int64_t)w;
+            }
+            ytwo += sa * sw * (double)p;
+            if (P) P[t * KB + kb] = p;
+            if (llabs(p) > pmax) pmax = llabs(p);
+        }
+        Y_def[t] = ydef;
+        Y_two[t] = ytwo;
+    }
+    return pmax;
+}
