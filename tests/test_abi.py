@@ -218,3 +218,30 @@ def test_group_wise_activation_options_checked_on_the_host(lib):
     assert mx.mx_linear_workspace_size(L, 8, act_group=128) == a16(8 * 1024) + a16(2 * 8 * 8)
     assert mx.mx_linear_workspace_size(L, 8) == a16(8 * 1024) + a16(2 * 8)
     assert mx.mx_linear_workspace_size(L, 2, act_group=128) == 0                 # fused
+
+
+def test_precision_search_argument_checks_before_any_launch(lib):
+    # mx_saliency: group, divisibility, leading dimensions and dtypes are refused on the
+    # host; no rows is a no-op.  None of these reaches a CUDA call.
+    P = ctypes.c_void_p(16)
+    S = ctypes.c_void_p(32)
+    assert lib.mx_saliency(P, 0, 256, P, 0, 256, 4, 256, 96, S, None) == 2     # group 96
+    assert lib.mx_saliency(P, 0, 256, P, 0, 256, 4, 200, 128, S, None) == 1    # K % group
+    assert lib.mx_saliency(P, 0, 100, P, 0, 256, 4, 256, 128, S, None) == 1    # ldw < K
+    assert lib.mx_saliency(P, 0, 256, P, 0, 255, 4, 256, 128, S, None) == 1    # ldg < K
+    assert lib.mx_saliency(P, 7, 256, P, 0, 256, 4, 256, 128, S, None) == 1    # W dtype
+    assert lib.mx_saliency(P, 0, 256, P, 2, 256, 4, 256, 128, S, None) == 1    # G dtype
+    assert lib.mx_saliency(P, 0, 256, P, 0, 256, -1, 256, 128, S, None) == 1   # N < 0
+    assert lib.mx_saliency(P, 0, 256, P, 0, 256, 0, 256, 128, S, None) == 0    # nothing to do
+    # mx_select_top: the workspace is a fixed small size; counts are checked first
+    nb = ctypes.c_size_t(0)
+    assert lib.mx_select_top_workspace_size(1 << 20, ctypes.byref(nb)) == 0
+    assert 0 < nb.value <= 4096 and nb.value % 16 == 0
+    assert lib.mx_select_top_workspace_size(-1, ctypes.byref(nb)) == 1
+    assert lib.mx_select_top_workspace_size(1 << 32, ctypes.byref(nb)) == 1
+    assert lib.mx_select_top_workspace_size(5, None) == 1
+    assert lib.mx_select_top(S, 10, 11, P, P, 4096, None) == 1                # n_top > n
+    assert lib.mx_select_top(S, 10, -1, P, P, 4096, None) == 1
+    assert lib.mx_select_top(S, -1, 0, P, P, 4096, None) == 1
+    assert lib.mx_select_top(S, 1 << 32, 0, P, P, 4096, None) == 1            # index must fit 32 bits
+    assert lib.mx_select_top(S, 0, 0, P, None, 0, None) == 0                  # nothing to do
