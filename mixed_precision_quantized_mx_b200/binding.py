@@ -10,6 +10,7 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -28,7 +29,7 @@ EXPORTED = ("mx_version", "mx_last_error", "mx_layout_init", "mx_layout_from_hea
             "mx_pack_weights", "mx_quant_act", "mx_gemm_workspace_size", "mx_gemm_select_path",
             "mx_gemm", "mx_linear_workspace_size", "mx_linear", "mx_linear_noalloc",
             "mx_quant_act_grouped", "mx_copy_mapped", "mx_saliency", "mx_select_top_workspace_size",
-            "mx_select_top")
+            "mx_select_top", "mx_bw_layout_init", "mx_bw_pack", "mx_bw_gemm")
 
 
 class MXError(RuntimeError):
@@ -44,6 +45,14 @@ class Layout(ctypes.Structure):
                [(n, ctypes.c_uint64) for n in
                 ("off_rowmap", "off_scales8", "off_codes8", "off_scales4", "off_zeros4",
                  "off_codes4", "total_bytes")]
+
+
+class BwLayout(ctypes.Structure):
+    """mirror of mx_bw_layout (block-wise bit widths)"""
+    _fields_ = [(n, ctypes.c_int32) for n in ("N", "K", "NB", "KB")] + \
+               [("table", ctypes.c_uint8 * 4), ("reserved0", ctypes.c_int32)] + \
+               [(n, ctypes.c_uint64) for n in
+                ("off_meta", "off_offsets", "off_scales", "off_zeros", "off_codes", "code_bytes", "total_bytes")]
 
 
 class GemmOpts(ctypes.Structure):
@@ -90,10 +99,13 @@ def lib() -> ctypes.CDLL:
     L.mx_saliency.argtypes = [P, I, I64, P, I, I64, I, I, I, P, P]
     L.mx_select_top_workspace_size.argtypes = [I64, ctypes.POINTER(Z)]
     L.mx_select_top.argtypes = [P, I64, I64, P, P, Z, P]
+    L.mx_bw_layout_init.argtypes = [I, I, P, P, ctypes.POINTER(BwLayout)]
+    L.mx_bw_pack.argtypes = [ctypes.POINTER(BwLayout), P, P, I, I64, P, P]
+    L.mx_bw_gemm.argtypes = [ctypes.POINTER(BwLayout), P, P, P, I, P, I64, P, P]
     for n in ("mx_layout_init", "mx_layout_from_header", "mx_pack_weights", "mx_quant_act",
               "mx_quant_act_grouped", "mx_gemm_workspace_size", "mx_gemm", "mx_linear_workspace_size", "mx_linear",
               "mx_linear_noalloc", "mx_copy_mapped", "mx_saliency", "mx_select_top_workspace_size",
-              "mx_select_top"):
+              "mx_select_top", "mx_bw_layout_init", "mx_bw_pack", "mx_bw_gemm"):
         getattr(L, n).restype = I
     _lib = L
     return L
@@ -273,3 +285,38 @@ def mx_select_top(S: torch.Tensor, n_top: int, is8: torch.Tensor | None = None, 
     _check(lib().mx_select_top(_ptr(S), n, n_top, _ptr(is8), _ptr(ws), ws.numel(), _stream(stream)),
            "mx_select_top")
     return is8
+
+
+# ------------------------------------------------------------------ block-wise bit widths
+def _host_bytes(a) -> ctypes.Array:
+    b = bytes(np.ascontiguousarray(np.asarray(a, dtype=np.uint8)).tobytes())
+    return (ctypes.c_uint8 * max(1, len(b))).from_buffer_copy(b if b else b"\0")
+
+
+def mx_bw_layout_init(N: int, K: int, table, meta) -> BwLayout:
+    """Geometry of a block-wise layer (see mx_blockwise.h); table: four widths, meta: the
+    packed 2-bit block codes (host bytes)."""
+    L = BwLayout()
+    _check(lib().mx_bw_layout_init(N, K, _host_bytes(table), _host_bytes(meta), ctypes.byref(L)),
+           "mx_bw_layout_init")
+    return L
+
+
+def mx_bw_pack(L: BwLayout, meta, W: torch.Tensor, blob: torch.Tensor, stream=None) -> None:
+    assert W.dim() == 2 and W.stride(1) == 1 and tuple(W.shape) == (L.N, L.K)
+    assert blob.numel() * blob.element_size() >= L.total_bytes
+    _check(lib().mx_bw_pack(ctypes.byref(L), _host_bytes(meta), _ptr(W), _dtype_code(W), W.stride(0), _ptr(blob),
+                            _stream(stream)), "mx_bw_pack")
+
+
+def mx_bw_gemm(L: BwLayout, blob: torch.Tensor, Aq: torch.Tensor, s_a: torch.Tensor, Y: torch.Tensor,
+               partials: torch.Tensor | None = None, stream=None) -> None:
+    assert Aq.dim() == 2 and Aq.is_contiguous() and Aq.dtype == torch.int8 and Aq.shape[1] == L.K
+    assert s_a.dtype == torch.float16 and Y.dtype == torch.float16 and Y.stride(1) == 1
+    M = Aq.shape[0]
+    assert blob.numel() * blob.element_size() >= L.total_bytes and s_a.numel() >= M
+    assert Y.shape[0] >= M and Y.shape[1] >= L.N
+    assert partials is None or (partials.dtype == torch.int32 and partials.is_contiguous()
+                                and partials.numel() >= M * L.N * L.KB)
+    _check(lib().mx_bw_gemm(ctypes.byref(L), _ptr(blob), _ptr(Aq), _ptr(s_a), Aq.shape[0], _ptr(Y), Y.stride(0),
+                            _ptr(partials), _stream(stream)), "mx_bw_gemm")

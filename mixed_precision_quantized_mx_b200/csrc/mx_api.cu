@@ -7,8 +7,11 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
+#include <algorithm>
 
 #include "mx_internal.cuh"
+#include "mx_blockwise.h"
 
 namespace {
 
@@ -110,6 +113,12 @@ cudaError_t launch_saliency(const void* W, mx_dtype wdt, int64_t ldw, const void
 size_t select_workspace_bytes();
 cudaError_t launch_select_top(const float* S, int64_t n, int64_t n_top, uint8_t* is8, void* workspace,
                               cudaStream_t s);
+
+// block-wise bit widths (blockwise.cu)
+cudaError_t launch_bw_pack(const mx_bw_layout& L, const void* W, mx_dtype wdt, int64_t ldw, uint8_t* blob,
+                           cudaStream_t s);
+cudaError_t launch_bw_gemm(const mx_bw_layout& L, const uint8_t* blob, const int8_t* Aq, const __half* s_a, int M,
+                           __half* Y, int64_t ldy, int32_t* P, cudaStream_t s);
 
 Geom make_geom(const mx_layout& L, const void* blob) {
     const uint8_t* b = static_cast<const uint8_t*>(blob);
@@ -444,6 +453,129 @@ mx_status mx_select_top(const float* S, int64_t n, int64_t n_top, uint8_t* is8, 
     if (!aligned16(workspace)) return fail(MX_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
     cudaError_t e = mx::launch_select_top(S, n, n_top, is8, workspace, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MX_OK : cuda_fail(e, "select_top launch");
+}
+
+// ---------------------------------------------------------------- block-wise bit widths
+namespace {
+
+constexpr uint32_t kBwMagic = 0x5742584Du;    // "MXBW"
+constexpr uint32_t kBwVersion = 1;
+constexpr uint64_t kBwHeaderBytes = 64;
+
+// the block offsets (16-byte units from the codes) of a layer, and their end
+mx_status bw_geometry(int N, int K, const uint8_t table[4], const uint8_t* meta, mx_bw_layout* L,
+                      std::vector<uint32_t>* offsets) {
+    if (N < 1 || K < MX_BW_BLOCK_COLS || K % MX_BW_BLOCK_COLS)
+        return fail(MX_ERR_INVALID_ARG, "N=%d K=%d: N >= 1, K a positive multiple of 128", N, K);
+    if (table == nullptr || meta == nullptr) return fail(MX_ERR_INVALID_ARG, "table or meta is NULL");
+    for (int c = 0; c < 4; ++c)
+        if (table[c] < 1 || table[c] > 8) return fail(MX_ERR_INVALID_ARG, "width table[%d]=%d outside 1..8", c, table[c]);
+    mx_bw_layout l;
+    memset(&l, 0, sizeof l);
+    l.N = N;
+    l.K = K;
+    l.NB = (N + MX_BW_BLOCK_ROWS - 1) / MX_BW_BLOCK_ROWS;
+    l.KB = K / MX_BW_BLOCK_COLS;
+    memcpy(l.table, table, 4);
+    const int64_t nblk = int64_t(l.NB) * l.KB;
+    if (offsets) offsets->assign(size_t(nblk) + 1, 0u);
+    uint64_t units = 0;                          // 16-byte units
+    for (int64_t bi = 0; bi < nblk; ++bi) {
+        if (offsets) (*offsets)[size_t(bi)] = uint32_t(units);
+        const int rb = int(bi / l.KB);
+        const int rows = std::min(MX_BW_BLOCK_ROWS, N - rb * MX_BW_BLOCK_ROWS);
+        const int b = table[(meta[bi >> 2] >> (2 * (bi & 3))) & 3];
+        units += uint64_t(rows) * uint64_t(b);   // 16 b bytes per row
+        if (units > 0xFFFFFFFFull) return fail(MX_ERR_UNSUPPORTED, "codes larger than 64 GiB");
+    }
+    if (offsets) (*offsets)[size_t(nblk)] = uint32_t(units);
+    l.code_bytes = units * 16;
+    l.off_meta = kBwHeaderBytes;
+    l.off_offsets = align16(l.off_meta + uint64_t((nblk + 3) / 4));
+    l.off_scales = align16(l.off_offsets + 4 * uint64_t(nblk + 1));
+    l.off_zeros = align16(l.off_scales + 2 * uint64_t(N) * l.KB);
+    l.off_codes = align16(l.off_zeros + uint64_t(N) * l.KB);
+    l.total_bytes = l.off_codes + l.code_bytes;
+    *L = l;
+    return MX_OK;
+}
+
+// a layout's fields agree with one another (as mx_bw_layout_init made them)
+mx_status bw_check(const mx_bw_layout* L) {
+    if (L == nullptr) return fail(MX_ERR_INVALID_ARG, "layout is NULL");
+    if (L->N < 1 || L->K < MX_BW_BLOCK_COLS || L->K % MX_BW_BLOCK_COLS ||
+        L->NB != (L->N + MX_BW_BLOCK_ROWS - 1) / MX_BW_BLOCK_ROWS || L->KB != L->K / MX_BW_BLOCK_COLS)
+        return fail(MX_ERR_INVALID_ARG, "layout geometry is inconsistent");
+    for (int c = 0; c < 4; ++c)
+        if (L->table[c] < 1 || L->table[c] > 8) return fail(MX_ERR_INVALID_ARG, "layout width table is invalid");
+    const uint64_t nblk = uint64_t(L->NB) * L->KB;
+    if (L->off_meta != kBwHeaderBytes || L->off_offsets != align16(L->off_meta + (nblk + 3) / 4) ||
+        L->off_scales != align16(L->off_offsets + 4 * (nblk + 1)) ||
+        L->off_zeros != align16(L->off_scales + 2 * uint64_t(L->N) * L->KB) ||
+        L->off_codes != align16(L->off_zeros + uint64_t(L->N) * L->KB) ||
+        L->total_bytes != L->off_codes + L->code_bytes || L->code_bytes % 16 ||
+        L->code_bytes < uint64_t(L->N) * L->K / 8 || L->code_bytes > uint64_t(L->N) * L->K)
+        return fail(MX_ERR_INVALID_ARG, "layout offsets are inconsistent");
+    return MX_OK;
+}
+
+}  // namespace
+
+mx_status mx_bw_layout_init(int N, int K, const uint8_t table[4], const uint8_t* meta, mx_bw_layout* out) {
+    if (out == nullptr) return fail(MX_ERR_INVALID_ARG, "out is NULL");
+    return bw_geometry(N, K, table, meta, out, nullptr);
+}
+
+mx_status mx_bw_pack(const mx_bw_layout* L, const uint8_t* meta, const void* W, mx_dtype wdtype, int64_t ldw,
+                     void* blob, void* stream) {
+    mx_status st;
+    if ((st = bw_check(L)) != MX_OK) return st;
+    mx_bw_layout ref;
+    std::vector<uint32_t> offsets;
+    if ((st = bw_geometry(L->N, L->K, L->table, meta, &ref, &offsets)) != MX_OK) return st;
+    if (memcmp(&ref, L, sizeof ref) != 0) return fail(MX_ERR_INVALID_ARG, "layout was not made from this meta");
+    if (wdtype != MX_F32 && wdtype != MX_F16) return fail(MX_ERR_INVALID_ARG, "bad dtype %d", int(wdtype));
+    if (ldw < L->K) return fail(MX_ERR_INVALID_ARG, "ldw=%lld < K=%d", (long long)ldw, L->K);
+    if ((st = check_device_ptr(W, "W")) != MX_OK) return st;
+    if ((st = check_device_ptr(blob, "blob")) != MX_OK) return st;
+    if (!aligned16(blob)) return fail(MX_ERR_ALIGNMENT, "blob must be 16-byte aligned");
+    // header, block codes and offsets, staged on the host and copied in the stream
+    std::vector<uint8_t> head(size_t(L->off_scales), 0);
+    const uint32_t h[6] = {kBwMagic, kBwVersion, uint32_t(L->N), uint32_t(L->K),
+                           uint32_t(L->table[0]) | uint32_t(L->table[1]) << 8 | uint32_t(L->table[2]) << 16 |
+                               uint32_t(L->table[3]) << 24,
+                           uint32_t(L->code_bytes >> 4)};
+    memcpy(head.data(), h, sizeof h);
+    const uint64_t nblk = uint64_t(L->NB) * L->KB;
+    memcpy(head.data() + L->off_meta, meta, size_t((nblk + 3) / 4));
+    memcpy(head.data() + L->off_offsets, offsets.data(), offsets.size() * sizeof(uint32_t));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(blob, 0, size_t(L->total_bytes), s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(blob, head.data(), head.size(), cudaMemcpyHostToDevice, s);
+    // a pageable source: the call returns once the bytes are staged, so `head` may go
+    if (e == cudaSuccess) e = mx::launch_bw_pack(*L, W, wdtype, ldw, static_cast<uint8_t*>(blob), s);
+    return e == cudaSuccess ? MX_OK : cuda_fail(e, "bw pack");
+}
+
+mx_status mx_bw_gemm(const mx_bw_layout* L, const void* blob, const int8_t* Aq, const void* s_a, int M, void* Y,
+                     int64_t ldy, int32_t* partials, void* stream) {
+    mx_status st;
+    if ((st = bw_check(L)) != MX_OK) return st;
+    if (M < 0) return fail(MX_ERR_INVALID_ARG, "M=%d", M);
+    if (M > 65535 * 8) return fail(MX_ERR_UNSUPPORTED, "M=%d: at most %d tokens per call", M, 65535 * 8);
+    if (ldy < L->N) return fail(MX_ERR_INVALID_ARG, "ldy=%lld < N=%d", (long long)ldy, L->N);
+    if (M == 0) return MX_OK;
+    if ((st = check_device_ptr(blob, "blob")) != MX_OK) return st;
+    if ((st = check_device_ptr(Aq, "Aq")) != MX_OK) return st;
+    if ((st = check_device_ptr(s_a, "s_a")) != MX_OK) return st;
+    if ((st = check_device_ptr(Y, "Y")) != MX_OK) return st;
+    if (partials && (st = check_device_ptr(partials, "partials")) != MX_OK) return st;
+    if (!aligned16(blob) || !aligned16(Aq)) return fail(MX_ERR_ALIGNMENT, "blob and Aq must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(s_a) % 2 || reinterpret_cast<uintptr_t>(Y) % 2)
+        return fail(MX_ERR_ALIGNMENT, "s_a and Y must be 2-byte aligned");
+    cudaError_t e = mx::launch_bw_gemm(*L, static_cast<const uint8_t*>(blob), Aq, static_cast<const __half*>(s_a), M,
+                                       static_cast<__half*>(Y), ldy, partials, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MX_OK : cuda_fail(e, "bw gemm");
 }
 
 mx_status mx_copy_mapped(void* dst, const void* src, size_t bytes, void* stream) {
