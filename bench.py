@@ -72,6 +72,9 @@ def parse():
     p.add_argument("--search", action="store_true",
                    help="the global precision search: channel saliency of one Llama-3-8B decoder "
                         "layer's seven linears, then the top-10%% choice over all 32 layers' rows")
+    p.add_argument("--blockwise", action="store_true",
+                   help="block-wise bit widths: the decode GEMM on Llama-3-8B up (K 4096, N 14336) "
+                        "at M 1, 4, 16 against HBM, widths {2, 3, 4, 8}")
     a = p.parse_args()
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -438,6 +441,70 @@ def run_search(a):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ block-wise bit widths
+BW_TABLE = (2, 3, 4, 8)
+BW_PROBS = (0.25, 0.25, 0.40, 0.10)       # about 3.6 bits per weight
+
+
+def run_blockwise(a):
+    """Times mx_bw_gemm on the Llama-3-8B up projection with seed-drawn block widths
+    (table {2, 3, 4, 8}, probabilities 0.25 / 0.25 / 0.40 / 0.10), M = 1, 4 and 16, over
+    rotated copies of the blob (>= 4x L2), with events on the launching stream after
+    warm-up.  Algorithmic bytes: model.bw_gemm_bytes."""
+    import torch
+    import oracle
+    from mixed_precision_quantized_mx_b200 import binding as mx
+    from mixed_precision_quantized_mx_b200 import build as mxbuild
+    from mixed_precision_quantized_mx_b200 import inputs, model
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    mxbuild.build()
+    peaks = load_peaks()
+    K, N = inputs.SHAPES["llama3-8b-up"]
+    rng = np.random.default_rng(a.seed)
+    codes = inputs.block_codes(rng, N, K, BW_PROBS)
+    meta = oracle.pack_block_codes(codes)
+    L = mx.mx_bw_layout_init(N, K, BW_TABLE, meta)
+    W = torch.from_numpy(inputs.weights(rng, N, K, outlier_frac=0.001)).to(dev)
+    blob0 = torch.empty(L.total_bytes, dtype=torch.uint8, device=dev)
+    mx.mx_bw_pack(L, meta, W, blob0)
+    torch.cuda.synchronize()
+    del W
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = int(min(16, max(2, math.ceil(4 * l2 / L.total_bytes))))
+    blobs = [blob0] + [blob0.clone() for _ in range(R - 1)]
+    s = torch.cuda.Stream(dev)
+    for M in (1, 4, 16):
+        X = torch.from_numpy(inputs.activations(rng, M, K, int(round(0.01 * K)))).to(dev)
+        Aq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sa = torch.empty(M, dtype=torch.float16, device=dev)
+        mx.mx_quant_act(X, Aq, sa)
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        steps = a.steps or 200
+        with torch.cuda.stream(s):
+            for i in range(max(a.warmup, R)):
+                mx.mx_bw_gemm(L, blobs[i % R], Aq, sa, Y, stream=s)
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(s)
+        with torch.cuda.stream(s):
+            for i in range(steps):
+                mx.mx_bw_gemm(L, blobs[i % R], Aq, sa, Y, stream=s)
+        ev1.record(s)
+        torch.cuda.synchronize()
+        us = ev0.elapsed_time(ev1) * 1e3 / steps
+        byts = model.bw_gemm_bytes(M, N, K, L.code_bytes)
+        gbs = byts / us / 1e3
+        print(json.dumps({
+            "metric": "blockwise_gemm_bandwidth", "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1,
+            "steps": steps, "warmup": a.warmup, "us_per_call": round(us, 3), "M": M,
+            "bits_per_weight": round(L.code_bytes * 8 / (N * K), 3), "dtype": "int8 (dp4a)", "data": "synthetic",
+            "config": {"workload": "llama3-8b up K=4096 N=14336, widths %s" % (BW_TABLE,), "rotated_copies": R},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None}}), flush=True)
+
+
 # ------------------------------------------------------------------ main arm
 def main():
     a = parse()
@@ -447,6 +514,8 @@ def main():
         return run_sweep(a)
     if a.search:
         return run_search(a)
+    if a.blockwise:
+        return run_blockwise(a)
 
     import torch
     import torch.distributed as dist

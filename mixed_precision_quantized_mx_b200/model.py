@@ -53,3 +53,17 @@ def step_bytes(M: int, N: int, K: int, group: int, n8: int, in_bytes: int = 2) -
 def linear_bytes(M: int, N: int, K: int, group: int, n8: int, in_bytes: int = 2) -> float:
     """The layer end to end: X in, packed weights, Y out."""
     return weight_bytes(N, K, group, n8) + float(in_bytes) * M * K + 2.0 * M * N
+
+
+def bw_weight_bytes(N: int, K: int, code_bytes: int) -> float:
+    """Block-wise bit widths: the blocks' codes (code_bytes, b / 8 bytes per weight), an fp16
+    scale and a uint8 zero per (row, 128-column block), the 2-bit block codes and the
+    uint32 block offsets."""
+    KB = K // 128
+    NB = (N + 63) // 64
+    return code_bytes + 3 * N * KB + (NB * KB + 3) // 4 + 4 * (NB * KB + 1)
+
+
+def bw_gemm_bytes(M: int, N: int, K: int, code_bytes: int) -> float:
+    """One block-wise GEMM call: weights, int8 activations with fp16 token scales, fp16 Y."""
+    return bw_weight_bytes(N, K, code_bytes) + M * K + 2 * M + 2 * M * N

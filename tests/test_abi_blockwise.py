@@ -75,3 +75,15 @@ def test_pack_and_gemm_host_checks_before_any_launch(lib, orc):
         setattr(bad, field, value)
         assert lib.mx_bw_gemm(ctypes.byref(bad), P, P, P, 0, P, 100, None, None) == 1, field
         assert lib.mx_bw_pack(ctypes.byref(bad), mx._host_bytes(meta), P, 0, 256, P, None) == 1, field
+
+
+def test_byte_model_counts_every_section_of_the_blob(lib, orc):
+    # the algorithmic weight bytes are the blob without its 64-byte header and alignment
+    from mixed_precision_quantized_mx_b200 import model
+    rng = np.random.default_rng(9)
+    for N, K in ((4096, 4096), (14336, 4096), (130, 640)):
+        codes = inputs.block_codes(rng, N, K, (0.25, 0.25, 0.4, 0.1))
+        L = mx.mx_bw_layout_init(N, K, [2, 3, 4, 8], orc.pack_block_codes(codes))
+        wb = model.bw_weight_bytes(N, K, L.code_bytes)
+        assert 64 <= L.total_bytes - wb <= 64 + 4 * 15
+        assert model.bw_gemm_bytes(3, N, K, L.code_bytes) == wb + 3 * K + 6 + 6 * N
