@@ -22,15 +22,15 @@
  *     are float16 (section 3.3)
  *   - restricted symmetric range +-(2^(b-1) - 1) (SBVR page, section 2.1)
  *
- * Readings where the text is silent (each one is listed in the design notes):
- *   R1 symmetric range [-127, 127], s = absmax / 127
- *   R3 the 4-bit range [lo, hi] always contains 0, so z fits uint4
- *   R4 round() is round-half-to-even
- *   R5 scales are computed in fp32, rounded to fp16 (nearest-even) and the
+ * Readings where the text is silent:
+ *   - symmetric range [-127, 127], s = absmax / 127
+ *   - the 4-bit range [lo, hi] always contains 0, so z fits uint4
+ *   - round() is round-half-to-even
+ *   - scales are computed in fp32, rounded to fp16 (nearest-even) and the
  *      ROUNDED fp16 value is the one used to quantize
- *   R7 a zero (or fp16-underflowed) scale becomes 1.0; an fp16 overflow
+ *   - a zero (or fp16-underflowed) scale becomes 1.0; an fp16 overflow
  *      saturates to 65504
- *   R10 fp32 quantization decisions: amax/127, (hi-lo)/15, x/s, -lo/s are
+ *   - fp32 quantization decisions: amax/127, (hi-lo)/15, x/s, -lo/s are
  *      each one IEEE fp32 operation; everything after the integer codes is
  *      exact integer (int64) or fp64 arithmetic here
  *
@@ -107,8 +107,8 @@ double mxo_fp16_value(uint16_t h)
 static float scale_to_fp16(float s32, uint16_t *bits)
 {
     double s16 = mxo_fp16_round((double)s32);
-    if (s16 > 65504.0) s16 = 65504.0;          /* R7 saturation */
-    if (s16 == 0.0) s16 = 1.0;                 /* R7 degenerate group */
+    if (s16 > 65504.0) s16 = 65504.0;          /* fp16 overflow saturates */
+    if (s16 == 0.0) s16 = 1.0;                 /* degenerate group */
     *bits = mxo_fp16_bits_of(s16);
     return (float)s16;                         /* exact */
 }

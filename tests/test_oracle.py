@@ -369,7 +369,7 @@ def test_gemm_group_activations(orc):
     assert err_group < err_token
 
 
-# --------------------------------------------------------------- global saliency (NEXT-2)
+# --------------------------------------------------------------- global saliency (precision search)
 def _asym4_grid_rows(rng, N, K, g):
     """W whose every group is exactly on its 4-bit asymmetric grid (codes 0 and 15 present)."""
     W = np.zeros((N, K))
