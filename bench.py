@@ -475,6 +475,21 @@ def run_blockwise(a):
     R = int(min(16, max(2, math.ceil(4 * l2 / L.total_bytes))))
     blobs = [blob0] + [blob0.clone() for _ in range(R - 1)]
     s = torch.cuda.Stream(dev)
+    cpu = None
+    if not a.no_cpu_baseline:
+        # the oracle's pack + GEMM of M = 1 on the first 256 rows, scaled to GB/s like the GPU line
+        rows = 256
+        Wc = inputs.weights(rng, rows, K)
+        bc = oracle.pack_blockwise(Wc, codes[:rows // 64], BW_TABLE)
+        Ac, sc = oracle.quant_act(inputs.activations(rng, 1, K, 4, dtype=np.float32))
+        reps, t0 = 0, time.perf_counter()
+        while reps == 0 or time.perf_counter() - t0 < 3.0:
+            oracle.gemm_blockwise(Ac, sc, bc)
+            reps += 1
+        dt = (time.perf_counter() - t0) / reps
+        cb = mx.mx_bw_layout_init(rows, K, BW_TABLE, oracle.pack_block_codes(codes[:rows // 64])).code_bytes
+        cpu = {"value": round(model.bw_gemm_bytes(1, rows, K, cb) / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
+               "kind": "oracle", "sample": "M=1 GEMM over the first %d rows, %d calls in 3 s" % (rows, reps)}
     for M in (1, 4, 16):
         X = torch.from_numpy(inputs.activations(rng, M, K, int(round(0.01 * K)))).to(dev)
         Aq = torch.empty((M, K), dtype=torch.int8, device=dev)
@@ -502,7 +517,8 @@ def run_blockwise(a):
             "bits_per_weight": round(L.code_bytes * 8 / (N * K), 3), "dtype": "int8 (dp4a)", "data": "synthetic",
             "config": {"workload": "llama3-8b up K=4096 N=14336, widths %s" % (BW_TABLE,), "rotated_copies": R},
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None}}), flush=True)
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None},
+            "cpu_baseline": cpu}), flush=True)
 
 
 # ------------------------------------------------------------------ main arm
