@@ -46,7 +46,10 @@ WORKLOADS = {
     "llama3-70b-up-m4096": (4096, 8192, 28672),
     "llama3-70b-down-m4096": (4096, 28672, 8192),
 }
-DEFAULT_WORKLOAD = "llama3-8b-qo-m1"
+DEFAULT_WORKLOAD = "llama3-70b-up-m4096"
+# lines measured after the named workload in the same run: the same weights at another M
+SECONDARY = {"llama3-70b-up-m4096": ("llama3-70b-up-m1",),
+             "llama3-70b-down-m4096": ("llama3-70b-down-m1",)}
 HBM_BOUND_MAX_M = 128        # below the ~150-token ridge the step is bound by HBM
 
 
@@ -65,6 +68,8 @@ def parse():
                    help="activation scales: 0 one per token; the weight group: one per token and group")
     p.add_argument("--impl", default="mx", choices=["mx", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-secondary", action="store_true",
+                   help="only the named workload (not the decode line measured after it)")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--sweep", action="store_true",
                    help="the K = N = 8192 sweep over 8-bit row fraction, M and group size: one JSON "
@@ -93,6 +98,10 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {1: "gemm_decode.cu", 2: "gemm_tc.cu", 3: "gemm_rows.cu", 4: "gemm_tc2.cu"}
+KERNEL_NAMES = {1: "gemm_decode_kernel (cluster split-K, CUDA cores)",
+                2: "gemm_tc_kernel (tcgen05)",
+                3: "gemm_rows_kernel (whole rows per CTA, CUDA cores)",
+                4: "gemm_tc2_kernel (tcgen05 on CTA pairs)"}
 
 
 def src_digest(path: int) -> str:
@@ -179,18 +188,57 @@ def oracle_step_sample(lay, budget_s: float = 0.5):
     return m, n, f"{budget} random (token, row) outputs of {M}x{N}"
 
 
-def time_oracle(lay, canonical, steps: int, min_seconds: float = 0.0, act_group: int = 0):
-    """Run the oracle's quantize + sampled GEMM; return (seconds per step, sample, fraction)."""
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def time_oracle(lay, canonical, steps: int, min_seconds: float = 0.0, act_group: int = 0,
+                threads: int = 1):
+    """Run the oracle's quantize + sampled GEMM; return (seconds per step, sample, fraction,
+    steps done).  With threads > 1 the sampled outputs are cut into `threads` disjoint
+    slices computed at the same time (the oracle's C routine runs with the interpreter
+    lock released), the quantizer once per step; the oracle's arithmetic is unchanged."""
     import oracle
-    m, n, desc = oracle_step_sample(lay)
+    from concurrent.futures import ThreadPoolExecutor
+    m, n, desc = oracle_step_sample(lay, budget_s=0.5 * threads)
     frac = len(m) / (lay.M * lay.N)
     X = lay.X.astype(np.float32)
+    cuts = np.linspace(0, len(m), threads + 1).astype(int)
+    pool = ThreadPoolExecutor(threads) if threads > 1 else None
     done, t0 = 0, time.perf_counter()
     while done < steps or time.perf_counter() - t0 < min_seconds:
         Aq, sa = oracle.quant_act(X, act_group=act_group)
-        oracle.gemm(Aq, sa, canonical, act_group=act_group, pairs=(m, n))
+        if pool is None:
+            oracle.gemm(Aq, sa, canonical, act_group=act_group, pairs=(m, n))
+        else:
+            futs = [pool.submit(oracle.gemm, Aq, sa, canonical, act_group, (m[cuts[i]:cuts[i + 1]],
+                                                                            n[cuts[i]:cuts[i + 1]]))
+                    for i in range(threads)]
+            for f in futs:
+                f.result()
         done += 1
-    return (time.perf_counter() - t0) / done, desc, frac, done
+    sec = (time.perf_counter() - t0) / done
+    if pool is not None:
+        pool.shutdown()
+    return sec, desc, frac, done
+
+
+def cpu_baseline(lay, canonical, unit: str, act_group: int, seconds: float = 10.0) -> dict:
+    """The oracle timed on this host's cores on a bounded sample of one step: all cores
+    (the reported value) and one core."""
+    units = step_units(lay.M, lay.K, lay.N, lay.group, lay.n8, unit)
+    cores = host_cores()
+    sec, desc, frac, done = time_oracle(lay, canonical, 1, min_seconds=seconds, act_group=act_group,
+                                        threads=cores)
+    sec1, desc1, frac1, done1 = time_oracle(lay, canonical, 1, min_seconds=seconds / 2, act_group=act_group)
+    return {"value": units * frac / sec, "unit": unit, "cores": cores, "kind": "oracle",
+            "sample": f"{done} steps on {cores} threads, each: quantize {lay.M}x{lay.K} activations + "
+                      f"{desc}, cut into {cores} slices",
+            "single_thread": {"value": units * frac1 / sec1, "unit": unit, "cores": 1,
+                              "sample": f"{done1} steps, each: quantize + {desc1}"}}
 
 
 def max_over_ranks(x: float, device=None) -> float:
@@ -220,6 +268,9 @@ def step_units(M, K, N, g, n8, unit):
 
 
 def run_reference(a):
+    """The oracle on this host's cores, on the same workload, metric and unit as the main
+    arm: each step quantizes the step's activations and computes a bounded sample of its
+    outputs, the sample cut into one slice per core."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -229,10 +280,12 @@ def run_reference(a):
     lay = inputs.llama_layer(M, K, N, a.frac8, a.group, seed=a.seed)
     can = oracle.pack(lay.W, lay.is8, lay.group)
     unit = "GB/s" if M <= HBM_BOUND_MAX_M else "TOPS"
-    time_oracle(lay, can, a.warmup, act_group=a.act_group)
-    sec, desc, frac, done = time_oracle(lay, can, a.steps or 5, act_group=a.act_group)
+    cores = host_cores()
+    time_oracle(lay, can, a.warmup, act_group=a.act_group, threads=cores)
+    sec, desc, frac, done = time_oracle(lay, can, a.steps or 5, act_group=a.act_group, threads=cores)
     value = step_units(M, K, N, a.group, lay.n8, unit) * frac / sec
-    sample = f"each step: quantize {M}x{K} activations + {desc} (fraction {frac:.3g} of the step)"
+    sample = (f"each step: quantize {M}x{K} activations + {desc} (fraction {frac:.3g} of the step), "
+              f"cut into {cores} slices on {cores} threads")
     line = {
         "metric": METRIC, "value": value, "unit": unit, "impl": "reference",
         "n_gpus": a.gpus, "steps": done, "warmup": a.warmup, "ms_per_step": sec * 1e3 / frac,
@@ -240,7 +293,7 @@ def run_reference(a):
         "data": "synthetic",
         "config": {"workload": a.workload, "M": M, "K": K, "N": N, "group": a.group,
                    "frac8": a.frac8, "n8": lay.n8, "act_group": a.act_group},
-        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -449,8 +502,9 @@ BW_PROBS = (0.25, 0.25, 0.40, 0.10)       # about 3.6 bits per weight
 def run_blockwise(a):
     """Times mx_bw_gemm on the Llama-3-8B up projection with seed-drawn block widths
     (table {2, 3, 4, 8}, probabilities 0.25 / 0.25 / 0.40 / 0.10), M = 1, 4 and 16, over
-    rotated copies of the blob (>= 4x L2), with events on the launching stream after
-    warm-up.  Algorithmic bytes: model.bw_gemm_bytes."""
+    rotated copies of the blob (at least 4x L2, the multiple is in the line), with events
+    on the launching stream after warm-up.  Before timing, each M's Y is checked against
+    the oracle on 512 sampled outputs.  Algorithmic bytes: model.bw_gemm_bytes."""
     import torch
     import oracle
     from mixed_precision_quantized_mx_b200 import binding as mx
@@ -466,13 +520,16 @@ def run_blockwise(a):
     codes = inputs.block_codes(rng, N, K, BW_PROBS)
     meta = oracle.pack_block_codes(codes)
     L = mx.mx_bw_layout_init(N, K, BW_TABLE, meta)
-    W = torch.from_numpy(inputs.weights(rng, N, K, outlier_frac=0.001)).to(dev)
+    Wh = inputs.weights(rng, N, K, outlier_frac=0.001)
+    W = torch.from_numpy(Wh).to(dev)
     blob0 = torch.empty(L.total_bytes, dtype=torch.uint8, device=dev)
     mx.mx_bw_pack(L, meta, W, blob0)
     torch.cuda.synchronize()
     del W
+    bref = oracle.pack_blockwise(Wh, codes, BW_TABLE)
+    del Wh
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    R = int(min(16, max(2, math.ceil(4 * l2 / L.total_bytes))))
+    R = int(max(2, math.ceil(4 * l2 / L.total_bytes)))
     blobs = [blob0] + [blob0.clone() for _ in range(R - 1)]
     s = torch.cuda.Stream(dev)
     cpu = None
@@ -496,6 +553,18 @@ def run_blockwise(a):
         sa = torch.empty(M, dtype=torch.float16, device=dev)
         mx.mx_quant_act(X, Aq, sa)
         Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        # the result is checked against the oracle on sampled outputs before anything is timed
+        mx.mx_bw_gemm(L, blob0, Aq, sa, Y, stream=s)
+        torch.cuda.synchronize()
+        Ao, so = oracle.quant_act(X.cpu().numpy().astype(np.float32))
+        pm = rng.integers(0, M, 512).astype(np.int32)
+        pn = rng.integers(0, N, 512).astype(np.int32)
+        _, yt, _, _ = oracle.gemm_blockwise(Ao, so, bref, pairs=(pm, pn))
+        yg = Y.cpu().numpy()[pm, pn].astype(np.float64)
+        rms = float(np.sqrt(np.mean(yt ** 2)))
+        if not (np.all(np.abs(yg - yt) <= 2e-3 * np.abs(yt) + 2e-3 * rms)
+                and np.linalg.norm(yg - yt) <= 2e-3 * np.linalg.norm(yt)):
+            raise SystemExit(f"blockwise GEMM at M={M} differs from the oracle on sampled outputs")
         steps = a.steps or 200
         with torch.cuda.stream(s):
             for i in range(max(a.warmup, R)):
@@ -515,48 +584,33 @@ def run_blockwise(a):
             "metric": "blockwise_gemm_bandwidth", "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1,
             "steps": steps, "warmup": a.warmup, "us_per_call": round(us, 3), "M": M,
             "bits_per_weight": round(L.code_bytes * 8 / (N * K), 3), "dtype": "int8 (dp4a)", "data": "synthetic",
-            "config": {"workload": "llama3-8b up K=4096 N=14336, widths %s" % (BW_TABLE,), "rotated_copies": R},
+            "config": {"workload": "llama3-8b up K=4096 N=14336, widths %s" % (BW_TABLE,), "rotated_copies": R,
+                       "l2": "blob rotates over %d copies (%.0f MB, %.1fx the %.0f MB L2)" % (
+                           R, R * L.total_bytes / 1e6, R * L.total_bytes / l2, l2 / 1e6),
+                       "checked": "Y within 2e-3 of the oracle on 512 sampled outputs before timing"},
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None},
             "cpu_baseline": cpu}), flush=True)
 
 
 # ------------------------------------------------------------------ main arm
-def main():
-    a = parse()
-    if a.impl == "reference":
-        return run_reference(a)
-    if a.sweep:
-        return run_sweep(a)
-    if a.search:
-        return run_search(a)
-    if a.blockwise:
-        return run_blockwise(a)
+TIMED_REPEATS = 5            # the K-step timed region is repeated; the median is reported
 
+
+def measure_layer(a, lay, workload: str, dev, rank: int, world: int, l2: int, peaks: dict) -> dict:
+    """One workload through mx_linear: pack (offline, timed on its own), then W warm-up
+    steps and TIMED_REPEATS timed regions of K steps replayed from CUDA graphs over rotated
+    copies (>= 4x L2); the dominant kernel timed live on its stream for the roofline; and
+    the end-to-end pass through MixedPrecisionLinear.graphed (pinned host X in, Y out)."""
     import torch
     import torch.distributed as dist
     from mixed_precision_quantized_mx_b200 import binding as mx
-    from mixed_precision_quantized_mx_b200 import build as mxbuild
-    from mixed_precision_quantized_mx_b200 import inputs, model
+    from mixed_precision_quantized_mx_b200 import model
     from mixed_precision_quantized_mx_b200.layer import MixedPrecisionLinear
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != a.gpus:
-        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
-    mxbuild.build()
-    mx.lib()
-
-    M, K, N = WORKLOADS[a.workload]
-    g = a.group
+    M, K, N = lay.M, lay.K, lay.N
+    g = lay.group
     ag = a.act_group
-    lay = inputs.llama_layer(M, K, N, a.frac8, g, seed=rank_seed(a.seed, rank))
     n8 = lay.n8
     L = mx.mx_layout_init(N, K, g, n8)
     unit = "GB/s" if M <= HBM_BOUND_MAX_M else "TOPS"
@@ -581,7 +635,6 @@ def main():
     del Wd
 
     # ---- rotated copies beyond L2
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     per_step = model.linear_bytes(M, N, K, g, n8, 2)
     R = int(min(64, max(2, math.ceil(4 * l2 / per_step))))
     R = max(2, min(R, int(20e9 // max(per_step, 1))))
@@ -599,7 +652,7 @@ def main():
     def step(i):
         mx.mx_linear(L, blobs[i], Xs[i], Ys[i], workspace=ws, path=a.path, act_group=ag)
 
-    gws_bytes = mx.mx_gemm_workspace_size(L, M, path=a.path)     # split sums of path 4, if any
+    gws_bytes = mx.mx_gemm_workspace_size(L, M, path=a.path)     # split sums of a K split, if any
     gws = torch.empty(max(gws_bytes, 16), dtype=torch.uint8, device=dev)
 
     def gemm_only(i):
@@ -651,7 +704,7 @@ def main():
     torch.cuda.synchronize()
 
     lead = torch.empty(int(2 * l2) // 4, dtype=torch.int32, device=dev)
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(dev.index)
     # sustained run of the same step graph (clock reference even for short timed regions)
     sampler.start()
     t_load0 = time.perf_counter()
@@ -662,26 +715,29 @@ def main():
 
     replay_steps(qw, g_wrem)                       # W warm-up steps
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    # an L2-sized fill ahead of the start event keeps the device busy while the host
-    # submits the step graphs, so the timed region holds the steps and not the
-    # submission gap; it also leaves L2 holding none of the step's inputs
-    with torch.cuda.stream(s):
-        lead.fill_(1)
+    times = []
     t_time0 = time.perf_counter()
-    ev0.record(s)
-    with torch.cuda.stream(s):
-        replay_steps(q, g_rem)
-    ev1.record(s)
-    torch.cuda.synchronize()
+    for _ in range(TIMED_REPEATS):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # an L2-sized fill ahead of the start event keeps the device busy while the host
+        # submits the step graphs, so the timed region holds the steps and not the
+        # submission gap; it also leaves L2 holding none of the step's inputs
+        with torch.cuda.stream(s):
+            lead.fill_(1)
+        ev0.record(s)
+        with torch.cuda.stream(s):
+            replay_steps(q, g_rem)
+        ev1.record(s)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        times.append(max_over_ranks(ev0.elapsed_time(ev1), dev))
     t_time1 = time.perf_counter()
-    if world > 1:
-        dist.barrier()
     sampler.stop()
-    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
+    ms = float(np.median(times))
     units_per_step = step_units(M, K, N, g, n8, unit)
     value = units_per_step * K_steps * world / (ms / 1e3)
 
@@ -699,7 +755,6 @@ def main():
     d1.record(s)
     torch.cuda.synchronize()
     gemm_ms = d0.elapsed_time(d1) / (3 * nd)
-    peaks = load_peaks()
     if bound == "hbm":
         algo = model.linear_bytes(M, N, K, g, n8, 2) if fused else model.gemm_bytes(M, N, K, g, n8)
         achieved = algo / (gemm_ms / 1e3) / 1e9
@@ -713,17 +768,13 @@ def main():
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if os.path.exists(tfile):
-        rec = json.load(open(tfile)).get(a.workload)
+        rec = json.load(open(tfile)).get(workload)
         if (rec and rec.get("src_digest") == src_digest(path_used) and rec.get("path") == path_used
                 and rec.get("fused", False) == fused):
             traffic = rec["dram_bytes_per_launch"]
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": {1: "gemm_decode_kernel (cluster split-K, CUDA cores)",
-                           2: "gemm_tc_kernel (tcgen05)",
-                           3: "gemm_rows_kernel (whole rows per CTA, CUDA cores)",
-                           4: "gemm_tc2_kernel (tcgen05 on CTA pairs)"}[path_used]
-                          + (", activation quantizer fused" if fused else ""),
+                "kernel": KERNEL_NAMES[path_used] + (", activation quantizer fused" if fused else ""),
                 "algorithmic_per_launch": algo, "launch_ms": gemm_ms,
                 "peak_source": (f"{peaks['source']} HBM copy" if bound == "hbm" else
                                 f"{peaks['source']} bf16 cuBLAS burst x 2 (nominal int8/bf16 ratio)")}
@@ -733,10 +784,13 @@ def main():
     Xpin = Xh.pin_memory()
     Ypin = torch.empty((M, N), dtype=torch.float16).pin_memory()
     runner = layer.graphed(Xpin, Ypin, path=a.path, act_group=ag)   # H2D, mx_linear, D2H: one graph
-    Ke = max(20, min(K_steps, 5000))
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
     for _ in range(3):
         runner.replay()
     torch.cuda.synchronize()
+    est_e2e = (time.perf_counter() - t0) / 3
+    Ke = max(20, min(K_steps, 5000, int(2.0 / max(est_e2e, 1e-7))))
     if world > 1:
         dist.barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -749,42 +803,104 @@ def main():
     e2e = {"value": units_per_step * world / (e2e_ms / 1e3), "unit": unit,
            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
            "ms_per_step": e2e_ms,
-           "api": "MixedPrecisionLinear.graphed: pinned X read in by a copy kernel, mx_linear, Y written to pinned host memory by a copy kernel, one graph per step"}
+           "api": "MixedPrecisionLinear.graphed: pinned X read in by a copy kernel, mx_linear, Y written "
+                  "to pinned host memory by a copy kernel, one graph per step"}
 
     clocks = sampler.summary(t_time0, t_time1) or sampler.summary(t_load0, t_load1)
     if clocks is not None and "error" not in clocks:
-        clocks["window"] = ("timed region" if sampler.summary(t_time0, t_time1)
-                            else "sustained replay of the same step graph just before the timed region")
-
-    cpu = None
-    if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        import oracle
-        can = oracle.pack(lay.W, lay.is8, g)
-        sec, desc, frac, done = time_oracle(lay, can, 1, min_seconds=10.0, act_group=ag)
-        cpu = {"value": units_per_step * frac / sec, "unit": unit, "cores": 1, "kind": "oracle",
-               "sample": f"{done} steps, each: quantize {M}x{K} activations + {desc}"}
-
+        clocks["window"] = ("timed regions" if sampler.summary(t_time0, t_time1)
+                            else "sustained replay of the same step graph just before the timed regions")
     # fused kernel, or activation quantizer + GEMM (+ the reduction of a K split)
     kernels_per_step = 1 if fused else 2 + (1 if gws_bytes > 0 else 0)
-    line = {
-        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K_steps,
-        "warmup": a.warmup, "ms_per_step": ms / K_steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": a.workload, "M": M, "K": K, "N": N, "group": g, "frac8": a.frac8,
-                   "act_group": ag,
-                   "n8": n8, "path": path_used, "fused_quantizer": fused,
+    out = {
+        "value": value, "unit": unit, "ms_per_step": ms / K_steps, "steps": K_steps,
+        "repeats_ms": [round(t, 4) for t in times],
+        "config": {"workload": workload, "M": M, "K": K, "N": N, "group": g, "frac8": a.frac8,
+                   "act_group": ag, "n8": n8, "path": path_used, "fused_quantizer": fused,
                    "l2": f"inputs rotate over {R} copies ({R * per_step / 1e6:.0f} MB >= 4x the "
                          f"{l2 / 1e6:.0f} MB L2); no flush",
-                   "graphs": "timed steps replayed from CUDA graphs"},
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                   "graphs": "timed steps replayed from CUDA graphs",
+                   "timing": f"median of {TIMED_REPEATS} timed regions of K steps"},
+        "roofline": roofline, "e2e": e2e,
         "gpu_launches": kernels_per_step * K_steps, "clocks": clocks,
         "tops": model.gemm_ops(M, N, K) * K_steps * world / (ms / 1e3) / 1e12,
         "gbs": model.linear_bytes(M, N, K, g, n8, 2) * K_steps * world / (ms / 1e3) / 1e9,
         "pack": {"ms": pack_ms, "weights_gb_per_s": (N * K * 4) / (pack_ms / 1e3) / 1e9},
     }
+    del g_full, g_rem, g_wrem, g_gemm, runner
+    del blobs, Xs, Aqs, sas, Ys, ws, gws, lead
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        return run_reference(a)
+    if a.sweep:
+        return run_sweep(a)
+    if a.search:
+        return run_search(a)
+    if a.blockwise:
+        return run_blockwise(a)
+
+    import torch
+    import torch.distributed as dist
+    from mixed_precision_quantized_mx_b200 import binding as mx
+    from mixed_precision_quantized_mx_b200 import build as mxbuild
+    from mixed_precision_quantized_mx_b200 import inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    mxbuild.build()
+    mx.lib()
+    peaks = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    M, K, N = WORKLOADS[a.workload]
+    lay = inputs.llama_layer(M, K, N, a.frac8, a.group, seed=rank_seed(a.seed, rank))
+    primary = measure_layer(a, lay, a.workload, dev, rank, world, l2, peaks)
+    secondary = []
+    if not a.no_secondary:
+        for name in SECONDARY.get(a.workload, ()):
+            M2, K2, N2 = WORKLOADS[name]
+            assert (K2, N2) == (K, N)
+            # the same weights and 8-bit rows, a batch of M2 tokens of the same distribution
+            rng = np.random.default_rng(rank_seed(a.seed, rank) + 7)
+            lay2 = inputs.Layer(inputs.activations(rng, M2, K, int(round(0.01 * K))), lay.W, lay.is8,
+                                lay.group, name)
+            sec = measure_layer(a, lay2, name, dev, rank, world, l2, peaks)
+            secondary.append((lay2, sec))
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        import oracle
+        can = oracle.pack(lay.W, lay.is8, lay.group)
+        cpu = cpu_baseline(lay, can, primary["unit"], a.act_group)
+        for lay2, sec in secondary:
+            sec["cpu_baseline"] = cpu_baseline(lay2, can, sec["unit"], a.act_group, seconds=6.0)
+
+    line = {
+        "metric": METRIC, "value": primary["value"], "unit": primary["unit"], "n_gpus": world,
+        "steps": primary["steps"], "warmup": a.warmup, "ms_per_step": primary["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic", "config": primary["config"], "roofline": primary["roofline"],
+        "cpu_baseline": cpu, "e2e": primary["e2e"], "gpu_launches": primary["gpu_launches"],
+        "clocks": primary["clocks"], "tops": primary["tops"], "gbs": primary["gbs"],
+        "repeats_ms": primary["repeats_ms"], "pack": primary["pack"],
+        "secondary": [dict(sec, metric=METRIC, n_gpus=world, warmup=a.warmup) for _, sec in secondary],
+    }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g_full, g_rem, g_wrem, g_gemm
     if world > 1:
         dist.destroy_process_group()
 

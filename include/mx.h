@@ -283,11 +283,14 @@ mx_status mx_linear(const mx_layout* L, const void* blob, const void* X, mx_dtyp
  * mx_linear_noalloc -- mx_linear with no workspace argument and no allocation.
  * The method has no counterpart of this call; it exists for callers that
  * cannot hand out device memory.  Where mx_linear needs scratch (the
- * two-kernel path: Aq of M*K bytes and s_a of 2*M bytes, each rounded up to 16
- * bytes, as mx_linear_workspace_size reports), this call uses a file-scope
- * device array of MX_NOALLOC_SCRATCH_BYTES bytes instead.  Its address on the
- * calling thread's current device is looked up with cudaGetSymbolAddress on
- * the first call that needs it on that device and kept for later calls.
+ * two-kernel path: Aq of M*K bytes, then s_a of 2*M bytes with one scale per
+ * token or 2*M*(K/g) bytes with act_group = g, each rounded up to 16 bytes, as
+ * mx_linear_workspace_size reports), this call uses a file-scope device array
+ * of MX_NOALLOC_SCRATCH_BYTES bytes instead.  Its address in the calling
+ * thread's current device context is looked up with cudaGetSymbolAddress on
+ * the first call that needs it on that device and kept for later calls; it is
+ * looked up again when the device's context has changed since (after
+ * cudaDeviceReset, for example).
  *   Arguments as mx_linear, less workspace and ws_bytes.
  * Nothing in the array has to start at zero: the quantizer writes every byte
  * of it that the GEMM then reads.  The call never allocates or frees device

@@ -240,9 +240,9 @@ NOALLOC_SCRATCH_BYTES = 4 << 20      # MX_NOALLOC_SCRATCH_BYTES
 
 def mx_linear_noalloc(L: Layout, blob: torch.Tensor, X: torch.Tensor, Y: torch.Tensor, path: int = 0,
                       split: int = 0, debug_partials: torch.Tensor | None = None,
-                      status: torch.Tensor | None = None, stream=None) -> None:
+                      status: torch.Tensor | None = None, act_group: int = 0, stream=None) -> None:
     assert X.dim() == 2 and X.stride(1) == 1
-    o = _opts(path, split, debug_partials, status)
+    o = _opts(path, split, debug_partials, status, act_group=act_group)
     _check(lib().mx_linear_noalloc(ctypes.byref(L), _ptr(blob), _ptr(X), _dtype_code(X), X.shape[0],
                                    X.stride(0), _ptr(Y), Y.stride(0), ctypes.byref(o), _stream(stream)),
            "mx_linear_noalloc")

@@ -667,27 +667,59 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[MX_NOALLOC_SCRATCH_BY
 namespace {
 
 constexpr int kNoAllocDevices = 64;
-void* g_noalloc_addr[kNoAllocDevices] = {};
+struct NoAllocSlot {
+    CUcontext ctx;     // the context the address belongs to
+    void* addr;
+};
+NoAllocSlot g_noalloc[kNoAllocDevices] = {};
 std::mutex g_noalloc_mu;
 
-// the array's address on the current device, looked up once per device
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// the driver's cuCtxGetCurrent, found once through the runtime
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// The array's address in the current device's context.  It is looked up once per
+// device and context: the first call on a device (and the first after that device's
+// primary context was torn down and made again, by cudaDeviceReset for example)
+// does the lookup; later calls reuse it.
 mx_status noalloc_scratch(void** addr) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= kNoAllocDevices)
         return fail(MX_ERR_UNSUPPORTED, "device %d beyond the %d this call tracks", dev, kNoAllocDevices);
+    // cudaSetDevice makes the device's primary context current (creating it if needed)
+    if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+    CUcontext ctx = nullptr;
+    CtxGetCurrentFn get = ctx_get_current_fn();
+    if (get == nullptr || get(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+        return fail(MX_ERR_CUDA, "no current CUDA context on device %d", dev);
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_addr[dev] == nullptr) {
+    NoAllocSlot& slot = g_noalloc[dev];
+    if (slot.addr == nullptr || slot.ctx != ctx) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) {
             cudaGetLastError();
             return cuda_fail(e, "cudaGetSymbolAddress of the scratch array");
         }
-        g_noalloc_addr[dev] = p;
+        slot.ctx = ctx;
+        slot.addr = p;
     }
-    *addr = g_noalloc_addr[dev];
+    *addr = slot.addr;
     return MX_OK;
 }
 

@@ -87,3 +87,20 @@ def test_largest_fit_and_first_refusal():
     assert e.value.status == 7
     torch.cuda.synchronize()
     assert torch.isnan(Y2).all()                               # nothing was launched
+
+
+def test_group_wise_activation_scales():
+    # act_group = g: s_a takes 2 M (K / g) bytes of the array, two calls in a row
+    lay = inputs.llama_layer(40, 2048, 768, seed=106)
+    L, blob = gpu_pack(lay.W, lay.is8, 128)
+    Xd = to_dev(lay.X)
+    n = mx.mx_linear_workspace_size(L, 40, act_group=128)
+    assert n >= 40 * 2048 + 2 * 40 * (2048 // 128)
+    ref = torch.empty((40, L.N), dtype=torch.float16, device=dev())
+    ws = torch.empty(mx.NOALLOC_SCRATCH_BYTES, dtype=torch.uint8, device=dev())
+    mx.mx_linear(L, blob, Xd, ref, workspace=ws, act_group=128)
+    for _ in range(2):
+        Y = nan_out(L, 40)
+        mx.mx_linear_noalloc(L, blob, Xd, Y, act_group=128)
+        torch.cuda.synchronize()
+        assert torch.equal(Y, ref)
