@@ -100,7 +100,9 @@ typedef struct mx_layout {
 typedef struct mx_gemm_opts {
     int32_t path;              /* 0 auto; 1 split-K CUDA-core path; 2 tensor-core path;
                                   3 row CUDA-core path (whole rows per CTA); 4 tensor-core
-                                  path on CTA pairs (cta_group::2, 256 rows x 128 tokens) */
+                                  path on CTA pairs (cta_group::2, 256 rows x 128 tokens);
+                                  5 tensor-core path on CTA pairs with 256-token tiles
+                                  (256 rows x 256 tokens, no K split) */
     int32_t split;             /* path 1: CTAs (a thread-block cluster, 1..8) that split
                                   the K range of each row unit (0 = auto); a split
                                   asked for under auto selects path 1 for M <= 16.
@@ -211,13 +213,20 @@ mx_status mx_gemm_workspace_size(const mx_layout* L, int M, const mx_gemm_opts* 
  *       4-bit (or 16 8-bit) rows over the whole K, no reduction between CTAs;
  *   1 = split-K path: M <= 16; the K split of each row unit is one thread-block
  *       cluster reduced through distributed shared memory;
- *   4 = tensor cores on CTA pairs (larger M): tcgen05.mma.cta_group::2 over 256
- *       weight rows x 128 tokens per pair of CTAs.
- * Auto selection tries them in that order.  2 = the one-CTA tensor-core kernel
- * (128 x 128 tiles) is taken only when opts->path asks for it.  Negative
- * mx_status on bad arguments.
+ *   4 = tensor cores on CTA pairs: tcgen05.mma.cta_group::2 over 256 weight
+ *       rows x 128 tokens per pair of CTAs, with a K split when the grid would
+ *       leave pairs idle;
+ *   5 = tensor cores on CTA pairs with 256-token tiles (prefill M): 256 weight
+ *       rows x 256 tokens per pair, M = N = 256 per MMA.
+ * Auto selection tries them in that order (5 from MX_PATH5_MIN_M tokens when
+ * its tiles fill the device).  2 = the one-CTA tensor-core kernel (128 x 128
+ * tiles) is taken only when opts->path asks for it.  Negative mx_status on bad
+ * arguments.
  */
 int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts);
+
+/* Smallest M at which automatic selection takes path 5. */
+#define MX_PATH5_MIN_M 512
 
 /*
  * mx_gemm -- Y = dequant(Aq, s_a) . dequant(W_packed)^T  (MixLLM section 3.3).

@@ -251,10 +251,14 @@ constexpr int kDecodeMaxM = 16;
 // split is asked for; larger M the tensor cores on CTA pairs, which measured at
 // least as fast as the one-CTA tensor-core kernel from 32 tokens up on the
 // Llama shapes (path 2 stays available when asked for).
+static int pair_count();
+
+// Prefill M: the 256-token pair kernel once its tiles give every CTA pair a unit.
 static int choose_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
     if (opts && opts->path) return opts->path;
     if (!(opts && opts->split > 0) && mx::plan_rows(*L, M).ok) return 3;
     if (M <= kDecodeMaxM && mx::plan_decode(*L, M, 0).ok) return 1;
+    if (M >= MX_PATH5_MIN_M && !(opts && opts->split > 1) && mx::tc3_units(*L, M) >= pair_count()) return 5;
     return 4;
 }
 
@@ -345,7 +349,7 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
         if (e != cudaSuccess) return cuda_fail(e, "decode GEMM launch");
         return MX_OK;
     }
-    if (path == 2 || path == 4) {
+    if (path == 2 || path == 4 || path == 5) {
         if (opts && opts->test_stall && !opts->status)
             return fail(MX_ERR_INVALID_ARG, "test_stall needs a status word");
         if (opts && opts->wait_timeout_us < 0) return fail(MX_ERR_INVALID_ARG, "wait_timeout_us < 0");
@@ -356,6 +360,13 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
             e = mx::launch_gemm_tc(*L, blob, Aq, s_a, M, Y, ldy, ag, opts ? opts->debug_partials : nullptr,
                                    opts ? opts->status : nullptr, timeout_ns, opts ? opts->test_stall : 0, s);
             if (e != cudaSuccess) return cuda_fail(e, "tensor-core GEMM launch");
+            return MX_OK;
+        }
+        if (path == 5) {
+            if (opts && opts->split > 1) return fail(MX_ERR_UNSUPPORTED, "split=%d: path 5 does not split K", opts->split);
+            e = mx::launch_gemm_tc3(*L, blob, Aq, s_a, M, Y, ldy, ag, opts ? opts->debug_partials : nullptr,
+                                    opts ? opts->status : nullptr, timeout_ns, opts ? opts->test_stall : 0, s);
+            if (e != cudaSuccess) return cuda_fail(e, "256-token pair tensor-core GEMM launch");
             return MX_OK;
         }
         // K splits: the caller's (needs the workspace) or automatic (taken only when the

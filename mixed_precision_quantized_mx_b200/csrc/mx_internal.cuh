@@ -220,4 +220,12 @@ cudaError_t launch_gemm_tc2(const mx_layout& L, const void* blob, const int8_t* 
                             float* part, int32_t* debug_partials, int32_t* status,
                             uint64_t timeout_ns, int stall_test, cudaStream_t s);
 
+// the same GEMM on CTA pairs with 256-token tiles (cta_group::2, M = N = 256 per MMA):
+// two group accumulators of 256 TMEM columns, one-k-block stages
+int tc3_units(const mx_layout& L, int M);                       // row-tile pairs x token tiles
+cudaError_t launch_gemm_tc3(const mx_layout& L, const void* blob, const int8_t* Aq,
+                            const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy, int ag,
+                            int32_t* debug_partials, int32_t* status, uint64_t timeout_ns,
+                            int stall_test, cudaStream_t s);
+
 }  // namespace mx

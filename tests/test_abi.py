@@ -138,7 +138,13 @@ def test_gemm_workspace_and_dispatch_on_m(lib):
     assert mx.mx_gemm_select_path(L, 1, split=2) == mx.PATH_SPLITK   # a split asks for clusters
     assert mx.mx_gemm_select_path(L, 16) == mx.PATH_SPLITK
     assert mx.mx_gemm_select_path(L, 17) == mx.PATH_PAIR           # tensor cores on CTA pairs
-    assert mx.mx_gemm_select_path(L, 2048) == mx.PATH_PAIR
+    # prefill M: 256-token pair tiles once they give every one of the 74 pairs a unit
+    # (17 row-tile pairs x 5 token tiles of 256 = 85 units at M = 1280)
+    assert mx.mx_gemm_select_path(L, 1024) == mx.PATH_PAIR
+    assert mx.mx_gemm_select_path(L, 1280) == mx.PATH_PAIR256
+    assert mx.mx_gemm_select_path(L, 2048) == mx.PATH_PAIR256
+    assert mx.mx_gemm_select_path(L, 2048, split=2) == mx.PATH_PAIR      # a K split is path 4's
+    assert mx.mx_gemm_workspace_size(L, 2048, path=mx.PATH_PAIR256) == 0
     assert mx.mx_gemm_select_path(L, 1, path=mx.PATH_TENSOR) == mx.PATH_TENSOR   # asked for
     # 16 tokens of a 64K-column activation slice cannot be staged per cluster: tensor cores
     Lbig = mx.mx_layout_init(1024, 65536, 128, 102)
