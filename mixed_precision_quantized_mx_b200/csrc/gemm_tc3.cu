@@ -13,9 +13,16 @@
 // tile this halves the widening work and the weight staging per multiply-
 // accumulate, and N = 256 is the MMA shape that runs at the full int8 rate.
 // Each CTA's TMEM (512 columns) holds two group accumulators of 128 rows x 256
-// tokens, preloaded with the fast int-to-float bias integer (section 3.3,
-// Figure 3), so the products land as fp32 bit patterns; while the tensor core
-// fills one, the epilogue drains the other.
+// tokens: the first MMA of a group overwrites one, and while the tensor core
+// fills it the epilogue drains the other.
+//
+// The epilogue converts P with the hardware int-to-float instruction (exact:
+// |P| < 2^22).  The paper's fast conversion (section 3.3, Figure 3) preloads the
+// accumulator with a bias integer so that a float subtract replaces the
+// conversion, because the A100 converts slowly; on this part the conversion
+// runs about as fast as an fp32 add, and the preload would write 128 KB of TMEM
+// per group and CTA, as much as the epilogue reads.  P and Y are the same either
+// way.
 //
 // Stages are one k-block (128 columns of K): 16 KB of int8 weight operand,
 // 16 KB of this CTA's tokens, 8 KB of raw uint4 codes and the zero points, five
@@ -27,9 +34,13 @@
 //   warp 0      weight copies: codes (uint4 raw, or pre-swizzled int8) and the
 //               zero points of the stage, from rotating lanes
 //   warp 1      token copies: one TMA box of 128 tokens x 128 bytes per stage
-//   warp 2      TMEM allocation (both CTAs); in the even CTA one thread issues
-//               the pair MMAs and commits to barriers in both CTAs
-//   warp 3      idle
+//   warps 2-3   TMEM allocation (warp 2, both CTAs); in the even CTA one thread
+//               of each issues the pair MMAs of one accumulator (even or odd
+//               groups) and commits to barriers in both CTAs.  Issuing a group
+//               blocks while the tensor core still runs the one before it, so a
+//               single issuer would notice the release of the other accumulator
+//               only after that; with one issuer per accumulator each waits on
+//               its own.
 //   warps 4-7   widening of 4-bit rows (uint4 -> int8 q - z), then an arrival
 //               on the even CTA's "stage ready" barrier
 //   warps 8-15  epilogue: warp w reads TMEM lane quarter w % 4, accumulator
@@ -64,17 +75,20 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiCols = 128;                   // accumulator columns (tokens) per epilogue warp
 constexpr int kThreads = 16 * 32;
 constexpr int kScaleRing = 4;
-constexpr int kPiece = 16;                      // TMEM columns per epilogue load
+constexpr int kPiece = 32;                      // TMEM columns per epilogue load
 constexpr int kSatGroups = 4;
 static_assert(kSlots * kSlotCols <= int(kTmemCols), "accumulators fit in TMEM");
 static_assert(kEpiWarps * kEpiCols == 4 * BN, "two epilogue warps per TMEM lane quarter");
 static_assert(kWidenChunks * kWidenThreads == BM * 4, "every raw chunk widened once");
 
 // registers per thread after the split: 256 threads at kLowRegs, 256 at kEpiRegs,
-// together the 128 x 512 the block is launched with
+// together the kLaunchRegs x 512 the block is launched with (a split above the
+// launch would leave setmaxnreg.inc waiting for ever, so the launcher checks the
+// compiled count)
+constexpr uint32_t kLaunchRegs = 128;
 constexpr uint32_t kLowRegs = 72;
 constexpr uint32_t kEpiRegs = 184;
-static_assert(256 * kLowRegs + 256 * kEpiRegs == 128 * kThreads, "register split adds up to the launch");
+static_assert(256 * kLowRegs + 256 * kEpiRegs == kLaunchRegs * kThreads, "register split adds up to the launch");
 
 struct __align__(1024) Smem {
     uint8_t A[kStages][kABytes];   // int8 weight operand (swizzled 128-byte rows)
@@ -84,10 +98,11 @@ struct __align__(1024) Smem {
     uint64_t full_w[kStages];      // this CTA's weight codes and zero points of the stage landed
     uint64_t full_t[kStages];      // this CTA's tokens of the stage landed
     uint64_t ready[kStages];       // (even CTA) both CTAs' operands of the stage are in place
-    uint64_t empty[kStages];       // (both) the pair MMAs reading the stage completed
+    uint64_t empty[kStages];       // (both) the pair MMAs reading the stage completed (one commit
+                                   // per group of the stage)
     uint64_t acc_full[kSlots];     // (both) a group accumulator is complete
     uint64_t acc_empty[kSlots];    // (even CTA) both CTAs drained and re-armed it
-    uint64_t mma_done;
+    uint64_t mma_done[kSlots];     // (even CTA) an issuer's MMAs all completed
     __align__(16) __half sat[kEpiWarps][kSatGroups][kEpiCols];   // group-wise token scales
     uint32_t tmem_base;
     int abort;
@@ -168,13 +183,13 @@ gemm_tc3_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
             mbar_init(&S.full_w[s], 1);
             mbar_init(&S.full_t[s], 1);
             mbar_init(&S.ready[s], 2 * kWidenWarps);
-            mbar_init(&S.empty[s], 1);
+            mbar_init(&S.empty[s], kKBlock / g.group);
         }
         for (int b = 0; b < kSlots; ++b) {
             mbar_init(&S.acc_full[b], 1);
             mbar_init(&S.acc_empty[b], 2 * kEpiWarps);
         }
-        mbar_init(&S.mma_done, 1);
+        for (int b = 0; b < kSlots; ++b) mbar_init(&S.mma_done[b], 1);
         S.abort = 0;
         fence_mbar_init();
         prefetch_tensormap(&amap);
@@ -250,8 +265,10 @@ gemm_tc3_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
         }
     tload_done:
         if (lane == 0) drain_stages(S.full_t, it, a.timeout_ns);
-    } else if (warp == 2) {
+    } else if (warp == 2 || warp == 3) {
         // ------------------------------------------------------------ pair MMAs (even CTA)
+        // issuer `mine` takes the groups of accumulator `mine`: every second group
+        const uint32_t mine = uint32_t(warp - 2);
         if (rank == 0 && lane == 0) {
             const uint32_t idesc = idesc_i8(2 * BM, BN);
             int it = 0;
@@ -260,34 +277,39 @@ gemm_tc3_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
+                    // does this stage hold a group of mine?  (gpk groups from gc on)
+                    if (gpk == 1 && (gc & 1u) != mine) {
+                        ++gc;
+                        continue;
+                    }
                     if (!mbar_wait_bounded(&S.ready[s], ph, abort, a.status, a.timeout_ns)) goto mma_out;
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(S.A[s]), b0 = smem_u32(S.B[s]);
                     for (int j = 0; j < gpk; ++j, ++gc) {
                         const uint32_t b = gc % kSlots;
-                        // use gc / kSlots of accumulator b: phase 0 is the epilogue's first bias preload
+                        if (b != mine) continue;
+                        // use gc / kSlots of accumulator b: phase 0 is the epilogue's first release
                         if (!mbar_wait_bounded(&S.acc_empty[b], (gc / kSlots) & 1, abort, a.status, a.timeout_ns))
                             goto mma_out;
                         tc_fence_after();
-                        // the accumulator holds the bias: every k-step adds
+                        // the group's first k-step overwrites the accumulator
                         for (int kk = 0; kk < ksteps; ++kk) {
                             const uint32_t off = uint32_t(j * g.group + kk * 32);
                             mma_i8_pair(tmem + b * kSlotCols, sw128_kmajor_desc(a0 + off),
-                                        sw128_kmajor_desc(b0 + off), idesc, 1u);
+                                        sw128_kmajor_desc(b0 + off), idesc, kk > 0 ? 1u : 0u);
                         }
                         mma_commit_pair(&S.acc_full[b]);
+                        mma_commit_pair(&S.empty[s]);    // once this group's MMAs are done, its part of
+                                                         // the stage may be refilled
                     }
-                    mma_commit_pair(&S.empty[s]);        // both CTAs may refill the stage
                 }
             }
         mma_out:
-            mma_commit_pair(&S.mma_done, 0x1);           // all MMAs issued so far complete before teardown
+            mma_commit_pair(&S.mma_done[mine], 0x1);     // all MMAs issued so far complete before teardown
             int dummy = 0;
-            mbar_wait_bounded(&S.mma_done, 0, &dummy, nullptr, a.timeout_ns);
+            mbar_wait_bounded(&S.mma_done[mine], 0, &dummy, nullptr, a.timeout_ns);
         }
-    } else if (warp == 3) {
-        // idle
-    } else if (warp < 8) {
+    } else {
         // ------------------------------------------------------------ widening (4-bit rows)
         const int wt = threadIdx.x - 4 * 32;
         int it = 0;
@@ -338,15 +360,7 @@ gemm_tc3_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
         const int row = q * 32 + lane;               // weight row within this CTA's tile
         const int cb = (e >> 2) * kEpiCols;          // first of this warp's columns (tokens) in the tile
         const uint32_t lane_addr = tmem + (uint32_t(q * 32) << 16) + uint32_t(cb);
-        const float2 nbias = make_float2(-kI2FBias, -kI2FBias);
-        // preload both accumulators with the bias, then hand them to the MMA
-#pragma unroll
-        for (int b = 0; b < kSlots; ++b)
-#pragma unroll
-            for (int c = 0; c < kEpiCols; c += 32) tmem_st_x32_splat(lane_addr + b * kSlotCols + c, kI2FBiasBits);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
+        // both accumulators start free
         if (lane == 0)
             for (int b = 0; b < kSlots; ++b) mbar_arrive_cluster(acc_empty_c + 8u * uint32_t(b));
         uint32_t gc = 0;
@@ -390,12 +404,12 @@ gemm_tc3_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
                         __syncwarp();
                     }
                     const uint32_t col0 = lane_addr + b * kSlotCols;
-                    // kPiece columns at a time: fp32 bit patterns bias + P
+                    // kPiece columns at a time: the int32 partials P
                     auto consume = [&](const uint32_t (&v)[kPiece], int piece) {
 #pragma unroll
                         for (int c = 0; c < kPiece / 2; ++c) {
-                            const float2 f = add2(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])),
-                                                  nbias);
+                            const float2 f = make_float2(__int2float_rn(int32_t(v[2 * c])),
+                                                         __int2float_rn(int32_t(v[2 * c + 1])));
                             const int k = piece * (kPiece / 2) + c;
                             if constexpr (AG) {
                                 const __half2 sh = *reinterpret_cast<const __half2*>(&sat[gi % kSatGroups][2 * k]);
@@ -409,31 +423,32 @@ gemm_tc3_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
 #pragma unroll
                             for (int c = 0; c < kPiece; ++c) {
                                 const int m = m0 + piece * kPiece + c;
-                                if (m < a.M) a.debug[(size_t(m) * g.N + orig) * g.G + gi] = int32_t(v[c] - kI2FBiasBits);
+                                if (m < a.M) a.debug[(size_t(m) * g.N + orig) * g.G + gi] = int32_t(v[c]);
                             }
                         }
                     };
-                    uint32_t v[kPiece];
-#pragma unroll
-                    for (int p = 0; p < kEpiCols / kPiece - 1; ++p) {
-                        tmem_ld_piece(col0 + p * kPiece, v);
-                        tmem_wait_ld();
-                        consume(v, p);
-                    }
-                    tmem_ld_piece(col0 + kEpiCols - kPiece, v);
+                    // two buffers: the load of piece p + 1 is in flight while piece p is
+                    // multiplied; after the last load the accumulator is released, before
+                    // the arithmetic on the last piece
+                    constexpr int kPieces = kEpiCols / kPiece;
+                    uint32_t va[kPiece], vb[kPiece];
+                    tmem_ld_piece(col0, va);
                     tmem_wait_ld();
-                    // the bias goes back and the accumulator is released before the
-                    // arithmetic on the last piece
-                    // eight columns per store: a wider splat would hold that many copies of the
-                    // bias in registers next to the accumulators
 #pragma unroll
-                    for (int c = 0; c < kEpiCols; c += 8) tmem_st_x8_splat(col0 + c, kI2FBiasBits);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(acc_empty_c + 8u * b);
+                    for (int p = 0; p < kPieces; ++p) {
+                        uint32_t (&cur)[kPiece] = (p & 1) ? vb : va;
+                        uint32_t (&nxt)[kPiece] = (p & 1) ? va : vb;
+                        if (p + 1 < kPieces) {
+                            tmem_ld_piece(col0 + (p + 1) * kPiece, nxt);
+                        } else {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive_cluster(acc_empty_c + 8u * b);
+                        }
+                        consume(cur, p);
+                        if (p + 1 < kPieces) tmem_wait_ld();
+                    }
                     ++gc;
-                    consume(v, kEpiCols / kPiece - 1);
                 }
             }
             if (orig >= 0) {
@@ -496,10 +511,15 @@ cudaError_t launch_gemm_tc3(const mx_layout& L, const void* blob, const int8_t* 
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (sms[dev] == 0) {
         for (auto k : {gemm_tc3_kernel<false, false>, gemm_tc3_kernel<true, false>, gemm_tc3_kernel<false, true>,
-                       gemm_tc3_kernel<true, true>})
+                       gemm_tc3_kernel<true, true>}) {
             if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(tc3_smem_bytes()))) !=
                 cudaSuccess)
                 return e;
+            // the register split must match the launch allocation
+            cudaFuncAttributes fa;
+            if ((e = cudaFuncGetAttributes(&fa, k)) != cudaSuccess) return e;
+            if (fa.numRegs != int(kLaunchRegs)) return cudaErrorInvalidConfiguration;
+        }
         int n = 0;
         if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
         sms[dev] = n;
