@@ -119,9 +119,18 @@ saliency_kernel(const TW* __restrict__ W, int64_t ldw, const TG* __restrict__ G,
                     }
                     const float sc = scale16(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
                     const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, sc)), 0.0f), 15.0f);
+                    const float rc = __frcp_rn(sc);
 #pragma unroll
                     for (int e = 0; e < E; ++e) {
-                        const float q = fminf(fmaxf(rintf(__fdiv_rn(w[u][e], sc)) + zf, 0.0f), 15.0f);
+                        // round(w / s) from w * (1 / s): the two differ by at most 3 2^-24 |w / s|,
+                        // so they round alike unless the product is within 2^-11 of a half-integer
+                        // (for |w / s| <= 1024; beyond that both clamp alike); there the exact
+                        // quotient decides, as in the packer
+                        const float t = __fmul_rn(w[u][e], rc);
+                        float rq = rintf(t);
+                        if (fabsf(t) <= 1024.0f && fabsf(fabsf(t - floorf(t)) - 0.5f) < 4.8828125e-4f)
+                            rq = rintf(__fdiv_rn(w[u][e], sc));
+                        const float q = fminf(fmaxf(rq + zf, 0.0f), 15.0f);
                         // (q - z) s is exact in fp32; the difference with w is taken in fp64
                         const double d = double(__fmul_rn(q - zf, sc)) - double(w[u][e]);
                         s1 = fma(double(gv[u][e]), d, s1);
