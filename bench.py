@@ -63,7 +63,8 @@ def parse():
     p.add_argument("--group", type=int, default=128)
     p.add_argument("--path", type=int, default=0,
                    help="0 auto, 1 split-K CUDA cores, 2 tensor cores, 3 whole rows per CTA, "
-                        "4 tensor cores on CTA pairs, 5 the same with 256-token tiles")
+                        "4 tensor cores on CTA pairs, 5 the same with 256-token tiles, "
+                        "6 tensor cores for decode-sized M (one CTA per row tile)")
     p.add_argument("--act-group", type=int, default=0,
                    help="activation scales: 0 one per token; the weight group: one per token and group")
     p.add_argument("--impl", default="mx", choices=["mx", "reference"])
@@ -97,12 +98,14 @@ def load_peaks():
             "source": "fallback"}
 
 
-KERNEL_SOURCES = {1: "gemm_decode.cu", 2: "gemm_tc.cu", 3: "gemm_rows.cu", 4: "gemm_tc2.cu", 5: "gemm_tc3.cu"}
+KERNEL_SOURCES = {1: "gemm_decode.cu", 2: "gemm_tc.cu", 3: "gemm_rows.cu", 4: "gemm_tc2.cu", 5: "gemm_tc3.cu",
+                  6: "gemm_tcd.cu"}
 KERNEL_NAMES = {1: "gemm_decode_kernel (cluster split-K, CUDA cores)",
                 2: "gemm_tc_kernel (tcgen05)",
                 3: "gemm_rows_kernel (whole rows per CTA, CUDA cores)",
                 4: "gemm_tc2_kernel (tcgen05 on CTA pairs)",
-                5: "gemm_tc3_kernel (tcgen05 on CTA pairs, 256-token tiles)"}
+                5: "gemm_tc3_kernel (tcgen05 on CTA pairs, 256-token tiles)",
+                6: "gemm_tcd_kernel (tcgen05 on one CTA per row tile, decode-sized token tile)"}
 
 
 def src_digest(path: int) -> str:

@@ -102,13 +102,17 @@ typedef struct mx_gemm_opts {
                                   3 row CUDA-core path (whole rows per CTA); 4 tensor-core
                                   path on CTA pairs (cta_group::2, 256 rows x 128 tokens);
                                   5 tensor-core path on CTA pairs with 256-token tiles
-                                  (256 rows x 256 tokens, no K split) */
+                                  (256 rows x 256 tokens, no K split); 6 tensor-core
+                                  path for decode-sized M <= 128 (one CTA per tile:
+                                  128 rows x the batch rounded up to 16 tokens) */
     int32_t split;             /* path 1: CTAs (a thread-block cluster, 1..8) that split
                                   the K range of each row unit (0 = auto); a split
                                   asked for under auto selects path 1 for M <= 16.
                                   path 4: K splits (1..8; 0 = auto: more than one only
                                   when the unsplit grid leaves CTA pairs idle and the
-                                  workspace holds the split sums) */
+                                  workspace holds the split sums).  path 6: K splits
+                                  (1..16; 0 = auto, taken when the workspace holds the
+                                  split sums) */
     int32_t* debug_partials;   /* device int32 [M][N][G] or NULL: every per-group
                                   int32 partial P[m][n][g] (original row order) */
     int32_t* status;           /* device int32 or NULL: kernel-side error code */

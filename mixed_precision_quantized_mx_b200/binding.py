@@ -23,7 +23,7 @@ STATUS_NAMES = {
 }
 MX_F32, MX_F16 = 0, 1
 TILE_ROWS, KBLOCK, HEADER_BYTES = 128, 128, 256
-PATH_AUTO, PATH_SPLITK, PATH_TENSOR, PATH_ROWS, PATH_PAIR, PATH_PAIR256 = 0, 1, 2, 3, 4, 5
+PATH_AUTO, PATH_SPLITK, PATH_TENSOR, PATH_ROWS, PATH_PAIR, PATH_PAIR256, PATH_TC_DECODE = 0, 1, 2, 3, 4, 5, 6
 
 EXPORTED = ("mx_version", "mx_last_error", "mx_layout_init", "mx_layout_from_header",
             "mx_pack_weights", "mx_quant_act", "mx_gemm_workspace_size", "mx_gemm_select_path",

@@ -575,9 +575,16 @@ cudaError_t launch_gemm_tc2(const mx_layout& L, const void* blob, const int8_t* 
                             : (ag ? gemm_tc2_kernel<false, true> : gemm_tc2_kernel<false, false>);
     k<<<2 * pairs, kThreads, tc2_smem_bytes(), s>>>(map, a);
     if ((e = cudaGetLastError()) != cudaSuccess || a.S == 1) return e;
-    const int64_t total = int64_t(M) * L.N;
-    const int blocks = int(std::min<int64_t>((total + 255) / 256, int64_t(sms[dev]) * 8));
-    split_reduce_kernel<<<blocks, 256, 0, s>>>(a.part, a.S, M, L.N, a.s_a, ag, a.Y, ldy);
+    return launch_split_reduce(a.part, a.S, M, L.N, s_a, ag, Y, ldy, sms[dev], s);
+}
+
+cudaError_t launch_split_reduce(const float* part, int S, int M, int N, const uint16_t* s_a, int ag, uint16_t* Y,
+                                int64_t ldy, int sms, cudaStream_t s) {
+    const int64_t total = int64_t(M) * N;
+    if (total == 0) return cudaSuccess;
+    const int blocks = int(std::min<int64_t>((total + 255) / 256, int64_t(sms) * 8));
+    split_reduce_kernel<<<blocks, 256, 0, s>>>(part, S, M, N, reinterpret_cast<const __half*>(s_a), ag,
+                                               reinterpret_cast<__half*>(Y), ldy);
     return cudaGetLastError();
 }
 

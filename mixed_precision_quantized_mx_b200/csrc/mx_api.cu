@@ -243,9 +243,12 @@ mx_status mx_quant_act_grouped(const void* X, mx_dtype xdtype, int M, int K, int
     return MX_OK;
 }
 
-// Decode-sized M is bound by HBM: the split-K CUDA-core path streams the
-// weights with enough CTAs; from 17 tokens on, the tensor cores.
+// Decode-sized M is bound by HBM: up to 8 tokens the split-K CUDA-core path
+// streams the weights with enough CTAs (16 when a cluster split is asked for);
+// from 9 to 128 tokens the decode tensor-core path, which measured faster on
+// the Llama shapes from about 8 tokens on.
 constexpr int kDecodeMaxM = 16;
+constexpr int kSplitKAutoMaxM = 8;
 
 // Short K and M <= 4 take the row kernel (whole rows per CTA) unless a cluster
 // split is asked for; larger M the tensor cores on CTA pairs, which measured at
@@ -256,8 +259,10 @@ static int pair_count();
 // Prefill M: the 256-token pair kernel once its tiles give every CTA pair a unit.
 static int choose_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
     if (opts && opts->path) return opts->path;
-    if (!(opts && opts->split > 0) && mx::plan_rows(*L, M).ok) return 3;
-    if (M <= kDecodeMaxM && mx::plan_decode(*L, M, 0).ok) return 1;
+    const bool split_asked = opts && opts->split > 0;
+    if (!split_asked && mx::plan_rows(*L, M).ok) return 3;
+    if (M <= (split_asked ? kDecodeMaxM : kSplitKAutoMaxM) && mx::plan_decode(*L, M, 0).ok) return 1;
+    if (M <= mx::kTcdMaxM) return 6;
     if (M >= MX_PATH5_MIN_M && !(opts && opts->split > 1) && mx::tc3_units(*L, M) >= pair_count()) return 5;
     return 4;
 }
@@ -286,10 +291,18 @@ static int pair_split(const mx_layout* L, int M, const mx_gemm_opts* opts) {
     return opts && opts->split > 0 ? opts->split : mx::tc2_auto_split(*L, M, pair_count());
 }
 
-// scratch mx_gemm uses at M tokens: the fp32 split sums of path 4, else nothing
+// K splits path 6 takes: the caller's, or the automatic choice
+static int tcd_split(const mx_layout* L, int M, const mx_gemm_opts* opts) {
+    return opts && opts->split > 0 ? opts->split : mx::tcd_auto_split(*L, M, 2 * pair_count());
+}
+
+// scratch mx_gemm uses at M tokens: the fp32 split sums of paths 4 and 6, else nothing
 static size_t gemm_ws_bytes(const mx_layout* L, int M, const mx_gemm_opts* opts) {
-    if (M <= 0 || choose_path(L, M, opts) != 4) return 0;
-    return mx::tc2_split_bytes(*L, M, pair_split(L, M, opts));
+    if (M <= 0) return 0;
+    const int path = choose_path(L, M, opts);
+    if (path == 4) return mx::tc2_split_bytes(*L, M, pair_split(L, M, opts));
+    if (path == 6 && M <= mx::kTcdMaxM) return mx::tcd_split_bytes(*L, M, tcd_split(L, M, opts));
+    return 0;
 }
 
 int mx_gemm_select_path(const mx_layout* L, int M, const mx_gemm_opts* opts) {
@@ -349,7 +362,7 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
         if (e != cudaSuccess) return cuda_fail(e, "decode GEMM launch");
         return MX_OK;
     }
-    if (path == 2 || path == 4 || path == 5) {
+    if (path == 2 || path == 4 || path == 5 || path == 6) {
         if (opts && opts->test_stall && !opts->status)
             return fail(MX_ERR_INVALID_ARG, "test_stall needs a status word");
         if (opts && opts->wait_timeout_us < 0) return fail(MX_ERR_INVALID_ARG, "wait_timeout_us < 0");
@@ -360,6 +373,31 @@ mx_status mx_gemm(const mx_layout* L, const void* blob, const int8_t* Aq, const 
             e = mx::launch_gemm_tc(*L, blob, Aq, s_a, M, Y, ldy, ag, opts ? opts->debug_partials : nullptr,
                                    opts ? opts->status : nullptr, timeout_ns, opts ? opts->test_stall : 0, s);
             if (e != cudaSuccess) return cuda_fail(e, "tensor-core GEMM launch");
+            return MX_OK;
+        }
+        if (path == 6) {
+            if (M > mx::kTcdMaxM) return fail(MX_ERR_UNSUPPORTED, "M=%d: path 6 serves at most %d tokens", M, mx::kTcdMaxM);
+            if (opts && (opts->split < 0 || opts->split > mx::kTcdMaxSplit))
+                return fail(MX_ERR_UNSUPPORTED, "split=%d: 1..%d on path 6", opts->split, mx::kTcdMaxSplit);
+            // K splits: the caller's (needs the workspace) or automatic (taken only when the
+            // workspace holds the split sums)
+            const bool asked = opts && opts->split > 0;
+            int S = tcd_split(L, M, opts);
+            const size_t need = mx::tcd_split_bytes(*L, M, S);
+            if (S > 1 && (workspace == nullptr || ws_bytes < need)) {
+                if (asked)
+                    return fail(MX_ERR_WORKSPACE, "split %d needs a workspace of %zu bytes, %zu given", S, need,
+                                workspace ? ws_bytes : size_t(0));
+                S = 1;
+            }
+            if (S > 1) {
+                if ((st = check_device_ptr(workspace, "workspace")) != MX_OK) return st;
+                if (!aligned16(workspace)) return fail(MX_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+            }
+            e = mx::launch_gemm_tcd(*L, blob, Aq, s_a, M, Y, ldy, ag, S, S > 1 ? static_cast<float*>(workspace) : nullptr,
+                                    opts ? opts->debug_partials : nullptr, opts ? opts->status : nullptr, timeout_ns,
+                                    opts ? opts->test_stall : 0, 2 * pair_count(), s);
+            if (e != cudaSuccess) return cuda_fail(e, "decode tensor-core GEMM launch");
             return MX_OK;
         }
         if (path == 5) {

@@ -220,6 +220,11 @@ cudaError_t launch_gemm_tc2(const mx_layout& L, const void* blob, const int8_t* 
                             float* part, int32_t* debug_partials, int32_t* status,
                             uint64_t timeout_ns, int stall_test, cudaStream_t s);
 
+// Y[m][n] = fp16(the S fp32 split sums part[k][m][n] added in split order, x s_a[m]) (group-
+// wise activation scales were applied per group when ag > 0): the second kernel of a K split
+cudaError_t launch_split_reduce(const float* part, int S, int M, int N, const uint16_t* s_a, int ag, uint16_t* Y,
+                                int64_t ldy, int sms, cudaStream_t s);
+
 // the same GEMM on CTA pairs with 256-token tiles (cta_group::2, M = N = 256 per MMA):
 // two group accumulators of 256 TMEM columns, one-k-block stages
 int tc3_units(const mx_layout& L, int M);                       // row-tile pairs x token tiles
@@ -227,5 +232,17 @@ cudaError_t launch_gemm_tc3(const mx_layout& L, const void* blob, const int8_t* 
                             const uint16_t* s_a, int M, uint16_t* Y, int64_t ldy, int ag,
                             int32_t* debug_partials, int32_t* status, uint64_t timeout_ns,
                             int stall_test, cudaStream_t s);
+
+// decode-sized M on the tensor cores of one SM each (cta_group::1, 128 weight rows x the
+// batch rounded up to 16 tokens): a unit is a row tile and a range of its k-blocks; with
+// S > 1 splits the fp32 sums [S][M][N] go to part and launch_split_reduce adds them
+constexpr int kTcdMaxM = 128;
+constexpr int kTcdMaxSplit = 16;
+int tcd_tokens(int M);                                          // the token tile NT
+int tcd_auto_split(const mx_layout& L, int M, int sms);
+size_t tcd_split_bytes(const mx_layout& L, int M, int S);       // part's bytes (0 for S = 1)
+cudaError_t launch_gemm_tcd(const mx_layout& L, const void* blob, const int8_t* Aq, const uint16_t* s_a, int M,
+                            uint16_t* Y, int64_t ldy, int ag, int S, float* part, int32_t* debug_partials,
+                            int32_t* status, uint64_t timeout_ns, int stall_test, int sms, cudaStream_t s);
 
 }  // namespace mx

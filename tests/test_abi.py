@@ -122,22 +122,30 @@ def test_host_argument_checks_before_any_launch(lib):
 
 def test_gemm_workspace_and_dispatch_on_m(lib):
     L = mx.mx_layout_init(4096, 4096, 128, 410)
-    for M in (1, 16, 2048):
+    for M in (1, 8, 2048):
         assert mx.mx_gemm_workspace_size(L, M) == 0
-    # 33 row tiles = 17 CTA pairs: one token tile leaves pairs idle, so path 4 splits K
-    # and sums the splits in a workspace; 16 token tiles fill the grid unsplit
-    n17 = mx.mx_gemm_workspace_size(L, 17)
-    assert n17 > 0 and n17 % (17 * 4096 * 4) == 0 and n17 // (17 * 4096 * 4) in range(2, 9)
+    # 33 row tiles of 128 rows: at 9..128 tokens the decode tensor-core path splits K
+    # (four ways: 132 units for 148 SMs; two at 100 tokens, whose split sums cost more)
+    # and sums the splits in a workspace
     a256 = lambda v: (v + 255) // 256 * 256
+    for M, S in ((16, 4), (17, 4), (100, 2)):
+        assert mx.mx_gemm_workspace_size(L, M) == a256(S * M * 4096 * 4)
     assert mx.mx_gemm_workspace_size(L, 17, split=3) == a256(3 * 17 * 4096 * 4)
     assert mx.mx_gemm_workspace_size(L, 17, path=mx.PATH_TENSOR) == 0     # the one-CTA kernel
     assert mx.mx_gemm_workspace_size(L, 17, split=1) == 0
+    # 17 CTA pairs at 129 tokens: one token tile leaves pairs idle, so path 4 splits K
+    n129 = mx.mx_gemm_workspace_size(L, 129)
+    assert n129 > 0 and n129 % (129 * 4096 * 4) == 0 and n129 // (129 * 4096 * 4) in range(2, 9)
     assert mx.mx_gemm_select_path(L, 1) == mx.PATH_ROWS          # short K, M <= 4, one wave
     assert mx.mx_gemm_select_path(L, 4) == mx.PATH_ROWS
     assert mx.mx_gemm_select_path(L, 5) == mx.PATH_SPLITK
+    assert mx.mx_gemm_select_path(L, 8) == mx.PATH_SPLITK
     assert mx.mx_gemm_select_path(L, 1, split=2) == mx.PATH_SPLITK   # a split asks for clusters
-    assert mx.mx_gemm_select_path(L, 16) == mx.PATH_SPLITK
-    assert mx.mx_gemm_select_path(L, 17) == mx.PATH_PAIR           # tensor cores on CTA pairs
+    assert mx.mx_gemm_select_path(L, 16, split=2) == mx.PATH_SPLITK
+    assert mx.mx_gemm_select_path(L, 9) == mx.PATH_TC_DECODE       # decode tensor cores, one CTA per tile
+    assert mx.mx_gemm_select_path(L, 16) == mx.PATH_TC_DECODE
+    assert mx.mx_gemm_select_path(L, 128) == mx.PATH_TC_DECODE
+    assert mx.mx_gemm_select_path(L, 129) == mx.PATH_PAIR          # tensor cores on CTA pairs
     # prefill M: 256-token pair tiles once they give every one of the 74 pairs a unit
     # (17 row-tile pairs x 5 token tiles of 256 = 85 units at M = 1280)
     assert mx.mx_gemm_select_path(L, 1024) == mx.PATH_PAIR
@@ -148,7 +156,7 @@ def test_gemm_workspace_and_dispatch_on_m(lib):
     assert mx.mx_gemm_select_path(L, 1, path=mx.PATH_TENSOR) == mx.PATH_TENSOR   # asked for
     # 16 tokens of a 64K-column activation slice cannot be staged per cluster: tensor cores
     Lbig = mx.mx_layout_init(1024, 65536, 128, 102)
-    assert mx.mx_gemm_select_path(Lbig, 16) == mx.PATH_PAIR
+    assert mx.mx_gemm_select_path(Lbig, 16) == mx.PATH_TC_DECODE
     # the row path needs K <= 4096 and one wave of CTAs
     assert mx.mx_gemm_select_path(mx.mx_layout_init(4096, 8192, 128, 410), 1) == mx.PATH_SPLITK
     assert mx.mx_gemm_select_path(mx.mx_layout_init(14336, 4096, 128, 1434), 1) == mx.PATH_SPLITK

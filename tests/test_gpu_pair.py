@@ -147,13 +147,13 @@ def test_pair_split_workspace_rules(orc):
         mx.mx_gemm(L, blob, Aq, sa, Y, path=mx.PATH_PAIR, split=2)
     assert e.value.status == 7
     # an automatic split without a workspace runs unsplit: bit-identical to split=1
-    assert mx.mx_gemm_workspace_size(L, M) > 0
-    mx.mx_gemm(L, blob, Aq, sa, Y)
+    assert mx.mx_gemm_workspace_size(L, M, path=mx.PATH_PAIR) > 0
+    mx.mx_gemm(L, blob, Aq, sa, Y, path=mx.PATH_PAIR)
     Y1, _, _ = gpu_gemm(L, blob, Aq, sa, path=mx.PATH_PAIR, split=1)
     torch.cuda.synchronize()
     assert torch.equal(Y.view(torch.int16), Y1.view(torch.int16))
     # with it, the automatic split agrees with the oracle
-    Ya, _, _ = gpu_gemm(L, blob, Aq, sa)
+    Ya, _, _ = gpu_gemm(L, blob, Aq, sa, path=mx.PATH_PAIR)
     Aq_o, sa_o = orc.quant_act(X.astype(np.float32))
     assert_y_close(Ya.cpu().numpy(), orc.gemm(Aq_o, sa_o, orc.pack(W, is8, 128))[1])
 
