@@ -67,3 +67,17 @@ def test_forward_group_wise_activations(orc, M):
     Aq, sa = orc.quant_act(lay.X.astype(np.float32), act_group=128)
     ref = orc.gemm(Aq, sa, orc.pack(lay.W, lay.is8, 128), act_group=128)[1]
     assert_y_close(Y.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("M", [2, 40])
+def test_sharded_linear_on_one_rank_equals_the_layer(orc, M):
+    # output-feature sharding with a single rank: the shard is the whole layer
+    from mixed_precision_quantized_mx_b200.tensor_parallel import ShardedLinear
+    lay = inputs.llama_layer(M, 512, 300, seed=40 + M)
+    sharded = ShardedLinear(torch.from_numpy(lay.W), torch.from_numpy(lay.is8), device=dev())
+    assert (sharded.start, sharded.stop, sharded.world) == (0, 300, 1)
+    X = torch.from_numpy(lay.X).to(dev())
+    Y = sharded(X)
+    assert_y_close(Y.cpu().numpy(), oracle_y(orc, lay.X, lay.W, lay.is8, 128))
+    whole = MixedPrecisionLinear(torch.from_numpy(lay.W).to(dev()), torch.from_numpy(lay.is8).to(dev()))
+    assert torch.equal(Y, whole(X))
