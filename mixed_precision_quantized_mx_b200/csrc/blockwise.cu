@@ -10,7 +10,10 @@
 // lanes below 4 b then store its words.
 //
 // GEMM (decode-sized M): one warp per output row, the tokens of one tile of 8 per
-// CTA row.  Per column block a lane takes codes 4l .. 4l + 3: their 4 b bits come
+// CTA row.  The eight rows of a CTA lie in one block row, whose blocks' widths and
+// code offsets the CTA stages in shared memory first; a warp then issues the loads
+// of 16 blocks (codes, and the zero points and scales one per lane) before using
+// any, so enough bytes are in flight.  Per column block a lane takes codes 4l .. 4l + 3: their 4 b bits come
 // from one or two of the row's 4 b words (one coalesced load, two shuffles, a
 // funnel shift), are spread into four bytes, and one byte-wise subtract of the
 // zero point gives four int8 (q - z) for dp4a with the token's activations.  The
@@ -28,7 +31,7 @@ constexpr int kBC = MX_BW_BLOCK_COLS;
 constexpr int kPackWarps = 8;
 constexpr int kGemmWarps = 8;
 constexpr int kTok = 8;           // tokens per CTA row of the grid
-constexpr int kPre = 4;           // column blocks whose loads are issued together
+constexpr int kPre = 16;          // column blocks whose loads are issued together (<= 32)
 
 // fp16 scale of an fp32 value: saturate at 65504, zero -> 1 (the packer's rule)
 __device__ __forceinline__ float scale16(float s32) {
@@ -115,45 +118,53 @@ bw_gemm_kernel(const uint8_t* __restrict__ codes, const uint32_t* __restrict__ o
                const uint8_t* __restrict__ meta, uint32_t table4, const __half* __restrict__ scales,
                const uint8_t* __restrict__ zeros, const int8_t* __restrict__ Aq, const __half* __restrict__ s_a,
                int M, int N, int K, int KB, __half* __restrict__ Y, int64_t ldy, int32_t* __restrict__ P) {
+    // the CTA's rows share one block row: its blocks' widths and code offsets, once
+    extern __shared__ uint32_t binfo[];                  // [KB]: offset in 16-byte units | width << 28
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int n = blockIdx.x * kGemmWarps + warp;
+    const int n0 = blockIdx.x * kGemmWarps;
+    const int rb = n0 / kBR;
+    for (int kb = threadIdx.x; kb < KB; kb += kGemmWarps * 32) {
+        const int64_t bi = int64_t(rb) * KB + kb;
+        binfo[kb] = __ldg(offsets + bi) | (uint32_t(block_width(meta, bi, table4)) << 28);
+    }
+    __syncthreads();
+    const int n = n0 + warp;
     if (n >= N) return;                                   // the whole warp; no block barrier follows
     const int m0 = blockIdx.y * kTok;
     const int mt = min(kTok, M - m0);
-    const int rb = n / kBR, r = n % kBR;
+    const int r = n % kBR;
     const int8_t* a_base = Aq + int64_t(m0) * K + lane * 4;
+    const uint8_t* zrow = zeros + int64_t(n) * KB;
+    const __half* srow = scales + int64_t(n) * KB;
     float yacc[kTok];
 #pragma unroll
     for (int t = 0; t < kTok; ++t) yacc[t] = 0.0f;
 
     for (int kb0 = 0; kb0 < KB; kb0 += kPre) {
-        // issue the loads of up to kPre blocks before using any
-        int bw[kPre];
-        uint32_t mine[kPre], zz[kPre];
-        float sw[kPre];
+        // issue the loads of up to kPre blocks before using any: each lane below 4 b its
+        // word of the block's codes, lane j the zero point and scale of block kb0 + j
+        uint32_t mine[kPre];
+        const uint32_t zl = kb0 + lane < KB && lane < kPre ? uint32_t(__ldg(zrow + kb0 + lane)) : 0u;
+        const float sl = kb0 + lane < KB && lane < kPre ? __half2float(__ldg(srow + kb0 + lane)) : 0.0f;
 #pragma unroll
         for (int j = 0; j < kPre; ++j) {
-            bw[j] = 0;
             mine[j] = 0;
-            zz[j] = 0;
-            sw[j] = 0.0f;
             const int kb = kb0 + j;
             if (kb < KB) {                                // warp-uniform
-                const int64_t bi = int64_t(rb) * KB + kb;
-                const int b = block_width(meta, bi, table4);
+                const uint32_t info = binfo[kb];
+                const int b = int(info >> 28);
                 const uint32_t* row = reinterpret_cast<const uint32_t*>(
-                    codes + (size_t(__ldg(offsets + bi)) << 4) + size_t(r) * 16 * b);
-                bw[j] = b;
+                    codes + (size_t(info & 0x0FFFFFFFu) << 4) + size_t(r) * 16 * b);
                 if (lane < 4 * b) mine[j] = __ldg(row + lane);
-                zz[j] = uint32_t(__ldg(zeros + int64_t(n) * KB + kb)) * 0x01010101u;
-                sw[j] = __half2float(__ldg(scales + int64_t(n) * KB + kb));
             }
         }
 #pragma unroll
         for (int j = 0; j < kPre; ++j) {
             const int kb = kb0 + j;
             if (kb >= KB) break;                          // warp-uniform
-            const int b = bw[j];
+            const int b = int(binfo[kb] >> 28);
+            const uint32_t zz = __shfl_sync(0xffffffffu, zl, j) * 0x01010101u;
+            const float sw = __shfl_sync(0xffffffffu, sl, j);
             const int bit = 4 * b * lane, w0 = bit >> 5, sh = bit & 31;
             const uint32_t lo_w = __shfl_sync(0xffffffffu, mine[j], w0);
             const uint32_t hi_w = __shfl_sync(0xffffffffu, mine[j], min(w0 + 1, 31));
@@ -164,13 +175,13 @@ bw_gemm_kernel(const uint8_t* __restrict__ codes, const uint32_t* __restrict__ o
                 bytes = (x & mask) | (((x >> b) & mask) << 8) | (((x >> (2 * b)) & mask) << 16) |
                         (((x >> (3 * b)) & mask) << 24);
             }
-            const int d = int(__vsub4(bytes, zz[j]));     // four int8 (q - z)
+            const int d = int(__vsub4(bytes, zz));        // four int8 (q - z)
             const int8_t* a = a_base + int64_t(kb) * kBC;
 #pragma unroll
             for (int t = 0; t < kTok; ++t) {
                 if (t < mt) {                             // warp-uniform
                     const int p = __dp4a(d, __ldg(reinterpret_cast<const int*>(a + int64_t(t) * K)), 0);
-                    yacc[t] = fmaf(sw[j], float(p), yacc[t]);
+                    yacc[t] = fmaf(sw, float(p), yacc[t]);
                     if (P != nullptr) {
                         int s = p;
 #pragma unroll
@@ -219,7 +230,10 @@ cudaError_t launch_bw_gemm(const mx_bw_layout& L, const uint8_t* blob, const int
     const uint32_t table4 = uint32_t(L.table[0]) | uint32_t(L.table[1]) << 8 | uint32_t(L.table[2]) << 16 |
                             uint32_t(L.table[3]) << 24;
     const dim3 grid(unsigned((L.N + kGemmWarps - 1) / kGemmWarps), unsigned((M + kTok - 1) / kTok));
-    bw_gemm_kernel<<<grid, kGemmWarps * 32, 0, s>>>(
+    const size_t smem = size_t(L.KB) * 4;                // the block row's widths and offsets
+    if (smem > 48 * 1024) return cudaErrorInvalidValue;
+    if ((L.code_bytes >> 4) >= (uint64_t(1) << 28)) return cudaErrorInvalidValue;   // offsets packed in 28 bits
+    bw_gemm_kernel<<<grid, kGemmWarps * 32, smem, s>>>(
         blob + L.off_codes, reinterpret_cast<const uint32_t*>(blob + L.off_offsets), blob + L.off_meta, table4,
         reinterpret_cast<const __half*>(blob + L.off_scales), blob + L.off_zeros, Aq, s_a, M, L.N, L.K, L.KB, Y, ldy,
         P);
