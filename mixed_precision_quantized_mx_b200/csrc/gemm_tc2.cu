@@ -478,6 +478,10 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(const float* __restri
                                                            const __half* __restrict__ s_a, int ag, __half* Y,
                                                            int64_t ldy) {
     const int64_t total = int64_t(M) * N;
+    // launched as a programmatic dependent: resident while the GEMM finishes, it reads
+    // the sums only once that kernel completed; its own dependents may start at once
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     for (int64_t i = int64_t(blockIdx.x) * 256 + threadIdx.x; i < total; i += int64_t(gridDim.x) * 256) {
         const int m = int(i / N), n = int(i % N);
         float v = part[i];
@@ -583,9 +587,17 @@ cudaError_t launch_split_reduce(const float* part, int S, int M, int N, const ui
     const int64_t total = int64_t(M) * N;
     if (total == 0) return cudaSuccess;
     const int blocks = int(std::min<int64_t>((total + 255) / 256, int64_t(sms) * 8));
-    split_reduce_kernel<<<blocks, 256, 0, s>>>(part, S, M, N, reinterpret_cast<const __half*>(s_a), ag,
-                                               reinterpret_cast<__half*>(Y), ldy);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, split_reduce_kernel, part, S, M, N, reinterpret_cast<const __half*>(s_a), ag,
+                              reinterpret_cast<__half*>(Y), ldy);
 }
 
 }  // namespace mx

@@ -15,19 +15,45 @@
 // accumulators (NT columns) TMEM holds up to eight, so the epilogue drains them
 // while the tensor core fills the next ones.
 //
+// At these sizes every step of a k-block's way is short, and what sets the pace is
+// how many steps wait on one another.  Measured on this part: one thread issues a
+// bulk copy only every few hundred ns whatever its size, a copy lands about a
+// microsecond after issue, an MMA issue takes about 60 ns, and a barrier hand-over
+// about 100 ns.  Hence:
+//   R ring   the weights as stored, in 8 KB slots: a 4-bit k-block (uint4 codes)
+//            takes one slot, its zero points beside it, an 8-bit k-block (int8
+//            codes, stored pre-swizzled) two consecutive ones.  The copies move
+//            chunks of four slots (one bulk copy per run of one unit's slots), and
+//            a chunk is free once it is widened, so the ring is deep and the copies
+//            run far ahead of the tensor core.
+//   A ring   the int8 weight operand, written by the widening warps (a stage always
+//            by the same group), freed by the MMAs (a commit per group).
+//   B ring   the batch's tokens, one TMA box per chunk of four k-blocks (two from
+//            NT = 64); a chunk is freed by one commit of each MMA issuer.
+//   widening groups of two warps take every fourth k-block each (every second
+//            from NT = 64), so that several k-blocks are widened at once.
+// Chunks are aligned to the ring (they start at a multiple of the chunk size and may
+// hold runs of two units), so they never wrap a ring.  A chunk's bytes are counted
+// on the barrier of its first slot.  A barrier's parity names its phase only to a
+// waiter at most one phase away, so every waiter of a barrier waits on each of its
+// phases in order: every widening group waits on every weight chunk and releases it
+// (the copy thread re-arms a chunk once all have), each MMA issuer waits on every
+// token chunk (each holds k-blocks of both), and an operand stage always belongs to
+// the same widening group.
+//
 // Roles (16 warps, one CTA per SM, persistent over the units):
-//   warp 0       weight copies: per stage one k-block of the tile's codes (uint4
-//                raw, or pre-swizzled int8) and its zero points, from rotating lanes
-//   warps 1-2    TMEM allocation (warp 1); one thread of each issues the MMAs and
-//                commits of every second group (the accumulators of one parity).
-//                At small N an MMA executes faster than a thread can issue the
-//                next one, so two issuers keep the tensor core fed
-//   warp 3       token copies: one TMA box of NT tokens x 128 bytes per stage.
-//                Issuing a copy takes a thread long compared with a k-block's work
-//                at decode sizes, so weights and tokens come from different warps
-//   warps 4-     widening of 4-bit rows (uint4 -> int8 q - z), then an arrival on
-//                the stage's "ready" barrier (8 warps; 4 at NT = 128, whose MMAs
-//                take longer)
+//   warp 0       weight copies into the R ring.  The weights do not depend on the
+//                kernel before this one in the stream (under programmatic dependent
+//                launch), so they stream from the start
+//   warps 1-2    TMEM allocation (warp 1); one thread of each waits for the tokens
+//                and the operand and issues the MMAs and commits of every second
+//                group (the accumulators of one parity).  At small N an MMA executes
+//                faster than a thread can issue the next one (about 60 ns), so two
+//                issuers keep the tensor core fed
+//   warp 3       token copies into the B ring, after griddepcontrol.wait
+//   warps 4-     widening: 4-bit codes to int8 q - z, 8-bit codes copied as they
+//                are, from the R ring into the group's A stage, then an arrival on
+//                the stage's "ready" barrier
 //   last warps   epilogue: warp w reads TMEM lane quarter w % 4, kEpiCols tokens each;
 //                the group's partials are converted with cvt.rn.f32.s32 (exact:
 //                |P| < 2^22) and scaled in fp32
@@ -45,41 +71,55 @@ using namespace sm100;
 
 constexpr int BM = 128;                         // weight rows per tile (UMMA M)
 constexpr int kABytes = BM * kKBlock;           // int8 weight operand of one k-block
-constexpr int kRawBytes = BM * kKBlock / 2;     // uint4 codes of one k-block
-constexpr int kZBytes = 2 * BM;                 // zero points of up to two groups
+constexpr int kSlotBytes = BM * kKBlock / 2;    // an R slot: the uint4 codes of one k-block
+constexpr int kZBytes = 2 * BM;                 // zero points of up to two groups per slot
+constexpr int kCR = 4;                          // R slots per chunk
+constexpr int kGW = 2;                          // warps per widening group
 constexpr int kWiden0 = 4;                      // first widening warp
 constexpr int kScaleRing = 2;
 
+constexpr int token_chunk(int NT) { return NT <= 32 ? 4 : 2; }   // k-blocks per token chunk
+
 template <int NT>
 struct Cfg {
-    static constexpr int kWidenWarps = NT <= 64 ? 8 : 4;
-    static constexpr int kWidenThreads = kWidenWarps * 32;
-    static constexpr int kWidenChunks = BM * 4 / kWidenThreads;   // 16-byte raw chunks per thread and stage
-    static constexpr int kEpiWarp0 = kWiden0 + kWidenWarps;      // first epilogue warp (a multiple of 4)
-    static constexpr int kEpiWarps = NT <= 64 ? 4 : 8;
+    static constexpr int kWidenWarps = NT <= 32 ? 8 : 4;
+    static constexpr int kGroups = kWidenWarps / kGW;          // widening groups
+    static constexpr int kGT = kGW * 32;                       // threads per widening group
+    static constexpr int kEpiWarp0 = kWiden0 + kWidenWarps;    // first epilogue warp (a multiple of 4)
+    static constexpr int kEpiWarps = NT <= 32 ? 4 : 8;
     static constexpr int kEpiCols = NT * 4 / kEpiWarps;       // tokens per epilogue warp
     static constexpr int kPiece = kEpiCols >= 32 && NT <= 64 ? 32 : 16;   // TMEM columns per load
     static constexpr int kSlots = NT <= 64 ? 8 : 4;           // group accumulators in TMEM (even: one
                                                               // parity per issuer)
     static constexpr uint32_t kTmemCols = kSlots * NT <= 128 ? 128 : kSlots * NT <= 256 ? 256 : 512;
-    static constexpr int kStages = NT <= 64 ? 6 : 5;
+    static constexpr int kA = 4;                              // int8 operand stages (stage s: group s % kGroups)
+    static constexpr int kCB = token_chunk(NT);
+    static constexpr int kB = NT <= 32 ? 12 : NT == 64 ? 6 : 4;    // token stages
+    static constexpr int kBChunks = kB / kCB;
+    static constexpr int kR = NT <= 16 ? 16 : NT <= 64 ? 12 : 8;   // raw weight slots
     static constexpr int kBBytes = NT * kKBlock;
     static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
     static_assert(kThreads == 512, "16 warps: 128 registers per thread");
     static_assert(kSlots * NT <= int(kTmemCols), "accumulators fit in TMEM");
     static_assert(kEpiCols % kPiece == 0, "whole loads");
+    static_assert(kB % kCB == 0 && kR % kCR == 0, "chunks never wrap a ring");
+    static_assert(kBChunks >= 2 && kR >= 2 * kCR, "rings hold two chunks");
+    static_assert(kSlotBytes % (16 * kGT) == 0, "whole 16-byte chunks per widening thread");
+    static_assert(kA % kGroups == 0, "an operand stage always belongs to the same widening group");
 };
 
 template <int NT>
 struct __align__(1024) Smem {
-    uint8_t A[Cfg<NT>::kStages][kABytes];        // int8 weight operand (swizzled 128-byte rows)
-    uint8_t B[Cfg<NT>::kStages][Cfg<NT>::kBBytes];   // the batch's tokens (swizzled by the copy)
-    uint8_t R[Cfg<NT>::kStages][kRawBytes];      // raw uint4 codes of 4-bit rows
-    uint8_t Z[Cfg<NT>::kStages][kZBytes];        // zero points of the stage's groups, [group][row]
-    uint64_t full_w[Cfg<NT>::kStages];           // the stage's weight codes and zero points landed
-    uint64_t full_t[Cfg<NT>::kStages];           // the stage's tokens landed
-    uint64_t ready[Cfg<NT>::kStages];            // the stage's operands are in place
-    uint64_t empty[Cfg<NT>::kStages];            // the MMAs reading the stage completed (one commit per group)
+    uint8_t A[Cfg<NT>::kA][kABytes];             // int8 weight operand (swizzled 128-byte rows)
+    uint8_t B[Cfg<NT>::kB][Cfg<NT>::kBBytes];    // the batch's tokens (swizzled by the copy)
+    uint8_t R[Cfg<NT>::kR][kSlotBytes];          // weights as stored (4-bit: one slot, 8-bit: two)
+    uint8_t Z[Cfg<NT>::kR][kZBytes];             // zero points: a run's lie contiguously from its first slot
+    uint64_t r_full[Cfg<NT>::kR];                // a weight chunk landed (the barrier of its first slot)
+    uint64_t r_rel[Cfg<NT>::kR / kCR];           // every widening warp is done with a weight chunk
+    uint64_t b_full[Cfg<NT>::kB];                // a token chunk landed (the barrier of its first stage)
+    uint64_t b_empty[Cfg<NT>::kBChunks];         // the MMAs reading a token chunk completed (one per issuer)
+    uint64_t ready[Cfg<NT>::kA];                 // the operand is written
+    uint64_t a_empty[Cfg<NT>::kA];               // the MMAs reading the operand completed (one commit per group)
     uint64_t acc_full[Cfg<NT>::kSlots];          // a group accumulator is complete
     uint64_t acc_empty[Cfg<NT>::kSlots];         // the epilogue drained it
     uint64_t mma_done[2];                        // an issuer's MMAs all completed
@@ -113,6 +153,10 @@ __device__ __forceinline__ uint32_t widen_hi(uint32_t w, uint32_t zc) {
 __device__ __forceinline__ void tmem_ld_piece(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld_x16(taddr, r); }
 __device__ __forceinline__ void tmem_ld_piece(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld_x32(taddr, r); }
 
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 struct Unit {
     int t;        // row tile
     int ks;       // K split
@@ -132,9 +176,23 @@ __device__ __forceinline__ Unit unit_of(const TcdArgs& a, int u) {
     return r;
 }
 
+// A run: consecutive slots (stages) of one unit inside one chunk, one copy.
+struct WRun {
+    const uint8_t* src;    // codes
+    const uint8_t* zsrc;   // zero points (4-bit units)
+    int slot;              // first slot (running count)
+    uint32_t bytes, zbytes;
+};
+struct TRun {
+    int kb;                // first k-block
+    int n;                 // k-blocks
+    int stage;             // first stage (running count)
+};
+
 template <int NT, bool DEBUG, bool AG>
 __global__ void __launch_bounds__(Cfg<NT>::kThreads, 1)
-gemm_tcd_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ TcdArgs a) {
+gemm_tcd_kernel(const __grid_constant__ CUtensorMap amap1, const __grid_constant__ CUtensorMap amapC,
+                const __grid_constant__ TcdArgs a) {
     using C = Cfg<NT>;
     extern __shared__ uint8_t smem_raw[];
     Smem<NT>& S = *reinterpret_cast<Smem<NT>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -145,11 +203,13 @@ gemm_tcd_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
     volatile int* abort = &S.abort;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&S.full_w[s], 1);
-            mbar_init(&S.full_t[s], 1);
-            mbar_init(&S.ready[s], C::kWidenWarps);
-            mbar_init(&S.empty[s], gpk);
+        for (int s = 0; s < C::kR; ++s) mbar_init(&S.r_full[s], 1);
+        for (int c = 0; c < C::kR / kCR; ++c) mbar_init(&S.r_rel[c], C::kWidenWarps);
+        for (int s = 0; s < C::kB; ++s) mbar_init(&S.b_full[s], 1);
+        for (int c = 0; c < C::kBChunks; ++c) mbar_init(&S.b_empty[c], 2);
+        for (int s = 0; s < C::kA; ++s) {
+            mbar_init(&S.ready[s], kGW);
+            mbar_init(&S.a_empty[s], gpk);
         }
         for (int b = 0; b < C::kSlots; ++b) {
             mbar_init(&S.acc_full[b], 1);
@@ -159,7 +219,8 @@ gemm_tcd_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
         mbar_init(&S.mma_done[1], 1);
         S.abort = 0;
         fence_mbar_init();
-        prefetch_tensormap(&amap);
+        prefetch_tensormap(&amap1);
+        prefetch_tensormap(&amapC);
     }
     if (warp == 1) {
         tmem_alloc(&S.tmem_base, C::kTmemCols);
@@ -169,90 +230,189 @@ gemm_tcd_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
+    // the next kernel in the stream may be scheduled now; it waits for this one to
+    // complete before it touches anything this one reads or writes
+    if (threadIdx.x == 0) griddep_launch();
 
-    if (warp == 0 || warp == 3) {
-        // ------------------------------------------------------------ copies
-        // warp 0: the weight codes and zero points; warp 3: the tokens
-        const bool wts = warp == 0;
-        uint64_t* full = wts ? S.full_w : S.full_t;
-        int it = 0;
+    if (warp == 0) {
+        // ------------------------------------------------------------ weight copies (R ring)
+        // every lane keeps the same bookkeeping; lane 0 waits and arms, the runs'
+        // copies are spread over the lanes
+        WRun run[kCR];
+        int nrun = 0, ir = 0, armed = 0, nchunk = 0;
+        auto flush = [&](int end) -> bool {
+            const int base = (end - 1) & ~(kCR - 1);
+            uint32_t total = 0;
+            for (int j = 0; j < nrun; ++j) total += run[j].bytes + run[j].zbytes;
+            bool ok = true;
+            if (lane == 0) {
+                // the chunk's place released by every widening warp in the previous pass
+                ok = mbar_wait_bounded(&S.r_rel[(base % C::kR) / kCR], ((base / C::kR) & 1) ^ 1, abort, a.status,
+                                       a.timeout_ns);
+                if (ok) mbar_arrive_expect_tx(&S.r_full[base % C::kR], total);
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+            uint64_t* bar = &S.r_full[base % C::kR];
+            const int l0 = (nchunk * 2 * kCR) & 31;
+            for (int j = 0; j < nrun; ++j) {
+                if (lane == ((l0 + 2 * j) & 31)) bulk_g2s(S.R[run[j].slot % C::kR], run[j].src, run[j].bytes, bar);
+                if (run[j].zbytes != 0 && lane == ((l0 + 2 * j + 1) & 31))
+                    bulk_g2s(&S.Z[run[j].slot % C::kR][0], run[j].zsrc, run[j].zbytes, bar);
+            }
+            nrun = 0;
+            ++nchunk;
+            armed = end;
+            return true;
+        };
         if (!a.stall_test) {
             for (int u = blockIdx.x; u < a.n_units; u += gridDim.x) {
                 const Unit un = unit_of(a, u);
-                for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
-                    const int s = it % C::kStages;
-                    const uint32_t ph = (it / C::kStages) & 1;
-                    bool ok = true;
-                    if (lane == 0) ok = mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, a.status, a.timeout_ns);
-                    if (!__shfl_sync(0xffffffffu, ok, 0)) goto load_done;
-                    if (wts) {
-                        const uint32_t cbytes = uint32_t(un.eight ? kABytes : kRawBytes);
-                        const uint32_t zbytes = un.eight ? 0u : uint32_t(gpk * BM);
-                        if (lane == 0) mbar_arrive_expect_tx(&full[s], cbytes + zbytes);
-                        __syncwarp();
-                        const size_t blk = size_t(un.lt) * g.kblocks + kb;
-                        if (lane == (it & 15)) {
-                            if (un.eight)
-                                bulk_g2s(S.A[s], reinterpret_cast<const uint8_t*>(g.codes8) + blk * kABytes, cbytes,
-                                         &full[s]);
-                            else
-                                bulk_g2s(S.R[s], g.codes4 + blk * kRawBytes, cbytes, &full[s]);
-                        }
-                        if (zbytes != 0 && lane == 16 + (it & 15))
-                            bulk_g2s(S.Z[s], g.zeros4 + (size_t(un.lt) * g.G + size_t(kb) * gpk) * kTileRows, zbytes,
-                                     &full[s]);
-                    } else {
-                        // tokens past M read as zeros; the box is always counted whole
-                        if (lane == 0) mbar_arrive_expect_tx(&full[s], uint32_t(C::kBBytes));
-                        __syncwarp();
-                        if (lane == (it & 31)) tma_load_3d(S.B[s], &amap, 0, 0, kb, &full[s]);
-                    }
+                const int w = un.eight ? 2 : 1;
+                const int ns = (un.kb1 - un.kb0) * w;       // the unit's slots
+                const size_t blk = size_t(un.lt) * g.kblocks + un.kb0;
+                // slot o of the unit holds bytes [o, o + 1) x 8 KB of its codes
+                const uint8_t* src = un.eight ? reinterpret_cast<const uint8_t*>(g.codes8) + blk * kABytes
+                                              : g.codes4 + blk * kSlotBytes;
+                const uint8_t* zsrc = g.zeros4 + (size_t(un.lt) * g.G + size_t(un.kb0) * gpk) * kTileRows;
+                for (int o = 0; o < ns;) {
+                    const int take = min(ns - o, kCR - ir % kCR);
+                    run[nrun].src = src + size_t(o) * kSlotBytes;
+                    run[nrun].zsrc = zsrc + size_t(o) * gpk * kTileRows;
+                    run[nrun].slot = ir;
+                    run[nrun].bytes = uint32_t(take * kSlotBytes);
+                    run[nrun].zbytes = un.eight ? 0u : uint32_t(take * gpk * BM);
+                    ++nrun;
+                    ir += take;
+                    o += take;
+                    if (ir % kCR == 0 && !flush(ir)) goto wload_done;
                 }
             }
+            if (ir % kCR != 0) flush(ir);
         }
-    load_done:
-        // no copy may target this CTA's shared memory after it exits
-        if (lane == 0)
-            for (int j = max(0, it - C::kStages); j < it; ++j) {
+    wload_done:
+        // no copy may target this CTA's shared memory after it exits: wait for the
+        // last use of every chunk place
+        if (lane == 0 && armed > 0) {
+            const int last = (armed - 1) & ~(kCR - 1);
+            for (int b = max(0, last - C::kR + kCR); b <= last; b += kCR) {
                 int dummy = 0;
-                mbar_wait_bounded(&full[j % C::kStages], (j / C::kStages) & 1, &dummy, nullptr, a.timeout_ns);
+                mbar_wait_bounded(&S.r_full[b % C::kR], (b / C::kR) & 1, &dummy, nullptr, a.timeout_ns);
             }
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ token copies (B ring)
+        griddep_wait();                              // the tokens come from the previous kernel
+        constexpr int kCB = C::kCB;
+        TRun run[kCB];
+        int nrun = 0, ia = 0, armed = 0, nchunk = 0;
+        auto flush = [&](int end) -> bool {
+            const int base = (end - 1) & ~(kCB - 1);
+            const int ci = base / kCB;
+            bool ok = true;
+            if (lane == 0) {
+                // the chunk's place released in the previous pass (one arrival per issuer)
+                ok = mbar_wait_bounded(&S.b_empty[ci % C::kBChunks], ((ci / C::kBChunks) & 1) ^ 1, abort, a.status,
+                                       a.timeout_ns);
+                // tokens past M read as zeros; the boxes are always counted whole
+                if (ok) mbar_arrive_expect_tx(&S.b_full[base % C::kB], uint32_t((end - base) * C::kBBytes));
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+            uint64_t* bar = &S.b_full[base % C::kB];
+            int l = (nchunk * kCB) & 31;
+            for (int j = 0; j < nrun; ++j) {
+                if (run[j].n == kCB) {
+                    if (lane == (l & 31)) tma_load_3d(S.B[run[j].stage % C::kB], &amapC, 0, 0, run[j].kb, bar);
+                    ++l;
+                } else {
+                    for (int t = 0; t < run[j].n; ++t, ++l)
+                        if (lane == (l & 31)) tma_load_3d(S.B[(run[j].stage + t) % C::kB], &amap1, 0, 0, run[j].kb + t, bar);
+                }
+            }
+            nrun = 0;
+            ++nchunk;
+            armed = end;
+            return true;
+        };
+        if (!a.stall_test) {
+            for (int u = blockIdx.x; u < a.n_units; u += gridDim.x) {
+                const Unit un = unit_of(a, u);
+                for (int kb = un.kb0; kb < un.kb1;) {
+                    const int take = min(un.kb1 - kb, kCB - ia % kCB);
+                    run[nrun].kb = kb;
+                    run[nrun].n = take;
+                    run[nrun].stage = ia;
+                    ++nrun;
+                    ia += take;
+                    kb += take;
+                    if (ia % kCB == 0 && !flush(ia)) goto tload_done;
+                }
+            }
+            if (ia % kCB != 0) flush(ia);
+        }
+    tload_done:
+        if (lane == 0 && armed > 0) {
+            const int last = (armed - 1) & ~(kCB - 1);
+            for (int b = max(0, last - C::kB + kCB); b <= last; b += kCB) {
+                int dummy = 0;
+                mbar_wait_bounded(&S.b_full[b % C::kB], (b / C::kB) & 1, &dummy, nullptr, a.timeout_ns);
+            }
+        }
     } else if (warp <= 2) {
         // ------------------------------------------------------------ MMAs
         // issuer `mine` takes the groups with gc % 2 == mine (accumulators of that parity)
         const uint32_t mine = uint32_t(warp - 1);
         if (lane == 0) {
             const uint32_t idesc = idesc_i8(BM, NT);
-            int it = 0;
+            int ia = 0, hb_seen = -1;
             uint32_t gc = 0;
+            bool any = false;                        // an MMA of mine reads the current token chunk
             for (int u = blockIdx.x; u < a.n_units; u += gridDim.x) {
                 const Unit un = unit_of(a, u);
-                for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
-                    const int s = it % C::kStages;
-                    const uint32_t ph = (it / C::kStages) & 1;
-                    // a stage without a group of mine (one group per k-block): skip it
-                    if (gpk == 1 && (gc & 1u) != mine) {
-                        ++gc;
-                        continue;
-                    }
-                    if (!mbar_wait_bounded(&S.ready[s], ph, abort, a.status, a.timeout_ns)) goto mma_out;
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(S.A[s]), b0 = smem_u32(S.B[s]);
-                    for (int j = 0; j < gpk; ++j, ++gc) {
-                        if ((gc & 1u) != mine) continue;
-                        const uint32_t b = gc % C::kSlots;
-                        // use gc / kSlots of accumulator b: phase 0 is the epilogue's first release
-                        if (!mbar_wait_bounded(&S.acc_empty[b], (gc / C::kSlots) & 1, abort, a.status, a.timeout_ns))
+                const bool last_unit = u + int(gridDim.x) >= a.n_units;
+                for (int kb = un.kb0; kb < un.kb1; ++kb, ++ia) {
+                    const int sa = ia % C::kA, sb = ia % C::kB;
+                    if (gpk == 2 || (gc & 1u) == mine) {
+                        // the k-block's tokens: their chunk's barrier, once per chunk (every chunk
+                        // but the last holds k-blocks of both issuers, so each issuer waits on
+                        // every chunk barrier in the order of its phases)
+                        const int hb = ia & ~(C::kCB - 1);
+                        if (hb != hb_seen) {
+                            if (!mbar_wait_bounded(&S.b_full[hb % C::kB], (hb / C::kB) & 1, abort, a.status,
+                                                   a.timeout_ns))
+                                goto mma_out;
+                            hb_seen = hb;
+                        }
+                        if (!mbar_wait_bounded(&S.ready[sa], (ia / C::kA) & 1, abort, a.status, a.timeout_ns))
                             goto mma_out;
                         tc_fence_after();
-                        // the group's first k-step overwrites the accumulator
-                        for (int kk = 0; kk < ksteps; ++kk) {
-                            const uint32_t off = uint32_t(j * g.group + kk * 32);
-                            mma_i8(tmem + b * NT, sw128_kmajor_desc(a0 + off), sw128_kmajor_desc(b0 + off), idesc,
-                                   kk > 0 ? 1u : 0u);
+                        const uint32_t a0 = smem_u32(S.A[sa]), b0 = smem_u32(S.B[sb]);
+                        for (int j = 0; j < gpk; ++j, ++gc) {
+                            if ((gc & 1u) != mine) continue;
+                            const uint32_t b = gc % C::kSlots;
+                            // use gc / kSlots of accumulator b: phase 0 is the epilogue's first release
+                            if (!mbar_wait_bounded(&S.acc_empty[b], (gc / C::kSlots) & 1, abort, a.status,
+                                                   a.timeout_ns))
+                                goto mma_out;
+                            tc_fence_after();
+                            // the group's first k-step overwrites the accumulator
+                            for (int kk = 0; kk < ksteps; ++kk) {
+                                const uint32_t off = uint32_t(j * g.group + kk * 32);
+                                mma_i8(tmem + b * NT, sw128_kmajor_desc(a0 + off), sw128_kmajor_desc(b0 + off),
+                                       idesc, kk > 0 ? 1u : 0u);
+                            }
+                            mma_commit(&S.acc_full[b]);
+                            mma_commit(&S.a_empty[sa]);
+                            any = true;
                         }
-                        mma_commit(&S.acc_full[b]);
-                        mma_commit(&S.empty[s]);
+                    } else {
+                        ++gc;                        // the other issuer's group
+                    }
+                    // leaving a token chunk: release it (after my MMAs that read it)
+                    if ((ia + 1) % C::kCB == 0 || (last_unit && kb + 1 == un.kb1)) {
+                        uint64_t* be = &S.b_empty[(ia / C::kCB) % C::kBChunks];
+                        if (any) mma_commit(be);
+                        else mbar_arrive(be);
+                        any = false;
                     }
                 }
             }
@@ -261,50 +421,94 @@ gemm_tcd_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
             int dummy = 0;
             mbar_wait_bounded(&S.mma_done[mine], 0, &dummy, nullptr, a.timeout_ns);
         }
-    } else if (warp < C::kEpiWarp0) {
-        // ------------------------------------------------------------ widening (4-bit rows)
-        constexpr int kWidenThreads = C::kWidenThreads, kWidenChunks = C::kWidenChunks;
-        const int wt = threadIdx.x - kWiden0 * 32;
-        int it = 0;
+    } else if (warp >= kWiden0 && warp < C::kEpiWarp0) {
+        // ------------------------------------------------------------ widening (R ring -> A ring)
+        // group q (kGW warps) widens the k-blocks with ia % kGroups == q into operand
+        // stage ia % kA (always its own).  Every group waits on every weight chunk's
+        // barrier and releases every chunk, in order: the copy thread re-arms a chunk
+        // only after all widening warps released it, so no group can be two phases
+        // away from a barrier it waits on
+        constexpr int kGT = C::kGT, kPer = kSlotBytes / 16 / kGT;   // 16-byte chunks per thread and slot
+        const int q = (warp - kWiden0) / kGW;
+        const int gt = threadIdx.x - (kWiden0 + q * kGW) * 32;      // thread within the group
+        int ir = 0, ia = 0;
+        int entered = -kCR, released = 0;           // last weight chunk waited on, next to release
         for (int u = blockIdx.x; u < a.n_units; u += gridDim.x) {
             const Unit un = unit_of(a, u);
-            for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
-                const int s = it % C::kStages;
-                const uint32_t ph = (it / C::kStages) & 1;
-                // the weights to widen, then the tokens: the MMA needs both
-                bool ok = mbar_wait_bounded(&S.full_w[s], ph, abort, a.status, a.timeout_ns);
-                ok = ok && mbar_wait_bounded(&S.full_t[s], ph, abort, a.status, a.timeout_ns);
+            const int w = un.eight ? 2 : 1;
+            const int ufs = ir;                      // the unit's first slot
+            for (int kb = un.kb0; kb < un.kb1; ++kb, ++ia, ir += w) {
+                // enter the chunks up to the one holding the k-block's last slot
+                bool ok = true;
+                while (ok && entered + kCR <= ir + w - 1) {
+                    entered += kCR;
+                    ok = mbar_wait_bounded(&S.r_full[entered % C::kR], (entered / C::kR) & 1, abort, a.status,
+                                           a.timeout_ns);
+                }
                 if (!__all_sync(0xffffffffu, ok)) goto widen_done;
-                if (!un.eight) {
-                    const uint8_t* raw = S.R[s];
-                    uint8_t* out = S.A[s];
-                    const uint8_t* zs = S.Z[s];
-                    uint4 w[kWidenChunks];
+                if (ia % C::kGroups == q) {
+                    const int sa = ia % C::kA;
+                    ok = mbar_wait_bounded(&S.a_empty[sa], ((ia / C::kA) & 1) ^ 1, abort, a.status, a.timeout_ns);
+                    if (!__all_sync(0xffffffffu, ok)) goto widen_done;
+                    uint8_t* out = S.A[sa];
+                    if (!un.eight) {
+                        // the run holding this slot starts at the later of its chunk's and its unit's first slot
+                        const int h0 = ir & ~(kCR - 1), rs = max(h0, ufs);
+                        const uint8_t* raw = S.R[ir % C::kR];
+                        const uint8_t* zs = &S.Z[rs % C::kR][0] + (ir - rs) * gpk * BM;
+                        uint4 wv[kPer];
+                        uint32_t zb[kPer];
 #pragma unroll
-                    for (int j = 0; j < kWidenChunks; ++j)
-                        w[j] = *reinterpret_cast<const uint4*>(raw + (wt + kWidenThreads * j) * 16);
+                        for (int j = 0; j < kPer; ++j) {
+                            const int i = gt + kGT * j, r = i >> 2, c = i & 3;
+                            wv[j] = *reinterpret_cast<const uint4*>(raw + i * 16);
+                            // z of the group holding this chunk's 32 codes
+                            zb[j] = zs[(gpk == 2 ? (c >> 1) : 0) * BM + r];
+                        }
 #pragma unroll
-                    for (int j = 0; j < kWidenChunks; ++j) {
-                        const int i = wt + kWidenThreads * j, r = i >> 2, c = i & 3;
-                        // (128 - z) in every byte, z of the group holding this chunk's 32 codes
-                        const uint32_t zc = (0x80u - uint32_t(zs[(c * 32 / g.group) * BM + r])) * 0x01010101u;
-                        uint4 o0, o1;
-                        o0.x = widen_lo(w[j].x, zc); o0.y = widen_hi(w[j].x, zc);
-                        o0.z = widen_lo(w[j].y, zc); o0.w = widen_hi(w[j].y, zc);
-                        o1.x = widen_lo(w[j].z, zc); o1.y = widen_hi(w[j].z, zc);
-                        o1.z = widen_lo(w[j].w, zc); o1.w = widen_hi(w[j].w, zc);
-                        *reinterpret_cast<uint4*>(out + swz128_offset(r, 2 * c)) = o0;
-                        *reinterpret_cast<uint4*>(out + swz128_offset(r, 2 * c + 1)) = o1;
+                        for (int j = 0; j < kPer; ++j) {
+                            const int i = gt + kGT * j, r = i >> 2, c = i & 3;
+                            const uint32_t zc = (0x80u - zb[j]) * 0x01010101u;   // (128 - z) in every byte
+                            uint4 o0, o1;
+                            o0.x = widen_lo(wv[j].x, zc); o0.y = widen_hi(wv[j].x, zc);
+                            o0.z = widen_lo(wv[j].y, zc); o0.w = widen_hi(wv[j].y, zc);
+                            o1.x = widen_lo(wv[j].z, zc); o1.y = widen_hi(wv[j].z, zc);
+                            o1.z = widen_lo(wv[j].w, zc); o1.w = widen_hi(wv[j].w, zc);
+                            *reinterpret_cast<uint4*>(out + swz128_offset(r, 2 * c)) = o0;
+                            *reinterpret_cast<uint4*>(out + swz128_offset(r, 2 * c + 1)) = o1;
+                        }
+                    } else {
+                        // the stored 8-bit operand is already in the MMA's layout: its two
+                        // slots (the second may wrap to the ring's start) copied as they are
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint8_t* raw = S.R[(ir + h) % C::kR];
+                            uint4 wv[kPer];
+#pragma unroll
+                            for (int j = 0; j < kPer; ++j) wv[j] = *reinterpret_cast<const uint4*>(raw + (gt + kGT * j) * 16);
+#pragma unroll
+                            for (int j = 0; j < kPer; ++j)
+                                *reinterpret_cast<uint4*>(out + h * kSlotBytes + (gt + kGT * j) * 16) = wv[j];
+                        }
                     }
                     fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.ready[sa]);
                 }
+                // release the chunks whose slots all precede the next k-block
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&S.ready[s]);
+                for (; released + kCR <= ir + w; released += kCR)
+                    if (lane == 0) mbar_arrive(&S.r_rel[(released % C::kR) / kCR]);
             }
         }
+        // the last, partly filled chunk
+        __syncwarp();
+        for (; released <= entered; released += kCR)
+            if (lane == 0) mbar_arrive(&S.r_rel[(released % C::kR) / kCR]);
     widen_done:;
-    } else {
+    } else if (warp >= C::kEpiWarp0) {
         // ------------------------------------------------------------ epilogue
+        griddep_wait();                              // s_a, Y and part belong to the stream's order
         constexpr int kCols = C::kEpiCols, kPiece = C::kPiece;
         const int e = warp - C::kEpiWarp0;
         const int q = warp & 3;                      // TMEM lane quarter of this warp
@@ -408,10 +612,13 @@ gemm_tcd_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
 }
 
 template <int NT>
-size_t tcd_smem() { return sizeof(Smem<NT>) + 1024; }
+size_t tcd_smem() {
+    static_assert(sizeof(Smem<NT>) + 1024 <= 227 * 1024, "shared memory of one CTA");
+    return sizeof(Smem<NT>) + 1024;
+}
 
 template <int NT>
-cudaError_t launch_nt(const mx_layout& L, const CUtensorMap& map, const TcdArgs& a, int grid, bool debug, int ag,
+cudaError_t launch_nt(const CUtensorMap& map1, const CUtensorMap& mapC, const TcdArgs& a, int grid, bool debug, int ag,
                       cudaStream_t s) {
     static bool configured[64] = {};
     int dev = 0;
@@ -428,8 +635,17 @@ cudaError_t launch_nt(const mx_layout& L, const CUtensorMap& map, const TcdArgs&
     }
     auto k = debug ? (ag ? gemm_tcd_kernel<NT, true, true> : gemm_tcd_kernel<NT, true, false>)
                    : (ag ? gemm_tcd_kernel<NT, false, true> : gemm_tcd_kernel<NT, false, false>);
-    k<<<grid, Cfg<NT>::kThreads, tcd_smem<NT>(), s>>>(map, a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(Cfg<NT>::kThreads);
+    cfg.dynamicSmemBytes = tcd_smem<NT>();
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // weights stream before the wait
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, map1, mapC, a);
 }
 
 }  // namespace
@@ -476,17 +692,20 @@ cudaError_t launch_gemm_tcd(const mx_layout& L, const void* blob, const int8_t* 
     EncodeTiledFn enc = encode_fn(&e);
     if (e != cudaSuccess) return e;
     const int NT = tcd_tokens(M);
-    // activations as a 3-D tensor [k-block][token][128 bytes]: one box brings one
-    // k-block of the batch as swizzled 128-byte rows
-    CUtensorMap map;
+    // activations as a 3-D tensor [k-block][token][128 bytes]: one box brings one k-block
+    // of the batch as swizzled 128-byte rows (map1), or a chunk of consecutive k-blocks
+    // (mapC)
+    CUtensorMap map1, mapC;
     const cuuint64_t dims[3] = {cuuint64_t(kKBlock), cuuint64_t(M), cuuint64_t(L.kblocks)};
     const cuuint64_t strides[2] = {cuuint64_t(L.K), cuuint64_t(kKBlock)};
-    const cuuint32_t box[3] = {cuuint32_t(kKBlock), cuuint32_t(NT), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(Aq), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    for (int z : {1, token_chunk(NT)}) {
+        const cuuint32_t box[3] = {cuuint32_t(kKBlock), cuuint32_t(NT), cuuint32_t(z)};
+        CUresult r = enc(z == 1 ? &map1 : &mapC, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(Aq), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
     TcdArgs a{};
     a.g = make_geom(L, blob);
     a.s_a = reinterpret_cast<const __half*>(s_a);
@@ -505,10 +724,10 @@ cudaError_t launch_gemm_tcd(const mx_layout& L, const void* blob, const int8_t* 
     const int grid = std::min(a.n_units, sms);
     const bool dbg = debug_partials != nullptr;
     switch (NT) {
-        case 16: e = launch_nt<16>(L, map, a, grid, dbg, ag, s); break;
-        case 32: e = launch_nt<32>(L, map, a, grid, dbg, ag, s); break;
-        case 64: e = launch_nt<64>(L, map, a, grid, dbg, ag, s); break;
-        default: e = launch_nt<128>(L, map, a, grid, dbg, ag, s); break;
+        case 16: e = launch_nt<16>(map1, mapC, a, grid, dbg, ag, s); break;
+        case 32: e = launch_nt<32>(map1, mapC, a, grid, dbg, ag, s); break;
+        case 64: e = launch_nt<64>(map1, mapC, a, grid, dbg, ag, s); break;
+        default: e = launch_nt<128>(map1, mapC, a, grid, dbg, ag, s); break;
     }
     if (e != cudaSuccess || a.S == 1) return e;
     return launch_split_reduce(a.part, a.S, M, L.N, s_a, ag, Y, ldy, sms, s);
