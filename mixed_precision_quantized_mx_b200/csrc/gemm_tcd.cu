@@ -652,23 +652,28 @@ cudaError_t launch_nt(const CUtensorMap& map1, const CUtensorMap& mapC, const Tc
 
 int tcd_tokens(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
 
-// The K split with the smallest estimated time: the larger of the streaming time of
-// the weights plus the split sums (written, then read back by the reduction) and the
-// time of the k-blocks the busiest SM processes, plus a launch for the reduction.
-// The estimates assume HBM at about 6 TB/s and about 0.2 us per k-block and SM.
+// The K split with the smallest estimated time: the units the busiest SM processes
+// (waves), each costing its k-blocks at the time one k-block takes an SM at this
+// token tile plus the fill and drain of the pipeline, as measured on this part
+// (about 0.45 us per k-block at 16 tokens to 0.9 us at 128, where the epilogue
+// drains larger accumulators, and about 3 us per unit); a split adds the reduction
+// kernel and the split sums (written, then read back), and the weights cannot stream
+// faster than HBM (about 6 TB/s).
 int tcd_auto_split(const mx_layout& L, int M, int sms) {
     const int tiles = L.t8 + L.t4, nkb = L.kblocks;
     if (M <= 0 || sms <= 0) return 1;
-    const double bw = 6.0e6, t_kb = 0.2, t_launch = 2.0;          // bytes per us, us, us
+    const int NT = tcd_tokens(M);
+    const double t_kb = NT <= 16 ? 0.45 : NT <= 32 ? 0.55 : NT <= 64 ? 0.68 : 0.9;   // us per k-block and SM
+    const double bw = 6.0e6, t_unit = 3.0, t_split = 4.0;                             // bytes per us, us, us
     const double wbytes = double(L.n8) * L.K + double(L.n4) * L.K / 2 + 2.5 * double(L.N) * L.G;
     int best = 1;
     double best_t = 1e30;
     for (int S = 1; S <= kTcdMaxSplit && S <= nkb; ++S) {
         const int per = (nkb + S - 1) / S;
         if ((nkb + per - 1) / per != S) continue;            // no empty split
-        const double sums = S > 1 ? 8.0 * S * M * double(L.N) : 0.0;
-        const double t = std::max(double((tiles * S + sms - 1) / sms) * per * t_kb, (wbytes + sums) / bw) +
-                         (S > 1 ? t_launch : 0.0);
+        const double waves = double((tiles * S + sms - 1) / sms);
+        const double t = std::max(waves * (per * t_kb + t_unit), wbytes / bw) +
+                         (S > 1 ? t_split + 8.0 * S * M * double(L.N) / bw : 0.0);
         if (t < best_t) {
             best_t = t;
             best = S;

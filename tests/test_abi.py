@@ -125,10 +125,9 @@ def test_gemm_workspace_and_dispatch_on_m(lib):
     for M in (1, 8, 2048):
         assert mx.mx_gemm_workspace_size(L, M) == 0
     # 33 row tiles of 128 rows: at 9..128 tokens the decode tensor-core path splits K
-    # (four ways: 132 units for 148 SMs; two at 100 tokens, whose split sums cost more)
-    # and sums the splits in a workspace
+    # four ways (132 units for 148 SMs) and sums the splits in a workspace
     a256 = lambda v: (v + 255) // 256 * 256
-    for M, S in ((16, 4), (17, 4), (100, 2)):
+    for M, S in ((16, 4), (17, 4), (100, 4)):
         assert mx.mx_gemm_workspace_size(L, M) == a256(S * M * 4096 * 4)
     assert mx.mx_gemm_workspace_size(L, 17, split=3) == a256(3 * 17 * 4096 * 4)
     assert mx.mx_gemm_workspace_size(L, 17, path=mx.PATH_TENSOR) == 0     # the one-CTA kernel
