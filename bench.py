@@ -43,13 +43,15 @@ WORKLOADS = {
     "llama3-8b-down-m2048": (2048, 14336, 4096),
     "llama3-70b-up-m1": (1, 8192, 28672),
     "llama3-70b-down-m1": (1, 28672, 8192),
+    "llama3-70b-up-m16": (16, 8192, 28672),
+    "llama3-70b-down-m16": (16, 28672, 8192),
     "llama3-70b-up-m4096": (4096, 8192, 28672),
     "llama3-70b-down-m4096": (4096, 28672, 8192),
 }
 DEFAULT_WORKLOAD = "llama3-70b-up-m4096"
 # lines measured after the named workload in the same run: the same weights at another M
-SECONDARY = {"llama3-70b-up-m4096": ("llama3-70b-up-m1",),
-             "llama3-70b-down-m4096": ("llama3-70b-down-m1",)}
+SECONDARY = {"llama3-70b-up-m4096": ("llama3-70b-up-m1", "llama3-70b-up-m16"),
+             "llama3-70b-down-m4096": ("llama3-70b-down-m1", "llama3-70b-down-m16")}
 HBM_BOUND_MAX_M = 128        # below the ~150-token ridge the step is bound by HBM
 
 
