@@ -33,8 +33,8 @@ __device__ __forceinline__ float scale16(float s32) {
     return __half2float(h);
 }
 
-// E consecutive elements as fp32: one vector load (streaming, read once) when kVec,
-// else E scalar loads
+// E consecutive elements as fp32: 16-byte vector loads (streaming, read once) when
+// kVec, else E scalar loads
 template <typename T, int E, bool kVec> struct Vec;
 template <int E> struct Vec<float, E, false> {
     static __device__ __forceinline__ void load(const float* p, float (&v)[E]) {
@@ -48,43 +48,43 @@ template <int E> struct Vec<__half, E, false> {
         for (int e = 0; e < E; ++e) v[e] = __half2float(__ldg(p + e));
     }
 };
-template <> struct Vec<float, 4, true> {
-    static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
-        const float4 x = __ldcs(reinterpret_cast<const float4*>(p));
-        v[0] = x.x, v[1] = x.y, v[2] = x.z, v[3] = x.w;
+template <int E> struct Vec<float, E, true> {
+    static_assert(E % 4 == 0, "whole float4 loads");
+    static __device__ __forceinline__ void load(const float* p, float (&v)[E]) {
+#pragma unroll
+        for (int j = 0; j < E / 4; ++j) {
+            const float4 x = __ldcs(reinterpret_cast<const float4*>(p) + j);
+            v[4 * j] = x.x, v[4 * j + 1] = x.y, v[4 * j + 2] = x.z, v[4 * j + 3] = x.w;
+        }
     }
 };
-template <> struct Vec<float, 2, true> {
-    static __device__ __forceinline__ void load(const float* p, float (&v)[2]) {
-        const float2 x = __ldcs(reinterpret_cast<const float2*>(p));
-        v[0] = x.x, v[1] = x.y;
-    }
-};
-template <> struct Vec<__half, 4, true> {
-    static __device__ __forceinline__ void load(const __half* p, float (&v)[4]) {
-        const uint2 x = __ldcs(reinterpret_cast<const uint2*>(p));
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&x.x));
-        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&x.y));
-        v[0] = a.x, v[1] = a.y, v[2] = b.x, v[3] = b.y;
-    }
-};
-template <> struct Vec<__half, 2, true> {
-    static __device__ __forceinline__ void load(const __half* p, float (&v)[2]) {
-        const unsigned x = __ldcs(reinterpret_cast<const unsigned*>(p));
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&x));
-        v[0] = a.x, v[1] = a.y;
+template <int E> struct Vec<__half, E, true> {
+    static_assert(E % 8 == 0, "whole 16-byte loads");
+    static __device__ __forceinline__ void load(const __half* p, float (&v)[E]) {
+#pragma unroll
+        for (int j = 0; j < E / 8; ++j) {
+            const uint4 x = __ldcs(reinterpret_cast<const uint4*>(p) + j);
+            const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[h]));
+                v[8 * j + 2 * h] = f.x, v[8 * j + 2 * h + 1] = f.y;
+            }
+        }
     }
 };
 
 // One row is scored by `split` warps (1, 2, 4 or 8), each over a contiguous range of
-// groups; a group of 32 E columns is one load of E elements per lane, and U groups
-// are loaded before any is used, so each lane has U (E of W + E of G) in flight.  The
-// warps' fp64 partial sums are added in warp order (deterministic for a shape).
-template <typename TW, typename TG, int E, int U, bool kVec>
+// groups.  A group of kL * E columns is kL lanes of E consecutive elements, so a warp
+// takes 32 / kL groups at a time: the group's range needs log2(kL) shuffle steps and
+// its scale and zero point are computed once per E elements of a lane.  U such steps
+// are loaded before any is used (U (E of W + E of G) per lane in flight).  The warps'
+// fp64 partial sums are added in warp order (deterministic for a shape).
+template <typename TW, typename TG, int E, int kL, int U, bool kVec>
 __global__ void __launch_bounds__(kSalWarps * 32)
 saliency_kernel(const TW* __restrict__ W, int64_t ldw, const TG* __restrict__ G, int64_t ldg, int N, int K,
                 int split, float* __restrict__ S) {
-    constexpr int kGroup = 32 * E;
+    constexpr int kGroup = kL * E, kGPW = 32 / kL;   // columns per group, groups per warp step
     __shared__ double part_sum[kSalWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int slot = warp / split, part = warp % split;
@@ -92,49 +92,55 @@ saliency_kernel(const TW* __restrict__ W, int64_t ldw, const TG* __restrict__ G,
     const int n_groups = K / kGroup;
     const int per = (n_groups + split - 1) / split;
     const int g_begin = min(n_groups, part * per), g_end = min(n_groups, g_begin + per);
+    const int sub = lane / kL;                       // this lane's group within a warp step
     double s1 = 0.0;
-    if (n < N) {                                   // warp-uniform
-        const TW* w_row = W + int64_t(n) * ldw + lane * E;
-        const TG* g_row = G + int64_t(n) * ldg + lane * E;
-        for (int gi = g_begin; gi < g_end; gi += U) {
+    if (n < N) {                                     // warp-uniform
+        const TW* w_row = W + int64_t(n) * ldw + (lane % kL) * E;
+        const TG* g_row = G + int64_t(n) * ldg + (lane % kL) * E;
+        for (int gi = g_begin; gi < g_end; gi += U * kGPW) {
             float w[U][E], gv[U][E];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                if (gi + u < g_end) {              // warp-uniform
-                    Vec<TW, E, kVec>::load(w_row + int64_t(gi + u) * kGroup, w[u]);
-                    Vec<TG, E, kVec>::load(g_row + int64_t(gi + u) * kGroup, gv[u]);
+                const int grp = gi + u * kGPW + sub;
+                if (grp < g_end) {
+                    Vec<TW, E, kVec>::load(w_row + int64_t(grp) * kGroup, w[u]);
+                    Vec<TG, E, kVec>::load(g_row + int64_t(grp) * kGroup, gv[u]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) w[u][e] = 0.0f, gv[u][e] = 0.0f;
                 }
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                if (gi + u < g_end) {
-                    // the group's range (0 included), then its fp16 scale and zero point
-                    float lo = 0.0f, hi = 0.0f;
+                if (gi + u * kGPW >= g_end) break;   // warp-uniform: no group of this step
+                const bool valid = gi + u * kGPW + sub < g_end;
+                // the group's range (0 included), then its fp16 scale and zero point
+                float lo = 0.0f, hi = 0.0f;
 #pragma unroll
-                    for (int e = 0; e < E; ++e) lo = fminf(lo, w[u][e]), hi = fmaxf(hi, w[u][e]);
+                for (int e = 0; e < E; ++e) lo = fminf(lo, w[u][e]), hi = fmaxf(hi, w[u][e]);
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-                        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-                    }
-                    const float sc = scale16(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
-                    const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, sc)), 0.0f), 15.0f);
-                    const float rc = __frcp_rn(sc);
+                for (int o = kL / 2; o > 0; o >>= 1) {   // within the group's kL lanes
+                    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+                    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+                }
+                if (!valid) continue;
+                const float sc = scale16(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
+                const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, sc)), 0.0f), 15.0f);
+                const float rc = __frcp_rn(sc);
 #pragma unroll
-                    for (int e = 0; e < E; ++e) {
-                        // round(w / s) from w * (1 / s): the two differ by at most 3 2^-24 |w / s|,
-                        // so they round alike unless the product is within 2^-11 of a half-integer
-                        // (for |w / s| <= 1024; beyond that both clamp alike); there the exact
-                        // quotient decides, as in the packer
-                        const float t = __fmul_rn(w[u][e], rc);
-                        float rq = rintf(t);
-                        if (fabsf(t) <= 1024.0f && fabsf(fabsf(t - floorf(t)) - 0.5f) < 4.8828125e-4f)
-                            rq = rintf(__fdiv_rn(w[u][e], sc));
-                        const float q = fminf(fmaxf(rq + zf, 0.0f), 15.0f);
-                        // (q - z) s is exact in fp32; the difference with w is taken in fp64
-                        const double d = double(__fmul_rn(q - zf, sc)) - double(w[u][e]);
-                        s1 = fma(double(gv[u][e]), d, s1);
-                    }
+                for (int e = 0; e < E; ++e) {
+                    // round(w / s) from w * (1 / s): the two differ by at most 3 2^-24 |w / s|,
+                    // so they round alike unless the product is within 2^-11 of a half-integer
+                    // (for |w / s| <= 1024; beyond that both clamp alike); there the exact
+                    // quotient decides, as in the packer
+                    const float t = __fmul_rn(w[u][e], rc);
+                    float rq = rintf(t);
+                    if (fabsf(t) <= 1024.0f && fabsf(fabsf(t - floorf(t)) - 0.5f) < 4.8828125e-4f)
+                        rq = rintf(__fdiv_rn(w[u][e], sc));
+                    const float q = fminf(fmaxf(rq + zf, 0.0f), 15.0f);
+                    // (q - z) s is exact in fp32; the difference with w is taken in fp64
+                    const double d = double(__fmul_rn(q - zf, sc)) - double(w[u][e]);
+                    s1 = fma(double(gv[u][e]), d, s1);
                 }
             }
         }
@@ -203,31 +209,34 @@ select_mark_kernel(const float* __restrict__ S, int64_t n, int64_t n_top, const 
         is8[i] = n_top >= n ? 1 : (n_top == 0 ? 0 : (sel_key(S, i) >= T ? 1 : 0));
 }
 
-template <typename TW, typename TG, int E, int U>
+template <typename TW, typename TG, int E, int kL, int U>
 cudaError_t launch_saliency_t(const void* W, int64_t ldw, const void* G, int64_t ldg, int N, int K, int split,
                               float* S, cudaStream_t s) {
     const TW* w = static_cast<const TW*>(W);
     const TG* g = static_cast<const TG*>(G);
-    // vector loads when every row's E-element runs are aligned to the vector size
-    const bool vec = reinterpret_cast<uintptr_t>(W) % (E * sizeof(TW)) == 0 && ldw % E == 0 &&
-                     reinterpret_cast<uintptr_t>(G) % (E * sizeof(TG)) == 0 && ldg % E == 0;
+    // vector loads when every row's E-element runs start on 16 bytes
+    const bool vec = reinterpret_cast<uintptr_t>(W) % 16 == 0 && (ldw * int64_t(sizeof(TW))) % 16 == 0 &&
+                     reinterpret_cast<uintptr_t>(G) % 16 == 0 && (ldg * int64_t(sizeof(TG))) % 16 == 0 &&
+                     (E * sizeof(TW)) % 16 == 0 && (E * sizeof(TG)) % 16 == 0;
     const dim3 grid((N + kSalWarps / split - 1) / (kSalWarps / split)), block(kSalWarps * 32);
     if (vec)
-        saliency_kernel<TW, TG, E, U, true><<<grid, block, 0, s>>>(w, ldw, g, ldg, N, K, split, S);
+        saliency_kernel<TW, TG, E, kL, U, true><<<grid, block, 0, s>>>(w, ldw, g, ldg, N, K, split, S);
     else
-        saliency_kernel<TW, TG, E, U, false><<<grid, block, 0, s>>>(w, ldw, g, ldg, N, K, split, S);
+        saliency_kernel<TW, TG, E, kL, U, false><<<grid, block, 0, s>>>(w, ldw, g, ldg, N, K, split, S);
     return cudaGetLastError();
 }
 
 template <typename TW, typename TG>
 cudaError_t launch_saliency_g(const void* W, int64_t ldw, const void* G, int64_t ldg, int N, int K, int group,
                               float* S, cudaStream_t s) {
-    // warps per row: enough rows' warps to fill every SM about 32 warps deep, at most
-    // one warp per group
+    // 8 lanes per group (16 elements each at group 128, 8 at 64): four groups per warp
+    // step.  Warps per row: enough rows' warps to fill every SM about 32 warps deep,
+    // while each warp keeps at least two steps of groups
+    constexpr int kL = 8, kGPW = 32 / kL;
     int split = 1;
-    while (split < kSalWarps && int64_t(N) * split < 148 * 32 && 2 * split <= K / group) split *= 2;
-    return group == 128 ? launch_saliency_t<TW, TG, 4, 4>(W, ldw, G, ldg, N, K, split, S, s)
-                        : launch_saliency_t<TW, TG, 2, 8>(W, ldw, G, ldg, N, K, split, S, s);
+    while (split < kSalWarps && int64_t(N) * split < 148 * 32 && 2 * split * 2 * kGPW <= K / group) split *= 2;
+    return group == 128 ? launch_saliency_t<TW, TG, 16, kL, 2>(W, ldw, G, ldg, N, K, split, S, s)
+                        : launch_saliency_t<TW, TG, 8, kL, 4>(W, ldw, G, ldg, N, K, split, S, s);
 }
 
 }  // namespace
