@@ -19,7 +19,11 @@
 // zero point gives four int8 (q - z) for dp4a with the token's activations.  The
 // lane keeps s_w * (its partial) in fp32 per token; one warp sum and s_a at the
 // end give Y.  With a partials buffer the exact int32 P[m, n, kb] is also
-// reduced and stored.
+// reduced and stored.  The CTA's token rows (at most 8 x K bytes) are staged in
+// shared memory once when they fit, so no warp waits on L2 for activations inside
+// the block loop; otherwise every warp reads them from global memory.
+#include <algorithm>
+
 #include "mx_internal.cuh"
 #include "mx_blockwise.h"
 
@@ -113,6 +117,7 @@ bw_pack_kernel(const T* __restrict__ W, int64_t ldw, int N, int KB, uint32_t tab
     if (lane < 4 * b) dst[lane] = words[warp][lane];
 }
 
+template <bool STAGED>
 __global__ void __launch_bounds__(kGemmWarps * 32)
 bw_gemm_kernel(const uint8_t* __restrict__ codes, const uint32_t* __restrict__ offsets,
                const uint8_t* __restrict__ meta, uint32_t table4, const __half* __restrict__ scales,
@@ -123,17 +128,27 @@ bw_gemm_kernel(const uint8_t* __restrict__ codes, const uint32_t* __restrict__ o
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int n0 = blockIdx.x * kGemmWarps;
     const int rb = n0 / kBR;
+    const int m0 = blockIdx.y * kTok;
+    const int mt = min(kTok, M - m0);
     for (int kb = threadIdx.x; kb < KB; kb += kGemmWarps * 32) {
         const int64_t bi = int64_t(rb) * KB + kb;
         binfo[kb] = __ldg(offsets + bi) | (uint32_t(block_width(meta, bi, table4)) << 28);
     }
+    // [mt][K] token codes after the block infos (16-byte aligned)
+    int8_t* act = reinterpret_cast<int8_t*>(binfo + ((KB + 3) & ~3));
+    if constexpr (STAGED) {
+        const int chunks = K / 16;                        // K is a multiple of 128
+        for (int i = threadIdx.x; i < mt * chunks; i += kGemmWarps * 32) {
+            const int t = i / chunks, c = i % chunks;
+            reinterpret_cast<uint4*>(act + int64_t(t) * K)[c] =
+                __ldg(reinterpret_cast<const uint4*>(Aq + int64_t(m0 + t) * K) + c);
+        }
+    }
     __syncthreads();
     const int n = n0 + warp;
     if (n >= N) return;                                   // the whole warp; no block barrier follows
-    const int m0 = blockIdx.y * kTok;
-    const int mt = min(kTok, M - m0);
     const int r = n % kBR;
-    const int8_t* a_base = Aq + int64_t(m0) * K + lane * 4;
+    const int8_t* a_base = (STAGED ? act : Aq + int64_t(m0) * K) + lane * 4;
     const uint8_t* zrow = zeros + int64_t(n) * KB;
     const __half* srow = scales + int64_t(n) * KB;
     float yacc[kTok];
@@ -180,7 +195,9 @@ bw_gemm_kernel(const uint8_t* __restrict__ codes, const uint32_t* __restrict__ o
 #pragma unroll
             for (int t = 0; t < kTok; ++t) {
                 if (t < mt) {                             // warp-uniform
-                    const int p = __dp4a(d, __ldg(reinterpret_cast<const int*>(a + int64_t(t) * K)), 0);
+                    const int av = STAGED ? *reinterpret_cast<const int*>(a + int64_t(t) * K)
+                                          : __ldg(reinterpret_cast<const int*>(a + int64_t(t) * K));
+                    const int p = __dp4a(d, av, 0);
                     yacc[t] = fmaf(sw, float(p), yacc[t]);
                     if (P != nullptr) {
                         int s = p;
@@ -230,10 +247,25 @@ cudaError_t launch_bw_gemm(const mx_bw_layout& L, const uint8_t* blob, const int
     const uint32_t table4 = uint32_t(L.table[0]) | uint32_t(L.table[1]) << 8 | uint32_t(L.table[2]) << 16 |
                             uint32_t(L.table[3]) << 24;
     const dim3 grid(unsigned((L.N + kGemmWarps - 1) / kGemmWarps), unsigned((M + kTok - 1) / kTok));
-    const size_t smem = size_t(L.KB) * 4;                // the block row's widths and offsets
-    if (smem > 48 * 1024) return cudaErrorInvalidValue;
+    const size_t info = size_t((L.KB + 3) & ~3) * 4;     // the block row's widths and offsets
+    if (info > 48 * 1024) return cudaErrorInvalidValue;
     if ((L.code_bytes >> 4) >= (uint64_t(1) << 28)) return cudaErrorInvalidValue;   // offsets packed in 28 bits
-    bw_gemm_kernel<<<grid, kGemmWarps * 32, smem, s>>>(
+    // the token rows of a CTA (up to kTok) staged when they fit: 96 KB leaves two CTAs per SM
+    const size_t staged = info + size_t(std::min(M, kTok)) * size_t(L.K);
+    const bool stage = staged <= 96 * 1024;
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        if ((e = cudaFuncSetAttribute(bw_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024)) !=
+            cudaSuccess)
+            return e;
+        configured[dev] = true;
+    }
+    auto k = stage ? bw_gemm_kernel<true> : bw_gemm_kernel<false>;
+    k<<<grid, kGemmWarps * 32, stage ? staged : info, s>>>(
         blob + L.off_codes, reinterpret_cast<const uint32_t*>(blob + L.off_offsets), blob + L.off_meta, table4,
         reinterpret_cast<const __half*>(blob + L.off_scales), blob + L.off_zeros, Aq, s_a, M, L.N, L.K, L.KB, Y, ldy,
         P);

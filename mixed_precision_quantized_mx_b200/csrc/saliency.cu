@@ -134,8 +134,12 @@ saliency_kernel(const TW* __restrict__ W, int64_t ldw, const TG* __restrict__ G,
                     // (for |w / s| <= 1024; beyond that both clamp alike); there the exact
                     // quotient decides, as in the packer
                     const float t = __fmul_rn(w[u][e], rc);
-                    float rq = rintf(t);
-                    if (fabsf(t) <= 1024.0f && fabsf(fabsf(t - floorf(t)) - 0.5f) < 4.8828125e-4f)
+                    // nearest integer, ties to even: adding and subtracting 1.5 2^23 rounds
+                    // exactly for |t| < 2^22 (the adds run on the FMA pipe, where a rounding
+                    // instruction would take the conversion unit the fp64 widenings need)
+                    float rq = fabsf(t) < 4194304.0f ? __fsub_rn(__fadd_rn(t, 12582912.0f), 12582912.0f) : rintf(t);
+                    // |t - rq| is 0.5 exactly at a half-integer, as |frac(t) - 0.5| is 0 there
+                    if (fabsf(t) <= 1024.0f && fabsf(fabsf(__fsub_rn(t, rq)) - 0.5f) < 4.8828125e-4f)
                         rq = rintf(__fdiv_rn(w[u][e], sc));
                     const float q = fminf(fmaxf(rq + zf, 0.0f), 15.0f);
                     // (q - z) s is exact in fp32; the difference with w is taken in fp64
