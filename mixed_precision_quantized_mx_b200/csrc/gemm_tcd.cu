@@ -407,11 +407,12 @@ gemm_tcd_kernel(const __grid_constant__ CUtensorMap amap1, const __grid_constant
                     } else {
                         ++gc;                        // the other issuer's group
                     }
-                    // leaving a token chunk: release it (after my MMAs that read it)
+                    // leaving a token chunk: release it (after my MMAs that read it).  Only
+                    // the CTA's last chunk can hold no k-block of mine; no copy waits on its
+                    // release, and an arrival for it could complete the phase of the chunk
+                    // this ring place held before, while the other issuer still reads it
                     if ((ia + 1) % C::kCB == 0 || (last_unit && kb + 1 == un.kb1)) {
-                        uint64_t* be = &S.b_empty[(ia / C::kCB) % C::kBChunks];
-                        if (any) mma_commit(be);
-                        else mbar_arrive(be);
+                        if (any) mma_commit(&S.b_empty[(ia / C::kCB) % C::kBChunks]);
                         any = false;
                     }
                 }
