@@ -161,6 +161,24 @@ def test_gemm_workspace_and_dispatch_on_m(lib):
     assert mx.mx_gemm_select_path(mx.mx_layout_init(14336, 4096, 128, 1434), 1) == mx.PATH_SPLITK
 
 
+@pytest.mark.parametrize("K,N,splits", [
+    # the fastest K split measured on a B200 for each shape at 16, 64 and 128 tokens (path 6,
+    # splits 1..16 swept, 10 % 8-bit rows, group 128): the cost model must pick it
+    (4096, 4096, (4, 4, 4)),        # Llama-3-8B q/o
+    (4096, 14336, (1, 1, 1)),       # 8B up
+    (14336, 4096, (4, 4, 4)),       # 8B down
+    (8192, 28672, (1, 1, 1)),       # 70B up
+    (28672, 8192, (2, 2, 2)),       # 70B down
+])
+def test_decode_split_model_picks_the_measured_fastest_split(lib, K, N, splits):
+    L = mx.mx_layout_init(N, K, 128, int(0.1 * N + 0.5))
+    for M, S in zip((16, 64, 128), splits):
+        assert mx.mx_gemm_select_path(L, M) == mx.PATH_TC_DECODE
+        ws = mx.mx_gemm_workspace_size(L, M)
+        got = ws // (M * N * 4) if ws else 1
+        assert got == S, (K, N, M, got, S)
+
+
 def test_linear_workspace_follows_the_fused_decode_rule(lib):
     L = mx.mx_layout_init(4096, 4096, 128, 410)
     import torch
